@@ -1,0 +1,130 @@
+"""Seeded synthetic inputs for the attention sub-block.
+
+Holds none of the method's arithmetic: only seeded random tensors with the
+shapes, value distributions and structure of the documented workloads.  Every
+tensor is produced on the CPU with its own ``torch.Generator`` (seed, seed+1, ...)
+so that a CPU check and the GPU path see the same bits.
+
+* q, k, v: fp32 N(0, 1) (times an optional scale), rounded to bf16 (round to
+  nearest even, torch's conversion).
+* q/k norm weights: fp32 U(0.5, 1.5).
+* positions: 0 .. T-1 per sequence (int32).
+* decode: per-sequence cache lengths uniform on [len_lo, len_hi]; K and V cache
+  rows N(0, 1) bf16, packed sequence after sequence as [rows, Hkv, D].
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+EPS = 1e-6
+THETA = 1.0e6
+HEAD_DIM = 128
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def _normal_bf16(shape, seed: int, scale: float = 1.0, chunk: int = 1 << 26) -> torch.Tensor:
+    """N(0,1)*scale rounded to bf16, drawn in chunks to bound host memory."""
+    n = int(np.prod(shape)) if len(shape) else 1
+    out = torch.empty(n, dtype=torch.bfloat16)
+    g = _gen(seed)
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        x = torch.randn(e - s, generator=g, dtype=torch.float32)
+        if scale != 1.0:
+            x.mul_(scale)
+        out[s:e] = x.to(torch.bfloat16)
+    return out.view(*shape)
+
+
+def _uniform(shape, seed: int, lo: float, hi: float) -> torch.Tensor:
+    return torch.rand(*shape, generator=_gen(seed), dtype=torch.float32) * (hi - lo) + lo
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    """Raw bf16 bit patterns of a CPU bf16 tensor as a uint16 numpy array."""
+    assert t.dtype == torch.bfloat16
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@dataclass
+class PrefillInputs:
+    q: torch.Tensor      # bf16 [B,T,H,D]
+    k: torch.Tensor      # bf16 [B,T,Hkv,D]
+    v: torch.Tensor      # bf16 [B,T,Hkv,D]
+    pos: torch.Tensor    # int32 [B,T]
+    wq: torch.Tensor     # fp32 [D]
+    wk: torch.Tensor     # fp32 [D]
+    theta: float = THETA
+    eps: float = EPS
+
+
+def prefill_inputs(B: int, T: int, H: int, Hkv: int, D: int = HEAD_DIM, seed: int = 0,
+                   scale: float = 1.0) -> PrefillInputs:
+    q = _normal_bf16((B, T, H, D), seed, scale)
+    k = _normal_bf16((B, T, Hkv, D), seed + 1, scale)
+    v = _normal_bf16((B, T, Hkv, D), seed + 2, scale)
+    wq = _uniform((D,), seed + 3, 0.5, 1.5)
+    wk = _uniform((D,), seed + 4, 0.5, 1.5)
+    pos = torch.arange(T, dtype=torch.int32).repeat(B, 1).contiguous()
+    return PrefillInputs(q, k, v, pos, wq, wk)
+
+
+@dataclass
+class DecodeInputs:
+    q: torch.Tensor        # bf16 [B,H,D]
+    k_cache: torch.Tensor  # bf16 [rows,Hkv,D]
+    v_cache: torch.Tensor  # bf16 [rows,Hkv,D]
+    offsets: torch.Tensor  # int64 [B+1], rows of sequence b: offsets[b] .. offsets[b+1]-1
+    seqlens: torch.Tensor  # int32 [B]
+    wq: torch.Tensor       # fp32 [D]
+    theta: float = THETA
+    eps: float = EPS
+
+    @property
+    def max_len(self) -> int:
+        return int(self.seqlens.max()) if self.seqlens.numel() else 0
+
+
+def decode_inputs(B: int = 64, H: int = 32, Hkv: int = 8, D: int = HEAD_DIM, seed: int = 0,
+                  len_lo: int = 1024, len_hi: int = 32768, seqlens=None) -> DecodeInputs:
+    if seqlens is None:
+        seqlens = torch.randint(len_lo, len_hi + 1, (B,), generator=_gen(seed + 10),
+                                dtype=torch.int64)
+    seqlens = torch.as_tensor(seqlens, dtype=torch.int64).reshape(B)
+    offsets = torch.zeros(B + 1, dtype=torch.int64)
+    offsets[1:] = torch.cumsum(seqlens, 0)
+    rows = int(offsets[-1])
+    q = _normal_bf16((B, H, D), seed)
+    k_cache = _normal_bf16((rows, Hkv, D), seed + 1)
+    v_cache = _normal_bf16((rows, Hkv, D), seed + 2)
+    wq = _uniform((D,), seed + 3, 0.5, 1.5)
+    return DecodeInputs(q, k_cache, v_cache, offsets, seqlens.to(torch.int32), wq)
+
+
+# The documented workloads, by name.
+WORKLOADS = {
+    "prefill_correctness": dict(kind="prefill", B=1, T=128, H=16, Hkv=8),
+    "gqa_sweep_mha": dict(kind="prefill", B=2, T=512, H=16, Hkv=16),
+    "gqa_sweep_hkv8": dict(kind="prefill", B=2, T=512, H=16, Hkv=8),
+    "gqa_sweep_hkv4": dict(kind="prefill", B=2, T=512, H=16, Hkv=4),
+    "gqa_sweep_mqa": dict(kind="prefill", B=2, T=512, H=16, Hkv=1),
+    "large_prefill": dict(kind="prefill", B=4, T=4096, H=32, Hkv=8, scale=0.5),
+    "batched_decode": dict(kind="decode", B=64, H=32, Hkv=8, len_lo=1024, len_hi=32768),
+    "long_context_prefill": dict(kind="prefill", B=1, T=32768, H=64, Hkv=8),
+}
+
+
+def make(name: str, seed: int = 0):
+    w = dict(WORKLOADS[name])
+    kind = w.pop("kind")
+    if kind == "prefill":
+        return prefill_inputs(seed=seed, **w)
+    return decode_inputs(seed=seed, **w)

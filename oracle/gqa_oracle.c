@@ -1,0 +1,329 @@
+/*
+ * gqa_oracle.c -- plain fp64 CPU oracle for the Qwen3 attention sub-block
+ * (per-head q/k RMSNorm -> RoPE -> grouped-query causal softmax(QK^T/sqrt(d) + M) V).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may load, call or link
+ * this file: only the tests, the smoke check and the benchmark's CPU-baseline leg
+ * use it.  It shares no code, header, table or constant with the CUDA library.
+ *
+ * Every step is the plain definition written out in double precision, with no
+ * blocking, fusion or reordering beyond the loops of the definition.  bf16
+ * inputs arrive as their raw 16-bit patterns and are widened to double exactly;
+ * fp32 norm weights are widened exactly; nothing is rounded on the way.
+ *
+ * Sources (pages of the reference, by title and section):
+ *  [A] "Qwen3系列1-理论基础&真实结构" (zhanghao0806.com), D1-2 (stable softmax
+ *      via z - max z), D1-4 (softmax(QK^T/sqrt(d_k) + M) V, row-wise softmax),
+ *      D1-5 (causal mask: position i sees j <= i, -inf before the softmax),
+ *      D2-1 (RMSNorm = gamma * x / sqrt(mean(x^2) + eps)), D2-2 (QK-Norm per
+ *      head on Q and K after projection, then RoPE; V gets neither; one scale
+ *      vector shared by all Q heads and one by all K heads; RoPE matrix R(pos)
+ *      with 2x2 rotation blocks on adjacent pairs), D2-3 (GQA; KV cache holds
+ *      K and V per KV head; decode attends one new token to the cache).
+ *  [B] "深入剖析Qwen3模型架构" (ewbang.com), 3.1.2 (GQA with K/V
+ *      repeat_interleave over query heads; RoPE on (x[::2], x[1::2]) pairs),
+ *      3.4.1 (inv_freq = base^(-2i/dim), base 1e6).
+ *  [C] "Qwen3" (selfknow.cn, nano-vllm walkthrough), "Attention 的 Forward 流程"
+ *      (order: q/k RMSNorm, then rotary embedding, then attention).
+ *  [D] "Qwen3学习日志" (2048ai.net), section 一 (GQA: H query heads in G groups
+ *      of h = H/G sharing one K/V head; G = H is MHA, G = 1 is MQA).
+ *
+ * Readings where the pages are silent or disagree (each also listed in the
+ * design notes): adjacent-pair RoPE; weight multiplies the normalised vector
+ * (not 1 + w) and eps sits inside the square root; the L2-normalize variant
+ * shown once in [B] 3.1.2 is not used; the 1/sqrt(D) scale is applied after
+ * RoPE; query head hq uses KV head hq / (H/Hkv); the causal mask is on the
+ * token index inside the sequence while `pos` only drives RoPE; decode sees
+ * every cached row (cache rows are already normed and rotated K, raw V).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Exact widening of a bf16 bit pattern: the bf16 value is the top half of an
+ * IEEE binary32, so shifting it up 16 bits gives the same number as a float. */
+static double bf16_bits_to_double(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* RMSNorm over one head vector, [A] D2-1: out_d = w_d * x_d / sqrt(mean(x^2) + eps). */
+void oracle_rmsnorm(const double *x, const double *w, double eps, int D, double *out)
+{
+    double ss = 0.0;
+    for (int d = 0; d < D; ++d)
+        ss += x[d] * x[d];
+    double inv_rms = 1.0 / sqrt(ss / (double)D + eps);
+    for (int d = 0; d < D; ++d)
+        out[d] = w[d] * x[d] * inv_rms;
+}
+
+/* RoPE on one head vector, [A] D2-2 (R(pos) block-diagonal with 2x2 rotations on
+ * adjacent pairs) and [B] 3.1.2 / 3.4.1 (pairs x[2i], x[2i+1]; angle pos * theta_i,
+ * theta_i = base^(-2i/D), i = 0 .. D/2-1):
+ *   out[2i]   = x[2i] cos(phi) - x[2i+1] sin(phi)
+ *   out[2i+1] = x[2i] sin(phi) + x[2i+1] cos(phi),   phi = pos * base^(-2i/D). */
+void oracle_rope(const double *x, double pos, double base, int D, double *out)
+{
+    for (int i = 0; i < D / 2; ++i) {
+        double theta_i = pow(base, -2.0 * (double)i / (double)D);
+        double phi = pos * theta_i;
+        double c = cos(phi), s = sin(phi);
+        double a = x[2 * i], b = x[2 * i + 1];
+        out[2 * i] = a * c - b * s;
+        out[2 * i + 1] = a * s + b * c;
+    }
+}
+
+/* q-hat / k-hat of one head vector: RMSNorm, then RoPE ([A] D2-2, [C] forward steps 4-5). */
+static void norm_then_rope(const uint16_t *xbits, const double *w, int32_t pos, double base,
+                           double eps, int D, double *tmp, double *out)
+{
+    for (int d = 0; d < D; ++d)
+        out[d] = bf16_bits_to_double(xbits[d]);
+    oracle_rmsnorm(out, w, eps, D, tmp);
+    oracle_rope(tmp, (double)pos, base, D, out);
+}
+
+/* Apply norm + RoPE to every head vector of x [N, nheads, D] with positions pos [N].
+ * Exposes the oracle's q-hat / k-hat (used by the tests to build a decode cache). */
+void oracle_qk_transform(const uint16_t *x, const int32_t *pos, const float *w, double base,
+                         double eps, int64_t N, int nheads, int D, double *out)
+{
+    double *wd = (double *)malloc(sizeof(double) * D);
+    for (int d = 0; d < D; ++d)
+        wd[d] = (double)w[d];
+#pragma omp parallel
+    {
+        double *tmp = (double *)malloc(sizeof(double) * D);
+#pragma omp for schedule(static)
+        for (int64_t n = 0; n < N; ++n)
+            for (int h = 0; h < nheads; ++h)
+                norm_then_rope(x + (n * nheads + h) * D, wd, pos[n], base, eps, D, tmp,
+                               out + (n * nheads + h) * D);
+        free(tmp);
+    }
+    free(wd);
+}
+
+/* One output row of attention, [A] D1-4 / D1-2: given the scores s_j of the visible
+ * keys (already masked to the visible set), p_j = e^{s_j - max s} / sum_l e^{s_l - max s},
+ * out = sum_j p_j v_j.  v_rows[j] points at key j's value vector. */
+static void softmax_weighted_sum(const double *s, int n, const double *const *v_rows, int D,
+                                 double *p, double *out)
+{
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j)
+        if (s[j] > m)
+            m = s[j];
+    double z = 0.0;
+    for (int j = 0; j < n; ++j) {
+        p[j] = exp(s[j] - m);
+        z += p[j];
+    }
+    for (int j = 0; j < n; ++j)
+        p[j] /= z;
+    for (int d = 0; d < D; ++d)
+        out[d] = 0.0;
+    for (int j = 0; j < n; ++j)
+        for (int d = 0; d < D; ++d)
+            out[d] += p[j] * v_rows[j][d];
+}
+
+/* Grouped-query scaled dot-product attention on already-transformed fp64 tensors.
+ * q [B,T,H,D], k/v [B,T,Hkv,D], out [B,T,H,D].  [D] section 一 and [B] 3.1.2: query
+ * head hq reads KV head hq / (H/Hkv).  causal != 0 applies [A] D1-5 (key j visible to
+ * row i iff j <= i); causal == 0 lets every row see every key.  Scores are
+ * q.k / sqrt(D), [A] D1-4.  If attn_w is not NULL it receives the weights
+ * [B,H,T,T] (zero where masked). */
+void oracle_sdpa_gqa(const double *q, const double *k, const double *v, int B, int T, int H,
+                     int Hkv, int D, int causal, double *out, double *attn_w)
+{
+    int h_per_kv = H / Hkv;
+    double inv_sqrt_d = 1.0 / sqrt((double)D);
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (T > 0 ? T : 1));
+        double *p = (double *)malloc(sizeof(double) * (T > 0 ? T : 1));
+        const double **vr = (const double **)malloc(sizeof(double *) * (T > 0 ? T : 1));
+#pragma omp for collapse(3) schedule(dynamic, 16)
+        for (int b = 0; b < B; ++b)
+            for (int hq = 0; hq < H; ++hq)
+                for (int i = 0; i < T; ++i) {
+                    int g = hq / h_per_kv;
+                    int n = causal ? i + 1 : T;
+                    const double *qi = q + (((int64_t)b * T + i) * H + hq) * D;
+                    for (int j = 0; j < n; ++j) {
+                        const double *kj = k + (((int64_t)b * T + j) * Hkv + g) * D;
+                        double dot = 0.0;
+                        for (int d = 0; d < D; ++d)
+                            dot += qi[d] * kj[d];
+                        s[j] = dot * inv_sqrt_d;
+                        vr[j] = v + (((int64_t)b * T + j) * Hkv + g) * D;
+                    }
+                    softmax_weighted_sum(s, n, vr, D, p, out + (((int64_t)b * T + i) * H + hq) * D);
+                    if (attn_w) {
+                        double *wrow = attn_w + (((int64_t)b * H + hq) * T + i) * T;
+                        for (int j = 0; j < T; ++j)
+                            wrow[j] = j < n ? p[j] : 0.0;
+                    }
+                }
+        free(s);
+        free(p);
+        free(vr);
+    }
+}
+
+/* Prefill: the whole sub-block on bf16 inputs ([C] forward steps 4-6).
+ * q [B,T,H,D], k/v [B,T,Hkv,D] bf16 bits; pos [B,T]; wq/wk [D] fp32; out [B,T,H,D] fp64. */
+void oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *pos,
+                    const float *wq, const float *wk, double base, double eps, int B, int T,
+                    int H, int Hkv, int D, double *out)
+{
+    int64_t ntok = (int64_t)B * T;
+    double *qh = (double *)malloc(sizeof(double) * (size_t)(ntok * H * D + 1));
+    double *kh = (double *)malloc(sizeof(double) * (size_t)(ntok * Hkv * D + 1));
+    double *vd = (double *)malloc(sizeof(double) * (size_t)(ntok * Hkv * D + 1));
+    oracle_qk_transform(q, pos, wq, base, eps, ntok, H, D, qh);
+    oracle_qk_transform(k, pos, wk, base, eps, ntok, Hkv, D, kh);
+    for (int64_t e = 0; e < ntok * Hkv * D; ++e)
+        vd[e] = bf16_bits_to_double(v[e]);
+    oracle_sdpa_gqa(qh, kh, vd, B, T, H, Hkv, D, 1, out, NULL);
+    free(qh);
+    free(kh);
+    free(vd);
+}
+
+/* Prefill for a chosen set of output rows only (for workloads too large to run in
+ * full on a CPU).  rows holds nrows triples (b, hq, i); out is [nrows, D].  Each row
+ * is computed from scratch by the same definition as oracle_prefill: q-hat of row i,
+ * k-hat of keys 0..i of KV head hq / (H/Hkv), causal softmax, weighted sum of V. */
+void oracle_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         const int32_t *pos, const float *wq, const float *wk, double base,
+                         double eps, int B, int T, int H, int Hkv, int D, int64_t nrows,
+                         const int64_t *rows, double *out)
+{
+    (void)B;
+    int h_per_kv = H / Hkv;
+    double inv_sqrt_d = 1.0 / sqrt((double)D);
+    double *wqd = (double *)malloc(sizeof(double) * D);
+    double *wkd = (double *)malloc(sizeof(double) * D);
+    for (int d = 0; d < D; ++d) {
+        wqd[d] = (double)wq[d];
+        wkd[d] = (double)wk[d];
+    }
+#pragma omp parallel
+    {
+        double *tmp = (double *)malloc(sizeof(double) * D);
+        double *qi = (double *)malloc(sizeof(double) * D);
+        double *kj = (double *)malloc(sizeof(double) * D);
+        double *s = (double *)malloc(sizeof(double) * (T > 0 ? T : 1));
+        double *p = (double *)malloc(sizeof(double) * (T > 0 ? T : 1));
+        double *vbuf = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * D);
+        const double **vr = (const double **)malloc(sizeof(double *) * (T > 0 ? T : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t b = rows[3 * r], hq = rows[3 * r + 1], i = rows[3 * r + 2];
+            int64_t g = hq / h_per_kv;
+            norm_then_rope(q + ((b * T + i) * H + hq) * D, wqd, pos[b * T + i], base, eps, D, tmp, qi);
+            for (int64_t j = 0; j <= i; ++j) {
+                norm_then_rope(k + ((b * T + j) * Hkv + g) * D, wkd, pos[b * T + j], base, eps, D, tmp, kj);
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dot += qi[d] * kj[d];
+                s[j] = dot * inv_sqrt_d;
+                const uint16_t *vj = v + ((b * T + j) * Hkv + g) * D;
+                for (int d = 0; d < D; ++d)
+                    vbuf[j * D + d] = bf16_bits_to_double(vj[d]);
+                vr[j] = vbuf + j * D;
+            }
+            softmax_weighted_sum(s, (int)(i + 1), vr, D, p, out + r * D);
+        }
+        free(tmp);
+        free(qi);
+        free(kj);
+        free(s);
+        free(p);
+        free(vbuf);
+        free(vr);
+    }
+    free(wqd);
+    free(wkd);
+}
+
+/* Decode: one new query token per sequence against its KV cache ([A] D2-3: prefill
+ * writes K/V to the cache, decode feeds one token and reads the cache).
+ * q [B,H,D] bf16 bits (raw: normed and rotated here at position qpos[b], or at
+ * position seqlens[b] when qpos is NULL); k_cache/v_cache [rows,Hkv,D] bf16 bits,
+ * sequence b owning rows offsets[b] .. offsets[b]+seqlens[b]-1, which are used as
+ * already-normed, already-rotated K and raw V; all of them are visible (the cache
+ * holds only earlier positions).  out [B,H,D] fp64. */
+void oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                   const int64_t *offsets, const int32_t *seqlens, const int32_t *qpos,
+                   const float *wq, double base, double eps, int B, int H, int Hkv, int D,
+                   double *out)
+{
+    int h_per_kv = H / Hkv;
+    double inv_sqrt_d = 1.0 / sqrt((double)D);
+    int32_t maxlen = 1;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] > maxlen)
+            maxlen = seqlens[b];
+    double *wqd = (double *)malloc(sizeof(double) * D);
+    for (int d = 0; d < D; ++d)
+        wqd[d] = (double)wq[d];
+#pragma omp parallel
+    {
+        double *tmp = (double *)malloc(sizeof(double) * D);
+        double *qi = (double *)malloc(sizeof(double) * D);
+        double *s = (double *)malloc(sizeof(double) * maxlen);
+        double *p = (double *)malloc(sizeof(double) * maxlen);
+        double *vbuf = (double *)malloc(sizeof(double) * (size_t)maxlen * D);
+        const double **vr = (const double **)malloc(sizeof(double *) * maxlen);
+#pragma omp for collapse(2) schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b)
+            for (int hq = 0; hq < H; ++hq) {
+                int g = hq / h_per_kv;
+                int32_t len = seqlens[b];
+                int32_t position = qpos ? qpos[b] : len;
+                norm_then_rope(q + ((int64_t)b * H + hq) * D, wqd, position, base, eps, D, tmp, qi);
+                for (int32_t j = 0; j < len; ++j) {
+                    int64_t row = offsets[b] + j;
+                    const uint16_t *kj = k_cache + (row * Hkv + g) * D;
+                    const uint16_t *vj = v_cache + (row * Hkv + g) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d)
+                        dot += qi[d] * bf16_bits_to_double(kj[d]);
+                    s[j] = dot * inv_sqrt_d;
+                    for (int d = 0; d < D; ++d)
+                        vbuf[(int64_t)j * D + d] = bf16_bits_to_double(vj[d]);
+                    vr[j] = vbuf + (int64_t)j * D;
+                }
+                softmax_weighted_sum(s, len, vr, D, p, out + ((int64_t)b * H + hq) * D);
+            }
+        free(tmp);
+        free(qi);
+        free(s);
+        free(p);
+        free(vbuf);
+        free(vr);
+    }
+    free(wqd);
+}
+
+/* Number of threads the OpenMP runtime will use (reported beside the CPU timing). */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,169 @@
+"""ctypes front end of the fp64 CPU oracle (``gqa_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU
+baseline leg are the only callers.  The product path (the CUDA library and its
+Python binding) never imports this module, and this module never imports the
+product path.
+
+Inputs are numpy arrays: bf16 tensors travel as their raw ``uint16`` bit
+patterns, positions as ``int32``, norm weights as ``float32``; every output is
+``float64``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gqa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``gqa_oracle.c`` into ``liboracle.so`` beside it (gcc, OpenMP)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c11", "-Wall",
+           "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I, L, Dd = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+            lib.oracle_rmsnorm.argtypes = [P, P, Dd, I, P]
+            lib.oracle_rope.argtypes = [P, Dd, Dd, I, P]
+            lib.oracle_qk_transform.argtypes = [P, P, P, Dd, Dd, L, I, I, P]
+            lib.oracle_sdpa_gqa.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
+            lib.oracle_prefill.argtypes = [P, P, P, P, P, P, Dd, Dd, I, I, I, I, I, P]
+            lib.oracle_prefill_rows.argtypes = [P, P, P, P, P, P, Dd, Dd, I, I, I, I, I,
+                                                L, P, P]
+            lib.oracle_decode.argtypes = [P, P, P, P, P, P, P, Dd, Dd, I, I, I, I, P]
+            lib.oracle_num_threads.restype = I
+            _lib = lib
+    return _lib
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0) if a is None else ctypes.c_void_p(a.ctypes.data)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def rmsnorm(x, w, eps: float) -> np.ndarray:
+    x = _c(x, np.float64)
+    w = _c(w, np.float64)
+    out = np.empty_like(x)
+    _load().oracle_rmsnorm(_p(x), _p(w), eps, x.shape[-1], _p(out))
+    return out
+
+
+def rope(x, pos: float, theta: float) -> np.ndarray:
+    x = _c(x, np.float64)
+    out = np.empty_like(x)
+    _load().oracle_rope(_p(x), float(pos), float(theta), x.shape[-1], _p(out))
+    return out
+
+
+def qk_transform(x_bits, pos, w, theta: float, eps: float) -> np.ndarray:
+    """x_bits [N, nheads, D] uint16 (bf16 bits), pos [N] -> fp64 [N, nheads, D]."""
+    x_bits = _c(x_bits, np.uint16)
+    N, nh, D = x_bits.shape
+    pos = _c(pos, np.int32).reshape(N)
+    w = _c(w, np.float32)
+    out = np.empty((N, nh, D), np.float64)
+    _load().oracle_qk_transform(_p(x_bits), _p(pos), _p(w), theta, eps, N, nh, D, _p(out))
+    return out
+
+
+def sdpa_gqa(q, k, v, causal: bool = True, return_weights: bool = False):
+    """fp64 q [B,T,H,D], k/v [B,T,Hkv,D] (already normed and rotated)."""
+    q = _c(q, np.float64)
+    k = _c(k, np.float64)
+    v = _c(v, np.float64)
+    B, T, H, D = q.shape
+    Hkv = k.shape[2]
+    assert H % Hkv == 0
+    out = np.empty((B, T, H, D), np.float64)
+    w = np.empty((B, H, T, T), np.float64) if return_weights else None
+    _load().oracle_sdpa_gqa(_p(q), _p(k), _p(v), B, T, H, Hkv, D, int(bool(causal)),
+                            _p(out), _p(w))
+    return (out, w) if return_weights else out
+
+
+def prefill(q_bits, k_bits, v_bits, pos, wq, wk, theta: float, eps: float) -> np.ndarray:
+    """Whole prefill sub-block: bf16 bits q [B,T,H,D], k/v [B,T,Hkv,D]; pos [B,T]."""
+    q_bits = _c(q_bits, np.uint16)
+    k_bits = _c(k_bits, np.uint16)
+    v_bits = _c(v_bits, np.uint16)
+    B, T, H, D = q_bits.shape
+    Hkv = k_bits.shape[2]
+    assert H % Hkv == 0
+    pos = _c(pos, np.int32).reshape(B, T)
+    wq = _c(wq, np.float32)
+    wk = _c(wk, np.float32)
+    out = np.empty((B, T, H, D), np.float64)
+    _load().oracle_prefill(_p(q_bits), _p(k_bits), _p(v_bits), _p(pos), _p(wq), _p(wk),
+                           theta, eps, B, T, H, Hkv, D, _p(out))
+    return out
+
+
+def prefill_rows(q_bits, k_bits, v_bits, pos, wq, wk, theta: float, eps: float,
+                 rows) -> np.ndarray:
+    """Selected output rows of prefill; rows is an int array [n, 3] of (b, hq, i)."""
+    q_bits = _c(q_bits, np.uint16)
+    k_bits = _c(k_bits, np.uint16)
+    v_bits = _c(v_bits, np.uint16)
+    B, T, H, D = q_bits.shape
+    Hkv = k_bits.shape[2]
+    pos = _c(pos, np.int32).reshape(B, T)
+    wq = _c(wq, np.float32)
+    wk = _c(wk, np.float32)
+    rows = _c(rows, np.int64).reshape(-1, 3)
+    assert (rows[:, 0] < B).all() and (rows[:, 1] < H).all() and (rows[:, 2] < T).all()
+    out = np.empty((rows.shape[0], D), np.float64)
+    _load().oracle_prefill_rows(_p(q_bits), _p(k_bits), _p(v_bits), _p(pos), _p(wq),
+                                _p(wk), theta, eps, B, T, H, Hkv, D, rows.shape[0],
+                                _p(rows), _p(out))
+    return out
+
+
+def decode(q_bits, k_cache_bits, v_cache_bits, offsets, seqlens, qpos, wq, theta: float,
+           eps: float) -> np.ndarray:
+    """Decode: q [B,H,D] bf16 bits; caches [rows,Hkv,D] bf16 bits; offsets [B(+1)] int64;
+    seqlens [B] int32 (>= 1); qpos [B] int32 or None (then qpos = seqlens)."""
+    q_bits = _c(q_bits, np.uint16)
+    k_cache_bits = _c(k_cache_bits, np.uint16)
+    v_cache_bits = _c(v_cache_bits, np.uint16)
+    B, H, D = q_bits.shape
+    Hkv = k_cache_bits.shape[1]
+    offsets = _c(offsets, np.int64)
+    seqlens = _c(seqlens, np.int32)
+    assert (seqlens >= 1).all()
+    qpos_a = None if qpos is None else _c(qpos, np.int32)
+    wq = _c(wq, np.float32)
+    out = np.empty((B, H, D), np.float64)
+    _load().oracle_decode(_p(q_bits), _p(k_cache_bits), _p(v_cache_bits), _p(offsets),
+                          _p(seqlens), _p(qpos_a), _p(wq), theta, eps, B, H, Hkv, D,
+                          _p(out))
+    return out

@@ -1,0 +1,385 @@
+"""Pins of the fp64 CPU oracle to things other than itself.
+
+Each test ties one part of the oracle to what the pages and the mathematics fix:
+worked examples with closed-form answers, invariants, degenerate cases that reduce
+to a library routine (torch fp64 on the CPU), and brute force on tiny inputs.
+Together they are chosen so that a plausible slip anywhere in the oracle (a dropped
+term, a wrong sign or index, a transposed operand, the wrong softmax axis, the
+wrong RoPE pairing or frequency) fails at least one of them.
+
+Sources: "Qwen3系列1-理论基础&真实结构" D1-2, D1-4, D1-5, D2-1, D2-2, D2-3;
+"深入剖析Qwen3模型架构" 3.1.2, 3.4.1; "Qwen3学习日志" section 一;
+"Qwen3" (nano-vllm walkthrough) "Attention 的 Forward 流程".
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle
+from grouped_query_causal_b200 import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+def _read_golden(name):
+    rows = {}
+    with open(os.path.join(GOLDEN, name), encoding="utf-8") as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, rest = line.split(None, 1)
+            if ";" in rest:
+                rows[key] = np.array([[float(t) for t in r.split()] for r in rest.split(";")])
+            else:
+                rows[key] = np.array([float(t) for t in rest.split()])
+    return rows
+
+
+# --------------------------------------------------------------------------------------
+# Worked examples (closed forms)
+# --------------------------------------------------------------------------------------
+
+def test_sdpa_worked_example_3_tokens_dim_2():
+    """D1-4 / D1-5 pen-and-paper task: scores / sqrt(2), causal mask, row softmax, P V."""
+    g = _read_golden("sdpa_3tok_d2.txt")
+    Q, K, V = g["Q"], g["K"], g["V"]
+    out, w = oracle.sdpa_gqa(Q[None, :, None, :], K[None, :, None, :], V[None, :, None, :],
+                             causal=True, return_weights=True)
+    out = out[0, :, 0, :]
+    w = w[0, 0]
+    a = math.exp(1.0 / math.sqrt(2.0))
+    # row 0 sees only key 0 (score 1/sqrt 2): weight 1
+    w0 = np.array([1.0, 0.0, 0.0])
+    # row 1: scores (0, 1/sqrt 2) -> (1, a) / (1 + a)
+    w1 = np.array([1.0, a, 0.0]) / (1.0 + a)
+    # row 2: scores (1/sqrt 2, 1/sqrt 2, 2/sqrt 2) -> (a, a, a^2) / (2a + a^2) = (1, 1, a) / (2 + a)
+    w2 = np.array([1.0, 1.0, a]) / (2.0 + a)
+    W = np.stack([w0, w1, w2])
+    np.testing.assert_allclose(w, W, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(out, W @ V, rtol=0, atol=1e-14)
+    # the numbers the closed forms give, to 6 places, for a reader checking by hand
+    np.testing.assert_allclose(out[1], [2.339524, 3.339524], atol=1e-6)
+    np.testing.assert_allclose(out[2], [3.510470, 4.510470], atol=1e-6)
+
+
+def test_rmsnorm_then_rope_worked_example_2d():
+    """D2-1 formula and D2-2 pen-and-paper task (RMSNorm of a 2-D query, RoPE, dot)."""
+    g = _read_golden("rmsnorm_rope_2d.txt")
+    x, w, eps, pos, key = g["x"], g["w"], float(g["eps"][0]), float(g["pos"][0]), g["key"]
+    normed = oracle.rmsnorm(x, w, eps)
+    # mean(x^2) + eps = (9 + 16)/2 + 3.5 = 16 -> divide by 4 exactly
+    np.testing.assert_allclose(normed, x / 4.0, rtol=0, atol=1e-15)
+    rotated = oracle.rope(normed, pos, 1.0e6)
+    # counter-clockwise quarter turn, R = [[cos, -sin], [sin, cos]]: (a, b) -> (-b, a)
+    np.testing.assert_allclose(rotated, [-normed[1], normed[0]], rtol=0, atol=1e-15)
+    assert abs(float(rotated @ key) - (-1.0 * 2 + 0.75 * -1)) < 1e-15
+
+
+def test_rmsnorm_weight_multiplies_and_eps_inside_root():
+    x = np.array([3.0, 4.0])
+    np.testing.assert_allclose(oracle.rmsnorm(x, [2.0, 0.5], 0.0), [6 / math.sqrt(12.5), 2 / math.sqrt(12.5)],
+                               rtol=1e-15)
+    # mean, not sum, of squares: D = 4 with two zeros -> mean = 25/4
+    x4 = np.array([3.0, 0.0, 4.0, 0.0])
+    np.testing.assert_allclose(oracle.rmsnorm(x4, np.ones(4), 0.0), x4 / 2.5, rtol=1e-15)
+
+
+def test_rope_adjacent_pairs_and_frequency():
+    """Pairs are (x[2i], x[2i+1]) ("深入剖析Qwen3模型架构" 3.1.2, D2-2 R(pos)); the angle of
+    pair i is pos * base^(-2i/D) (3.4.1)."""
+    base = 1.0e6
+    D = 4
+    # pair 0 has frequency 1: pos = pi/2 turns e0 into e1 (adjacent), not into e2 (half split)
+    np.testing.assert_allclose(oracle.rope([1.0, 0, 0, 0], math.pi / 2, base), [0, 1.0, 0, 0], atol=1e-15)
+    # pair 1 has frequency base^(-2/4) = 1e-3: pos = 500 pi is a quarter turn of (x2, x3)
+    np.testing.assert_allclose(oracle.rope([0, 0, 1.0, 0], 500 * math.pi, base), [0, 0, 0, 1.0], atol=1e-12)
+    # pos 0 is the identity
+    r = np.random.default_rng(0).standard_normal(128)
+    np.testing.assert_array_equal(oracle.rope(r, 0.0, base), r)
+    # with D = 128 the last pair has frequency base^(-126/128)
+    D = 128
+    x = np.zeros(D)
+    x[D - 2] = 1.0
+    pos = (math.pi / 2) / base ** (-(D - 2) / D)
+    y = oracle.rope(x, pos, base)
+    assert abs(y[D - 1] - 1.0) < 1e-9 and abs(y[D - 2]) < 1e-9
+
+
+def test_rope_preserves_norm_and_depends_on_relative_position():
+    """D2-2: rotation keeps the norm; q_m . k_n after RoPE depends only on m - n."""
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal(128)
+    k = rng.standard_normal(128)
+    for pos in [0, 1, 7, 127, 4095, 32767]:
+        assert abs(np.linalg.norm(oracle.rope(q, pos, 1e6)) - np.linalg.norm(q)) < 1e-12
+    for m, n in [(5, 3), (100, 0), (4000, 3999), (32767, 1)]:
+        ref = oracle.rope(q, m, 1e6) @ oracle.rope(k, n, 1e6)
+        for s in [1, 17, 1000, 20000]:
+            got = oracle.rope(q, m + s, 1e6) @ oracle.rope(k, n + s, 1e6)
+            assert abs(got - ref) < 1e-9 * max(1.0, abs(ref))
+
+
+# --------------------------------------------------------------------------------------
+# Softmax and mask invariants (D1-2, D1-4, D1-5)
+# --------------------------------------------------------------------------------------
+
+def test_softmax_rows_sum_to_one_and_masked_weights_are_zero():
+    rng = np.random.default_rng(2)
+    B, T, H, Hkv, D = 2, 9, 4, 2, 16
+    q = rng.standard_normal((B, T, H, D)) * 3
+    k = rng.standard_normal((B, T, Hkv, D)) * 3
+    v = rng.standard_normal((B, T, Hkv, D))
+    _, w = oracle.sdpa_gqa(q, k, v, causal=True, return_weights=True)
+    np.testing.assert_allclose(w.sum(-1), 1.0, rtol=0, atol=1e-12)
+    upper = np.triu(np.ones((T, T), bool), 1)
+    assert (w[..., upper] == 0.0).all()
+    assert (w[..., ~upper] > 0.0).all()
+    # V = one-hot rows: the output row is exactly the weight row (V is not transposed)
+    T2, D2 = 6, 8
+    q2 = rng.standard_normal((1, T2, 1, D2))
+    k2 = rng.standard_normal((1, T2, 1, D2))
+    v2 = np.eye(D2)[:T2][None, :, None, :]
+    out2, w2 = oracle.sdpa_gqa(q2, k2, v2, causal=True, return_weights=True)
+    np.testing.assert_allclose(out2[0, :, 0, :T2], w2[0, 0], atol=1e-15)
+    # all-ones V -> output 1 everywhere
+    out3 = oracle.sdpa_gqa(q, k, np.ones_like(v), causal=True)
+    np.testing.assert_allclose(out3, 1.0, atol=1e-14)
+
+
+def test_output_is_linear_in_v():
+    rng = np.random.default_rng(3)
+    B, T, H, Hkv, D = 1, 7, 4, 2, 8
+    q = rng.standard_normal((B, T, H, D))
+    k = rng.standard_normal((B, T, Hkv, D))
+    v1 = rng.standard_normal((B, T, Hkv, D))
+    v2 = rng.standard_normal((B, T, Hkv, D))
+    lhs = oracle.sdpa_gqa(q, k, 2.0 * v1 - 0.5 * v2)
+    rhs = 2.0 * oracle.sdpa_gqa(q, k, v1) - 0.5 * oracle.sdpa_gqa(q, k, v2)
+    np.testing.assert_allclose(lhs, rhs, atol=1e-13)
+
+
+# --------------------------------------------------------------------------------------
+# GQA structure ("Qwen3学习日志" section 一; "深入剖析Qwen3模型架构" 3.1.2)
+# --------------------------------------------------------------------------------------
+
+def _torch_sdpa_repeat_interleave(q, k, v, causal=True):
+    """torch fp64 on the CPU with K/V repeat_interleave'd to every query head (the
+    structure of the GQA snippet in 3.1.2), a library routine independent of the oracle."""
+    qt = torch.from_numpy(q).permute(0, 2, 1, 3)           # [B,H,T,D]
+    kt = torch.from_numpy(k).permute(0, 2, 1, 3)           # [B,Hkv,T,D]
+    vt = torch.from_numpy(v).permute(0, 2, 1, 3)
+    rep = q.shape[2] // k.shape[2]
+    kt = kt.repeat_interleave(rep, dim=1)
+    vt = vt.repeat_interleave(rep, dim=1)
+    scores = torch.matmul(qt, kt.transpose(-2, -1)) / math.sqrt(q.shape[-1])
+    if causal:
+        T = q.shape[1]
+        mask = torch.triu(torch.ones(T, T, dtype=torch.bool), 1)
+        scores = scores.masked_fill(mask, float("-inf"))
+    out = torch.matmul(torch.softmax(scores, dim=-1), vt)
+    return out.permute(0, 2, 1, 3).numpy()
+
+
+@pytest.mark.parametrize("H,Hkv", [(16, 16), (16, 8), (16, 4), (16, 1), (6, 2), (3, 1)])
+def test_group_map_matches_torch_repeat_interleave(H, Hkv):
+    rng = np.random.default_rng(4 + H + Hkv)
+    B, T, D = 2, 13, 16
+    q = rng.standard_normal((B, T, H, D))
+    k = rng.standard_normal((B, T, Hkv, D))
+    v = rng.standard_normal((B, T, Hkv, D))
+    np.testing.assert_allclose(oracle.sdpa_gqa(q, k, v), _torch_sdpa_repeat_interleave(q, k, v),
+                               rtol=0, atol=1e-12)
+
+
+def test_explicit_repetition_equals_grouped_indexing_bit_for_bit():
+    rng = np.random.default_rng(5)
+    B, T, H, Hkv, D = 1, 11, 8, 2, 16
+    q = rng.standard_normal((B, T, H, D))
+    k = rng.standard_normal((B, T, Hkv, D))
+    v = rng.standard_normal((B, T, Hkv, D))
+    rep = H // Hkv
+    grouped = oracle.sdpa_gqa(q, k, v)
+    repeated = oracle.sdpa_gqa(q, np.repeat(k, rep, axis=2), np.repeat(v, rep, axis=2))
+    np.testing.assert_array_equal(grouped, repeated)
+
+
+def test_mha_and_mqa_degeneracies():
+    """G = H is MHA (each head alone); G = 1 is MQA (every head on one shared K/V)."""
+    rng = np.random.default_rng(6)
+    B, T, H, D = 1, 10, 4, 8
+    q = rng.standard_normal((B, T, H, D))
+    k = rng.standard_normal((B, T, H, D))
+    v = rng.standard_normal((B, T, H, D))
+    mha = oracle.sdpa_gqa(q, k, v)
+    for h in range(H):
+        alone = oracle.sdpa_gqa(q[:, :, h:h + 1], k[:, :, h:h + 1], v[:, :, h:h + 1])
+        np.testing.assert_array_equal(mha[:, :, h:h + 1], alone)
+    mqa = oracle.sdpa_gqa(q, k[:, :, :1], v[:, :, :1])
+    for h in range(H):
+        alone = oracle.sdpa_gqa(q[:, :, h:h + 1], k[:, :, :1], v[:, :, :1])
+        np.testing.assert_array_equal(mqa[:, :, h:h + 1], alone)
+
+
+# --------------------------------------------------------------------------------------
+# The whole sub-block on bf16 inputs
+# --------------------------------------------------------------------------------------
+
+def _torch_prefill_fp64(inp: synthetic.PrefillInputs):
+    """The sub-block in torch fp64 following the pages' PyTorch structure: RMSNorm per
+    head ("Qwen3系列1" D2-1/D2-2), RoPE on (x[..., ::2], x[..., 1::2]) with
+    inv_freq = base^(-arange(0, D, 2)/D) (3.1.2 / 3.4.1), repeat_interleave GQA (3.1.2)."""
+    q = inp.q.double()
+    k = inp.k.double()
+    v = inp.v.double()
+    D = q.shape[-1]
+
+    def rms(x, w):
+        return w.double() * x / torch.sqrt(x.pow(2).mean(-1, keepdim=True) + inp.eps)
+
+    inv_freq = 1.0 / (inp.theta ** (torch.arange(0, D, 2, dtype=torch.float64) / D))
+    ang = inp.pos.double()[..., None] * inv_freq            # [B,T,D/2]
+    cos = torch.cos(ang)[:, :, None, :]
+    sin = torch.sin(ang)[:, :, None, :]
+
+    def rope(x):
+        xr, xi = x[..., ::2], x[..., 1::2]
+        return torch.stack([xr * cos - xi * sin, xr * sin + xi * cos], dim=-1).flatten(-2)
+
+    qh = rope(rms(q, inp.wq))
+    kh = rope(rms(k, inp.wk))
+    return _torch_sdpa_repeat_interleave(qh.numpy(), kh.numpy(), v.numpy())
+
+
+def _bits(t):
+    return synthetic.bf16_bits(t)
+
+
+@pytest.mark.parametrize("B,T,H,Hkv", [(1, 128, 16, 8), (2, 37, 6, 3), (1, 5, 2, 1)])
+def test_prefill_matches_torch_fp64_pipeline(B, T, H, Hkv):
+    inp = synthetic.prefill_inputs(B, T, H, Hkv, seed=11)
+    got = oracle.prefill(_bits(inp.q), _bits(inp.k), _bits(inp.v), inp.pos.numpy(), inp.wq.numpy(),
+                         inp.wk.numpy(), inp.theta, inp.eps)
+    np.testing.assert_allclose(got, _torch_prefill_fp64(inp), rtol=0, atol=1e-11)
+
+
+def test_prefill_rows_match_full_prefill():
+    inp = synthetic.prefill_inputs(2, 40, 4, 2, seed=12)
+    args = (_bits(inp.q), _bits(inp.k), _bits(inp.v), inp.pos.numpy(), inp.wq.numpy(), inp.wk.numpy(),
+            inp.theta, inp.eps)
+    full = oracle.prefill(*args)
+    rows = np.array([(b, h, i) for b in range(2) for h in range(4) for i in range(40)])
+    got = oracle.prefill_rows(*args, rows)
+    np.testing.assert_allclose(got, full[rows[:, 0], rows[:, 2], rows[:, 1]], rtol=0, atol=1e-13)
+
+
+def test_norm_scale_invariance():
+    """RMSNorm removes a positive scale of q or k (eps = 0): scaling the bf16 inputs
+    by 2 (exact in bf16) leaves the output unchanged."""
+    inp = synthetic.prefill_inputs(1, 24, 4, 2, seed=13)
+    args = dict(pos=inp.pos.numpy(), wq=inp.wq.numpy(), wk=inp.wk.numpy(), theta=inp.theta, eps=0.0)
+    a = oracle.prefill(_bits(inp.q), _bits(inp.k), _bits(inp.v), **args)
+    b = oracle.prefill(_bits(inp.q * 2), _bits(inp.k * 4), _bits(inp.v), **args)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def _bruteforce_prefill(qb, kb, vb, pos, wq, wk, theta, eps):
+    """Pure-Python loops on tiny inputs: widen bits, RMSNorm, rotate pairs, causal softmax."""
+    def widen(bits):
+        return float(np.array([int(bits) << 16], np.uint32).view(np.float32)[0])
+
+    B, T, H, D = qb.shape
+    Hkv = kb.shape[2]
+    rep = H // Hkv
+
+    def transform(vec_bits, w, p):
+        x = [widen(t) for t in vec_bits]
+        r = math.sqrt(sum(t * t for t in x) / D + eps)
+        y = [float(w[d]) * x[d] / r for d in range(D)]
+        z = list(y)
+        for i in range(D // 2):
+            ang = p * theta ** (-2.0 * i / D)
+            c, s = math.cos(ang), math.sin(ang)
+            z[2 * i] = y[2 * i] * c - y[2 * i + 1] * s
+            z[2 * i + 1] = y[2 * i] * s + y[2 * i + 1] * c
+        return z
+
+    out = np.zeros((B, T, H, D))
+    for b in range(B):
+        for hq in range(H):
+            g = hq // rep
+            for i in range(T):
+                qi = transform(qb[b, i, hq], wq, int(pos[b, i]))
+                s = []
+                for j in range(i + 1):
+                    kj = transform(kb[b, j, g], wk, int(pos[b, j]))
+                    s.append(sum(qi[d] * kj[d] for d in range(D)) / math.sqrt(D))
+                m = max(s)
+                e = [math.exp(t - m) for t in s]
+                z = sum(e)
+                for d in range(D):
+                    out[b, i, hq, d] = sum(e[j] / z * widen(vb[b, j, g, d]) for j in range(i + 1))
+    return out
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,D", [(1, 3, 2, 1, 2), (2, 5, 4, 2, 4), (1, 6, 3, 3, 8), (1, 4, 4, 1, 8)])
+def test_prefill_bruteforce_tiny(B, T, H, Hkv, D):
+    inp = synthetic.prefill_inputs(B, T, H, Hkv, D=D, seed=14)
+    args = (_bits(inp.q), _bits(inp.k), _bits(inp.v), inp.pos.numpy(), inp.wq.numpy(), inp.wk.numpy(),
+            1.0e4, 1e-6)
+    np.testing.assert_allclose(oracle.prefill(*args), _bruteforce_prefill(*args), rtol=0, atol=1e-12)
+
+
+def test_decode_equals_the_last_row_of_prefill():
+    """Decode attends the new token (at position L) to cache rows 0..L; with the cache
+    holding k-hat (normed, rotated K) and raw V it must equal row L of the causal
+    computation ("Qwen3系列1" D2-3: K/V are written to the cache before attention)."""
+    B, L, H, Hkv, D = 3, 20, 8, 2, 32
+    inp = synthetic.prefill_inputs(B, L + 1, H, Hkv, D=D, seed=15)
+    ntok = B * (L + 1)
+    kh = oracle.qk_transform(_bits(inp.k).reshape(ntok, Hkv, D), inp.pos.numpy().reshape(ntok),
+                             inp.wk.numpy(), inp.theta, inp.eps)
+    kh_bf16 = torch.from_numpy(kh).to(torch.bfloat16)       # the cache stores bf16
+    qh = oracle.qk_transform(_bits(inp.q).reshape(ntok, H, D), inp.pos.numpy().reshape(ntok),
+                             inp.wq.numpy(), inp.theta, inp.eps)
+    ref = oracle.sdpa_gqa(qh.reshape(B, L + 1, H, D), kh_bf16.double().numpy().reshape(B, L + 1, Hkv, D),
+                          inp.v.double().numpy())[:, L]
+    offsets = np.arange(B + 1, dtype=np.int64) * (L + 1)
+    seqlens = np.full(B, L + 1, np.int32)
+    qdec = _bits(inp.q)[:, L]                                # raw query of the last token
+    got = oracle.decode(qdec, _bits(kh_bf16).reshape(ntok, Hkv, D), _bits(inp.v).reshape(ntok, Hkv, D),
+                        offsets, seqlens, np.full(B, L, np.int32), inp.wq.numpy(), inp.theta, inp.eps)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    # qpos omitted -> the query sits at position len: here len = L + 1
+    got2 = oracle.decode(qdec, _bits(kh_bf16).reshape(ntok, Hkv, D), _bits(inp.v).reshape(ntok, Hkv, D),
+                         offsets, seqlens, None, inp.wq.numpy(), inp.theta, inp.eps)
+    got3 = oracle.decode(qdec, _bits(kh_bf16).reshape(ntok, Hkv, D), _bits(inp.v).reshape(ntok, Hkv, D),
+                         offsets, seqlens, np.full(B, L + 1, np.int32), inp.wq.numpy(), inp.theta, inp.eps)
+    np.testing.assert_array_equal(got2, got3)
+
+
+def test_decode_matches_torch_fp64_on_ragged_cache():
+    rng = np.random.default_rng(16)
+    B, H, Hkv, D = 4, 8, 2, 16
+    seqlens = np.array([1, 5, 17, 3], np.int32)
+    inp = synthetic.decode_inputs(B, H, Hkv, D, seed=16, seqlens=seqlens)
+    qpos = rng.integers(0, 1000, B).astype(np.int32)
+    got = oracle.decode(_bits(inp.q), _bits(inp.k_cache), _bits(inp.v_cache), inp.offsets.numpy(),
+                        inp.seqlens.numpy(), qpos, inp.wq.numpy(), inp.theta, inp.eps)
+    q = inp.q.double()
+    qn = inp.wq.double() * q / torch.sqrt(q.pow(2).mean(-1, keepdim=True) + inp.eps)
+    inv_freq = 1.0 / (inp.theta ** (torch.arange(0, D, 2, dtype=torch.float64) / D))
+    ang = torch.from_numpy(qpos).double()[:, None, None] * inv_freq
+    c, s = torch.cos(ang), torch.sin(ang)
+    qh = torch.stack([qn[..., ::2] * c - qn[..., 1::2] * s, qn[..., ::2] * s + qn[..., 1::2] * c], -1).flatten(-2)
+    for b in range(B):
+        o0, n = int(inp.offsets[b]), int(seqlens[b])
+        kc = inp.k_cache[o0:o0 + n].double().permute(1, 0, 2).repeat_interleave(H // Hkv, 0)   # [H,n,D]
+        vc = inp.v_cache[o0:o0 + n].double().permute(1, 0, 2).repeat_interleave(H // Hkv, 0)
+        p = torch.softmax((kc @ qh[b][:, :, None])[..., 0] / math.sqrt(D), -1)                # [H,n]
+        ref = (p[:, :, None] * vc).sum(1)
+        np.testing.assert_allclose(got[b], ref.numpy(), rtol=0, atol=1e-12)
