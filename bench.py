@@ -1,0 +1,485 @@
+"""Benchmark of the attention sub-block on B200: prefill attention TFLOP/s and decode
+KV-read GB/s, each against its roofline.
+
+One step = one pass of the whole hot path over one batch of synthetic inputs:
+  * prefill, large workload (B=4, T=4096, H=32, Hkv=8, D=128, inputs x0.5):
+    k-hat prologue (RMSNorm + RoPE of K) then the fused q-prologue + causal GQA
+    attention kernel;
+  * decode, batched workload (64 sequences, cache lengths U[1024, 32768], H=32,
+    Hkv=8, D=128): split-KV kernel then the log-sum-exp merge.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs the same step on its own GPU (independent
+replicas: weak scaling, no collective on the data path); the time is the max over
+ranks and the value counts the work of all ranks.  `--impl reference` times the
+fp64 CPU oracle on bounded samples of the same workloads on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from grouped_query_causal_b200 import synthetic  # noqa: E402
+
+METRIC = "prefill attn TFLOPS and decode KV-read GB/s on 1 B200, % of roofline"
+PREFILL = "large_prefill"
+DECODE = "batched_decode"
+KERNEL_SOURCES = ["prefill.cuh", "decode.cuh", "ptx.cuh", "rope.cuh", "gqa_attn.cu"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- workload sizes
+def prefill_flops(B, T, H, D=128):
+    """Algorithmic FLOPs of causal attention: QK^T and PV over the visible (i, j <= i)
+    pairs only, 2*D each: B*H*T(T+1)/2 pairs * 4D."""
+    return B * H * 2 * D * T * (T + 1)
+
+
+def decode_bytes(seqlens, H, Hkv, D=128):
+    """Algorithmic bytes of decode: every cached K and V row read once (bf16), plus the
+    bf16 query and the fp32 output."""
+    B = len(seqlens)
+    return int(sum(int(s) for s in seqlens)) * Hkv * D * 2 * 2 + B * H * D * 2 + B * H * D * 4
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "grouped_query_causal_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = t.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    from grouped_query_causal_b200 import binding as gqa
+    lib = gqa.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    pin = synthetic.make(PREFILL)
+    dec = synthetic.make(DECODE)
+    B, T, H, D = pin.q.shape
+    Hkv = pin.k.shape[2]
+    dB, dH, _ = dec.q.shape
+    dHkv = dec.k_cache.shape[1]
+    max_len = dec.max_len
+    flops = prefill_flops(B, T, H, D)
+    dbytes = decode_bytes(dec.seqlens.tolist(), dH, dHkv, D)
+
+    # device-resident inputs, outputs, workspaces
+    q, k, v, pos = pin.q.to(dev), pin.k.to(dev), pin.v.to(dev), pin.pos.to(dev)
+    wq, wk = pin.wq.to(dev), pin.wk.to(dev)
+    khat = torch.empty_like(k)
+    out = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
+    dq, kc, vc = dec.q.to(dev), dec.k_cache.to(dev), dec.v_cache.to(dev)
+    offs, sl, dwq = dec.offsets.to(dev), dec.seqlens.to(dev), dec.wq.to(dev)
+    dout = torch.empty((dB, dH, D), dtype=torch.float32, device=dev)
+    dws = torch.empty(gqa.decode_workspace_size(dB, dH, dHkv, max_len, D), dtype=torch.uint8, device=dev)
+    ptr = lambda t: t.data_ptr()  # noqa: E731
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        st = lib.gqa_attn_k_norm_rope(ptr(k), ptr(pos), ptr(wk), pin.theta, pin.eps, ptr(khat), B * T, Hkv, D, sh)
+        if ev:
+            ev[1].record(stream)
+        st |= lib.gqa_attn_prefill_khat(ptr(q), ptr(khat), ptr(v), ptr(pos), ptr(wq), pin.theta, pin.eps, ptr(out),
+                                        B, T, H, Hkv, D, sh)
+        if ev:
+            ev[2].record(stream)
+        st |= lib.gqa_attn_decode(ptr(dq), ptr(kc), ptr(vc), ptr(offs), ptr(sl), None, ptr(dwq), dec.theta, dec.eps,
+                                  ptr(dout), dB, dH, dHkv, D, max_len, ptr(dws), dws.numel(), sh)
+        if ev:
+            ev[3].record(stream)
+        if st != 0:
+            raise RuntimeError(f"library call failed with status {st}")
+
+    launches_per_step = 2 + 2   # k prologue + attention, decode split + merge
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if gqa.device_status() != 0:
+        raise RuntimeError("device status error after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    if gqa.device_status() != 0:
+        raise RuntimeError("device status error in the timed region")
+
+    total_ms = t0.elapsed_time(t1)
+    pro_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    dec_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    # max over ranks of every duration
+    times = torch.tensor([total_ms, pro_ms, attn_ms, dec_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    total_ms, pro_ms, attn_ms, dec_ms = times.tolist()
+    K = args.steps
+    prefill_s = (pro_ms + attn_ms) / 1e3
+    dec_s = dec_ms / 1e3
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    e2e = run_e2e(gqa, pin, dec, dev, stream, rank, world, max(3, min(K, 10)))
+
+    if rank != 0:
+        return None
+    pk, pk_kind = peaks()
+    hbm = float(pk["hbm_gbs"])
+    tc = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    attn_tflops = flops * K / (attn_ms / 1e3) / 1e12
+    dec_gbs = dbytes * K / dec_s / 1e9
+    traffic_attn = traffic_from_profiles("attn_fwd_kernel")
+    traffic_dec = traffic_from_profiles("decode_split_kernel")
+    line = {
+        "metric": METRIC,
+        "value": round(world * flops * K / prefill_s / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": "large prefill (B4 T4096 H32 Hkv8 D128, inputs x0.5, causal) + batched decode "
+                        "(64 seqs, cache len U[1024,32768], H32 Hkv8 D128)",
+            "prefill": {"B": B, "T": T, "H": H, "Hkv": Hkv, "D": D, "flops_per_step": flops},
+            "decode": {"B": dB, "H": dH, "Hkv": dHkv, "D": D, "cached_tokens": int(dec.seqlens.sum()),
+                       "bytes_per_step": dbytes},
+            "l2": "inputs larger than L2 (prefill q/k/v/out 470 MB; decode KV cache 4.4 GB); no flush",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "prefill_ms": round(1e3 * prefill_s / K, 4),
+        "decode": {
+            "value": round(world * dbytes * K / dec_s / 1e9, 1),
+            "unit": "GB/s",
+            "ms": round(1e3 * dec_s / K, 4),
+            "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(dec_gbs / hbm, 4), "traffic": traffic_dec,
+                         "kernel": "decode_split_kernel + decode_merge_kernel (one call)",
+                         "peak_source": f"hbm_gbs of {pk_kind}"},
+            "e2e": e2e["decode"],
+        },
+        "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": tc, "unit": "TFLOP/s",
+                     "frac": round(attn_tflops / tc, 4), "traffic": traffic_attn, "kernel": "attn_fwd_kernel",
+                     "attn_ms": round(attn_ms / K, 4), "k_prologue_ms": round(pro_ms / K, 4),
+                     "peak_source": f"bf16_tflops_sustained of {pk_kind}",
+                     "peak_burst": float(pk["bf16_tflops"])},
+        "e2e": e2e["prefill"],
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(pin, dec, budget_s=args.cpu_seconds)
+    return line
+
+
+def run_e2e(gqa, pin, dec, dev, stream, rank, world, steps):
+    """Same metrics through the public API with host (pinned) buffers: every step copies
+    that step's inputs host->device, runs the call, and reads the result back."""
+    lib = gqa.load()
+    sh = stream.cuda_stream
+    B, T, H, D = pin.q.shape
+    Hkv = pin.k.shape[2]
+    dB, dH, _ = dec.q.shape
+    dHkv = dec.k_cache.shape[1]
+    max_len = dec.max_len
+    hp = {n: getattr(pin, n).pin_memory() for n in ("q", "k", "v", "pos", "wq", "wk")}
+    hd = {"q": dec.q.pin_memory(), "k_cache": dec.k_cache.pin_memory(), "v_cache": dec.v_cache.pin_memory(),
+          "offsets": dec.offsets.pin_memory(), "seqlens": dec.seqlens.pin_memory(), "wq": dec.wq.pin_memory()}
+    dp = {n: torch.empty_like(t, device=dev) for n, t in hp.items()}
+    dd = {n: torch.empty_like(t, device=dev) for n, t in hd.items()}
+    out = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
+    hout = torch.empty((B, T, H, D), dtype=torch.float32).pin_memory()
+    dout = torch.empty((dB, dH, D), dtype=torch.float32, device=dev)
+    hdout = torch.empty((dB, dH, D), dtype=torch.float32).pin_memory()
+    pws = torch.empty(gqa.prefill_workspace_size(B, T, H, Hkv, D), dtype=torch.uint8, device=dev)
+    dws = torch.empty(gqa.decode_workspace_size(dB, dH, dHkv, max_len, D), dtype=torch.uint8, device=dev)
+    ptr = lambda t: t.data_ptr()  # noqa: E731
+    p_in = sum(t.numel() * t.element_size() for t in hp.values())
+    d_in = sum(t.numel() * t.element_size() for t in hd.values())
+
+    def prefill_step():
+        for n in hp:
+            dp[n].copy_(hp[n], non_blocking=True)
+        st = lib.gqa_attn_prefill(ptr(dp["q"]), ptr(dp["k"]), ptr(dp["v"]), ptr(dp["pos"]), ptr(dp["wq"]),
+                                  ptr(dp["wk"]), pin.theta, pin.eps, ptr(out), B, T, H, Hkv, D, ptr(pws),
+                                  pws.numel(), sh)
+        hout.copy_(out, non_blocking=True)
+        return st
+
+    def decode_step():
+        for n in hd:
+            dd[n].copy_(hd[n], non_blocking=True)
+        st = lib.gqa_attn_decode(ptr(dd["q"]), ptr(dd["k_cache"]), ptr(dd["v_cache"]), ptr(dd["offsets"]),
+                                 ptr(dd["seqlens"]), None, ptr(dd["wq"]), dec.theta, dec.eps, ptr(dout), dB, dH,
+                                 dHkv, D, max_len, ptr(dws), dws.numel(), sh)
+        hdout.copy_(dout, non_blocking=True)
+        return st
+
+    res = {}
+    for name, fn, units, unit, scale, b_in, b_out in (
+            ("prefill", prefill_step, prefill_flops(B, T, H, D), "TFLOP/s", 1e12, p_in, hout.numel() * 4),
+            ("decode", decode_step, decode_bytes(dec.seqlens.tolist(), dH, dHkv, D), "GB/s", 1e9, d_in,
+             hdout.numel() * 4)):
+        if fn() != 0:
+            raise RuntimeError(f"e2e {name} failed")
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            if fn() != 0:
+                raise RuntimeError(f"e2e {name} failed")
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
+        sec = ms.item() / 1e3
+        res[name] = {"value": round(world * units * steps / sec / scale, 3), "unit": unit,
+                     "h2d_bytes_per_step": int(b_in), "d2h_bytes_per_step": int(b_out), "steps": steps}
+    return res
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+def _prefill_sample_rows(T, H, B, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.stack([rng.integers(0, B, n), rng.integers(0, H, n), rng.integers(0, T, n)], 1).astype(np.int64)
+
+
+def oracle_prefill_sample(pin, rows):
+    from oracle import oracle
+    b = synthetic.bf16_bits
+    t0 = time.perf_counter()
+    oracle.prefill_rows(b(pin.q), b(pin.k), b(pin.v), pin.pos.numpy(), pin.wq.numpy(), pin.wk.numpy(), pin.theta,
+                        pin.eps, rows)
+    sec = time.perf_counter() - t0
+    D = pin.q.shape[-1]
+    return float(np.sum(rows[:, 2] + 1) * 4 * D), sec   # 4*D FLOP per visible (i, j) pair
+
+
+def oracle_decode_sample(dec, idx):
+    from oracle import oracle
+    b = synthetic.bf16_bits
+    offs = dec.offsets.numpy()
+    sl = dec.seqlens.numpy()
+    H, D = dec.q.shape[1], dec.q.shape[2]
+    Hkv = dec.k_cache.shape[1]
+    lo, hi = int(offs[idx].min()), int((offs[idx] + sl[idx]).max())
+    kc = b(dec.k_cache[lo:hi])
+    vc = b(dec.v_cache[lo:hi])
+    t0 = time.perf_counter()
+    oracle.decode(b(dec.q)[idx], kc, vc, np.append(offs[idx], hi) - lo, sl[idx], None, dec.wq.numpy(), dec.theta,
+                  dec.eps)
+    sec = time.perf_counter() - t0
+    return float(decode_bytes(sl[idx].tolist(), H, Hkv, D)), sec
+
+
+def cpu_baseline(pin, dec, budget_s=20.0):
+    """The oracle as it stands on the host cores, on bounded samples of both workloads."""
+    from oracle import oracle
+    B, T, H, D = pin.q.shape
+    oracle.num_threads()   # build + load before timing
+    # prefill: random rows of the large workload, doubled until about half the budget
+    n = 64
+    fl, sec = oracle_prefill_sample(pin, _prefill_sample_rows(T, H, B, n, 0))
+    while sec < budget_s / 4 and n < 1 << 16:
+        n *= 2
+        fl, sec = oracle_prefill_sample(pin, _prefill_sample_rows(T, H, B, n, n))
+    # decode: whole sequences (all heads), shortest first, about the other half
+    order = np.argsort(dec.seqlens.numpy())
+    m = 1
+    by, dsec = oracle_decode_sample(dec, order[:m])
+    while dsec < budget_s / 4 and m < len(order):
+        m = min(len(order), m * 2)
+        by, dsec = oracle_decode_sample(dec, np.sort(order[:m]))
+    return {"value": round(fl / sec / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"prefill: {n} random output rows (b, head, i) of the large prefill, {sec:.1f} s; "
+                      f"fp64 C, OpenMP",
+            "decode": {"value": round(by / dsec / 1e9, 4), "unit": "GB/s",
+                       "sample": f"decode: the {m} shortest sequences of the batched decode, all heads, {dsec:.1f} s"}}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle as it stands, on the host cores; each step is a
+    bounded sample (prefill rows + one decode sequence) of the same workloads."""
+    if rank != 0:
+        return None
+    from oracle import oracle
+    pin = synthetic.make(PREFILL)
+    dec = synthetic.make(DECODE)
+    B, T, H, D = pin.q.shape
+    order = np.argsort(dec.seqlens.numpy())
+    rows_per_step = 16
+    fl_t = sec_t = by_t = dsec_t = 0.0
+    for i in range(args.warmup + args.steps):
+        rows = _prefill_sample_rows(T, H, B, rows_per_step, 1000 + i)
+        fl, sec = oracle_prefill_sample(pin, rows)
+        by, dsec = oracle_decode_sample(dec, order[i % 4:i % 4 + 1])
+        if i >= args.warmup:
+            fl_t += fl
+            sec_t += sec
+            by_t += by
+            dsec_t += dsec
+    value = fl_t / sec_t / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * (sec_t + dsec_t) / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "large prefill (B4 T4096 H32 Hkv8 D128, inputs x0.5, causal) + batched decode "
+                               "(64 seqs, cache len U[1024,32768], H32 Hkv8 D128)",
+                   "sample_per_step": f"{rows_per_step} prefill output rows + 1 decode sequence (all heads)"},
+        "decode": {"value": round(by_t / dsec_t / 1e9, 4), "unit": "GB/s"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{rows_per_step} random prefill rows + 1 decode sequence per step"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_reference(args, rank, world) if args.impl == "reference" else run_ours(args, rank, world,
+                                                                                          local_rank)
+    finally:
+        if world > 1 and args.impl == "ours":
+            torch.distributed.destroy_process_group()
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,219 @@
+"""Python binding of ``libgqa_attn.so`` (the C ABI in ``include/gqa_attn.h``).
+
+Argument marshalling only: torch tensors supply device memory and the current
+CUDA stream; every step of the computation runs in the library's kernels.  There
+is no fallback: if the library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgqa_attn.so")
+
+GQA_OK = 0
+STATUS_NAMES = {
+    0: "GQA_OK", -1: "GQA_ERR_INVALID_ARG", -2: "GQA_ERR_UNSUPPORTED", -3: "GQA_ERR_WORKSPACE",
+    -4: "GQA_ERR_CUDA", -5: "GQA_ERR_DEVICE_TIMEOUT", -6: "GQA_ERR_DEVICE_INPUT",
+}
+# Every symbol the header declares.
+EXPORTS = ("gqa_status_string", "gqa_attn_prefill_workspace_size", "gqa_attn_prefill",
+           "gqa_attn_k_norm_rope", "gqa_attn_prefill_khat", "gqa_attn_decode_workspace_size",
+           "gqa_attn_decode", "gqa_attn_device_status")
+
+
+class GqaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library and declare its C signatures (raises if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m grouped_query_causal_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.gqa_status_string.argtypes = [I]
+    lib.gqa_status_string.restype = ctypes.c_char_p
+    lib.gqa_attn_prefill_workspace_size.argtypes = [I, I, I, I, I]
+    lib.gqa_attn_prefill_workspace_size.restype = Z
+    lib.gqa_attn_prefill.argtypes = [P, P, P, P, P, P, F, F, P, I, I, I, I, I, P, Z, P]
+    lib.gqa_attn_prefill.restype = I
+    lib.gqa_attn_k_norm_rope.argtypes = [P, P, P, F, F, P, ctypes.c_int64, I, I, P]
+    lib.gqa_attn_k_norm_rope.restype = I
+    lib.gqa_attn_prefill_khat.argtypes = [P, P, P, P, P, F, F, P, I, I, I, I, I, P]
+    lib.gqa_attn_prefill_khat.restype = I
+    lib.gqa_attn_decode_workspace_size.argtypes = [I, I, I, I, I]
+    lib.gqa_attn_decode_workspace_size.restype = Z
+    lib.gqa_attn_decode.argtypes = [P, P, P, P, P, P, P, F, F, P, I, I, I, I, I, P, Z, P]
+    lib.gqa_attn_decode.restype = I
+    lib.gqa_attn_device_status.argtypes = [P]
+    lib.gqa_attn_device_status.restype = I
+    _lib = lib
+    return lib
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check(t: torch.Tensor, name: str, dtype: torch.dtype, dim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dims, got {tuple(t.shape)}")
+
+
+def _raise(status: int, what: str):
+    if status != GQA_OK:
+        raise GqaError(status, what)
+
+
+def prefill_workspace_size(B: int, T: int, H: int, Hkv: int, D: int = 128) -> int:
+    return int(load().gqa_attn_prefill_workspace_size(B, T, H, Hkv, D))
+
+
+def decode_workspace_size(B: int, H: int, Hkv: int, max_len: int, D: int = 128) -> int:
+    return int(load().gqa_attn_decode_workspace_size(B, H, Hkv, D, max_len))
+
+
+def prefill(q, k, v, pos, qnorm_w, knorm_w, theta: float = 1.0e6, eps: float = 1e-6,
+            out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Causal GQA prefill with fused q/k RMSNorm + RoPE.  q [B,T,H,D] bf16, k/v
+    [B,T,Hkv,D] bf16, pos [B,T] int32, norm weights [D] fp32 -> out [B,T,H,D] fp32."""
+    lib = load()
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    _check(pos, "pos", torch.int32, 2)
+    _check(qnorm_w, "qnorm_w", torch.float32, 1)
+    _check(knorm_w, "knorm_w", torch.float32, 1)
+    B, T, H, D = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, T, Hkv, D) or v.shape != k.shape or pos.shape != (B, T):
+        raise ValueError("shape mismatch between q, k, v, pos")
+    if qnorm_w.shape != (D,) or knorm_w.shape != (D,):
+        raise ValueError("norm weights must be [D]")
+    if out is None:
+        out = torch.empty((B, T, H, D), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 4)
+    need = int(lib.gqa_attn_prefill_workspace_size(B, T, H, Hkv, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib.gqa_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(qnorm_w), _ptr(knorm_w),
+                              float(theta), float(eps), _ptr(out), B, T, H, Hkv, D, _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _raise(st, "gqa_attn_prefill")
+    return out
+
+
+def k_norm_rope(k, pos, knorm_w, theta: float = 1.0e6, eps: float = 1e-6,
+                out: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """k-hat = RoPE(RMSNorm(k)) in bf16.  k [..., Hkv, D] bf16 with one position per
+    token (pos has the leading shape of k) -> k_hat of k's shape (a decode cache)."""
+    lib = load()
+    if k.dtype != torch.bfloat16 or not k.is_cuda or not k.is_contiguous() or k.dim() < 2:
+        raise ValueError("k must be a contiguous CUDA bf16 tensor [..., Hkv, D]")
+    _check(knorm_w, "knorm_w", torch.float32, 1)
+    Hkv, D = k.shape[-2], k.shape[-1]
+    N = k.numel() // (Hkv * D) if k.numel() else 0
+    if pos.dtype != torch.int32 or not pos.is_cuda or not pos.is_contiguous() or pos.numel() != N:
+        raise ValueError("pos must be a contiguous CUDA int32 tensor with one entry per token")
+    if out is None:
+        out = torch.empty_like(k)
+    st = lib.gqa_attn_k_norm_rope(_ptr(k), _ptr(pos), _ptr(knorm_w), float(theta), float(eps), _ptr(out), N,
+                                  Hkv, D, _stream_handle(stream))
+    _raise(st, "gqa_attn_k_norm_rope")
+    return out
+
+
+def prefill_khat(q, k_hat, v, pos, qnorm_w, theta: float = 1.0e6, eps: float = 1e-6,
+                 out: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Attention stage of prefill on already normed + rotated keys (k_hat [B,T,Hkv,D])."""
+    lib = load()
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k_hat, "k_hat", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    _check(pos, "pos", torch.int32, 2)
+    _check(qnorm_w, "qnorm_w", torch.float32, 1)
+    B, T, H, D = q.shape
+    Hkv = k_hat.shape[2]
+    if k_hat.shape != (B, T, Hkv, D) or v.shape != k_hat.shape or pos.shape != (B, T):
+        raise ValueError("shape mismatch between q, k_hat, v, pos")
+    if out is None:
+        out = torch.empty((B, T, H, D), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 4)
+    st = lib.gqa_attn_prefill_khat(_ptr(q), _ptr(k_hat), _ptr(v), _ptr(pos), _ptr(qnorm_w), float(theta),
+                                   float(eps), _ptr(out), B, T, H, Hkv, D, _stream_handle(stream))
+    _raise(st, "gqa_attn_prefill_khat")
+    return out
+
+
+def decode(q, k_cache, v_cache, cache_offsets, seqlens, qnorm_w, max_len: int,
+           q_pos: Optional[torch.Tensor] = None, theta: float = 1.0e6, eps: float = 1e-6,
+           out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Split-KV decode.  q [B,H,D] bf16 (raw), caches [rows,Hkv,D] bf16 (normed/rotated
+    K, raw V), cache_offsets [B+1] int64, seqlens [B] int32, q_pos [B] int32 or None
+    (then the query sits at position seqlens[b]) -> out [B,H,D] fp32."""
+    lib = load()
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 3)
+    _check(v_cache, "v_cache", torch.bfloat16, 3)
+    _check(cache_offsets, "cache_offsets", torch.int64, 1)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    _check(qnorm_w, "qnorm_w", torch.float32, 1)
+    if q_pos is not None:
+        _check(q_pos, "q_pos", torch.int32, 1)
+    B, H, D = q.shape
+    Hkv = k_cache.shape[1]
+    if k_cache.shape[2] != D or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape mismatch")
+    if cache_offsets.shape != (B + 1,) or seqlens.shape != (B,):
+        raise ValueError("cache_offsets must be [B+1] and seqlens [B]")
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 3)
+    need = int(lib.gqa_attn_decode_workspace_size(B, H, Hkv, D, int(max_len)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib.gqa_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_offsets), _ptr(seqlens),
+                             _ptr(q_pos), _ptr(qnorm_w), float(theta), float(eps), _ptr(out), B, H, Hkv, D,
+                             int(max_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream_handle(stream))
+    _raise(st, "gqa_attn_decode")
+    return out
+
+
+def device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronize `stream`, read and clear the device error word; returns a status code."""
+    return int(load().gqa_attn_device_status(_stream_handle(stream)))
+
+
+def check_device_status(stream: Optional[torch.cuda.Stream] = None):
+    _raise(device_status(stream), "device status")

@@ -1,0 +1,324 @@
+// decode.cuh -- split-KV decode for sm_100a.
+//
+// One new query token per sequence attends to its whole KV cache ("Qwen3系列1-理论基础&
+// 真实结构" D2-3: decode feeds a single token and is bound by reading the cache).  The
+// work is bandwidth-bound: every cached K/V row is read exactly once, shared by the
+// h = H/Hkv query heads of its group ("深入剖析Qwen3模型架构" 3.1.2).
+//
+//  decode_split_kernel: one CTA per (sequence, KV head, 512-key chunk, head pass).
+//    The h query vectors are normed + rotated at the query position in the prologue;
+//    each warp streams 128 keys of the chunk with 16-byte loads (a half-warp per
+//    256-byte key row), first K (scores for all h heads), then V (weighted sum),
+//    and the four warp partials are merged into one (m, l, O) per head.
+//  decode_merge_kernel: log-sum-exp combination of the chunk partials of each
+//    (sequence, query head):  O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c.
+#pragma once
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+#include "rope.cuh"
+
+namespace gqa {
+
+constexpr int kChunk = 512;                // keys per split
+constexpr int kWarpKeys = kChunk / 4;      // keys per warp
+constexpr int kRowPairs = 8;               // row pairs in flight per warp (16 rows)
+constexpr int kMaxHeadsPerPass = 8;
+
+struct DecodeParams {
+    const uint16_t *q;        // bf16 [B, H, D]
+    const uint16_t *kc;       // bf16 [rows, Hkv, D]
+    const uint16_t *vc;       // bf16 [rows, Hkv, D]
+    const int64_t *offsets;   // [B + 1]
+    const int32_t *seqlens;   // [B]
+    const int32_t *qpos;      // [B] or nullptr
+    const float *wq;          // [D]
+    float *part_o;            // [B * maxC * H, D]
+    float *part_ml;           // [B * maxC * H, 2]
+    float *out;               // [B, H, D]
+    unsigned *err;
+    int B, H, Hkv, hpg, maxC, max_len;
+    float eps;
+    float scale_log2;         // log2(e) / sqrt(D)
+    RopeFreqs rf;
+};
+
+// Device-side bounds of sequence b: 1 <= len <= max_len and len fits its rows.
+__device__ __forceinline__ bool decode_seq_ok(const DecodeParams &p, int b, int &len, long long &off) {
+    len = p.seqlens[b];
+    off = p.offsets[b];
+    const long long cap = p.offsets[b + 1] - off;
+    return len >= 1 && len <= p.max_len && static_cast<long long>(len) <= cap && off >= 0;
+}
+
+template <int HG>
+struct HeadsLog2 {
+    static constexpr int value = HG == 1 ? 0 : HG == 2 ? 1 : HG == 4 ? 2 : 3;
+};
+
+// Sum HG per-lane partial dot products over the 16 lanes of each half-warp with a
+// butterfly that halves the vector at each of the first log2(HG) steps.  Returns the
+// full sum for head decode_head_of_lane<HG>(lane); all lanes of a half-warp that share
+// that head hold the same value.
+template <int HG>
+__device__ __forceinline__ float decode_reduce_heads(const float (&v)[HG], int lane) {
+    constexpr int LG = HeadsLog2<HG>::value;
+    float w[HG];
+#pragma unroll
+    for (int i = 0; i < HG; ++i) w[i] = v[i];
+#pragma unroll
+    for (int step = 0; step < 4; ++step) {
+        const int m = 8 >> step;
+        if (step < LG) {
+            const bool upper = (lane & m) != 0;
+            const int half = HG >> (step + 1);
+#pragma unroll
+            for (int i = 0; i < HG / 2; ++i) {
+                if (i < half) {
+                    const float keep = upper ? w[i + half] : w[i];
+                    const float send = upper ? w[i] : w[i + half];
+                    w[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+        } else {
+            w[0] += __shfl_xor_sync(0xffffffffu, w[0], m);
+        }
+    }
+    return w[0];
+}
+
+template <int HG>
+__device__ __forceinline__ int decode_head_of_lane(int lane) {
+    constexpr int LG = HeadsLog2<HG>::value;
+    int h = 0;
+#pragma unroll
+    for (int s = 0; s < LG; ++s)
+        if (lane & (8 >> s)) h += HG >> (s + 1);
+    return h;
+}
+
+template <int HG>
+__global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant__ DecodeParams p) {
+    constexpr int LG = HeadsLog2<HG>::value;
+    __shared__ __align__(16) float sq[HG][kHeadDim];
+    __shared__ __align__(16) float sbuf[4][kWarpKeys * HG];   // scores / probabilities, then partial O
+    __shared__ float sml[4][2][HG];
+
+    const int b = blockIdx.x / p.Hkv;
+    const int g = blockIdx.x % p.Hkv;
+    const int c = blockIdx.y;
+    const int jbase = blockIdx.z * HG;
+    int len;
+    long long off;
+    if (!decode_seq_ok(p, b, len, off)) {
+        if (c == 0 && g == 0 && blockIdx.z == 0 && threadIdx.x == 0) atomicOr(p.err, kErrInput);
+        return;
+    }
+    const int k0 = c * kChunk;
+    if (k0 >= len) return;
+    const int k1 = min(len, k0 + kChunk);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---- q prologue: RMSNorm + RoPE at the query position, scaled into base-2 logits
+    {
+        const int ps = p.qpos ? p.qpos[b] : len;
+        float cs0, sn0, cs1, sn1;
+        rope_cos_sin(ps, p.rf.inv_freq[2 * lane], cs0, sn0);
+        rope_cos_sin(ps, p.rf.inv_freq[2 * lane + 1], cs1, sn1);
+        const float4 w = reinterpret_cast<const float4 *>(p.wq)[lane];
+        for (int jj = warp; jj < HG; jj += 4) {
+            const int j = jbase + jj;
+            float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+            if (j < p.hpg) {
+                const int hq = g * p.hpg + j;
+                const uint2 raw = *reinterpret_cast<const uint2 *>(p.q + (static_cast<size_t>(b) * p.H + hq) * kHeadDim + 4 * lane);
+                const float x0 = bf16lo(raw.x), x1 = bf16hi(raw.x), x2 = bf16lo(raw.y), x3 = bf16hi(raw.y);
+                float ss = x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + p.eps);
+                const float a0 = w.x * x0 * inv, a1 = w.y * x1 * inv, a2 = w.z * x2 * inv, a3 = w.w * x3 * inv;
+                y0 = a0 * cs0 - a1 * sn0;
+                y1 = a0 * sn0 + a1 * cs0;
+                y2 = a2 * cs1 - a3 * sn1;
+                y3 = a2 * sn1 + a3 * cs1;
+            }
+            sq[jj][4 * lane + 0] = y0 * p.scale_log2;
+            sq[jj][4 * lane + 1] = y1 * p.scale_log2;
+            sq[jj][4 * lane + 2] = y2 * p.scale_log2;
+            sq[jj][4 * lane + 3] = y3 * p.scale_log2;
+        }
+    }
+    __syncthreads();
+
+    const int sub = lane & 15;    // elements 8*sub .. 8*sub+7 of a row
+    const int rsel = lane >> 4;   // which row of the pair
+    float qr[HG][8];
+#pragma unroll
+    for (int jj = 0; jj < HG; ++jj)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qr[jj][e] = sq[jj][8 * sub + e];
+
+    const int kw0 = k0 + warp * kWarpKeys;
+    const int kw1 = min(k1, kw0 + kWarpKeys);
+    const int nrow = max(0, kw1 - kw0);
+    float *sw = sbuf[warp];
+    const size_t row_stride = static_cast<size_t>(p.Hkv) * kHeadDim;
+    const uint16_t *kbase = p.kc + (static_cast<size_t>(off) * p.Hkv + g) * kHeadDim + 8 * sub;
+    const uint16_t *vbase = p.vc + (static_cast<size_t>(off) * p.Hkv + g) * kHeadDim + 8 * sub;
+    const bool writer = (lane & ((16 >> LG) - 1)) == 0;
+    const int my_head = decode_head_of_lane<HG>(lane);
+
+    // ---- K sweep: base-2 logits of the HG heads for each key of this warp
+    for (int base = kw0; base < kw1; base += 2 * kRowPairs) {
+        uint4 kv[kRowPairs];
+#pragma unroll
+        for (int u = 0; u < kRowPairs; ++u) {
+            const int row = base + 2 * u + rsel;
+            kv[u] = row < kw1 ? ldg_stream_v4(kbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kRowPairs; ++u) {
+            const uint32_t rw[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                x[2 * i] = bf16lo(rw[i]);
+                x[2 * i + 1] = bf16hi(rw[i]);
+            }
+            float part[HG];
+#pragma unroll
+            for (int jj = 0; jj < HG; ++jj) {
+                float acc = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc = fmaf(qr[jj][e], x[e], acc);
+                part[jj] = acc;
+            }
+            const float sfull = decode_reduce_heads<HG>(part, lane);
+            const int rl = base + 2 * u + rsel - kw0;   // < kWarpKeys by construction
+            if (writer) sw[rl * HG + my_head] = sfull;
+        }
+    }
+    __syncwarp();
+
+    // ---- per-warp softmax statistics; lane handles head lane % HG
+    const int nent = nrow * HG;
+    float mloc = -INFINITY;
+    for (int e = lane; e < nent; e += 32) mloc = fmaxf(mloc, sw[e]);
+#pragma unroll
+    for (int o = 16; o >= HG; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+    float lloc = 0.f;
+    for (int e = lane; e < nent; e += 32) {
+        const float pe = ex2_approx(sw[e] - mloc);
+        sw[e] = pe;
+        lloc += pe;
+    }
+#pragma unroll
+    for (int o = 16; o >= HG; o >>= 1) lloc += __shfl_xor_sync(0xffffffffu, lloc, o);
+    __syncwarp();
+
+    // ---- V sweep: weighted sum of this warp's value rows
+    float acc[HG][8];
+#pragma unroll
+    for (int jj = 0; jj < HG; ++jj)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[jj][e] = 0.f;
+    for (int base = kw0; base < kw1; base += 2 * kRowPairs) {
+        uint4 vv[kRowPairs];
+#pragma unroll
+        for (int u = 0; u < kRowPairs; ++u) {
+            const int row = base + 2 * u + rsel;
+            vv[u] = row < kw1 ? ldg_stream_v4(vbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kRowPairs; ++u) {
+            const int row = base + 2 * u + rsel;
+            if (row < kw1) {
+                const float *pr = sw + (row - kw0) * HG;
+                float pw[HG];
+#pragma unroll
+                for (int jj = 0; jj < HG; ++jj) pw[jj] = pr[jj];
+                const uint32_t rw[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float v0 = bf16lo(rw[i]), v1 = bf16hi(rw[i]);
+#pragma unroll
+                    for (int jj = 0; jj < HG; ++jj) {
+                        acc[jj][2 * i] = fmaf(pw[jj], v0, acc[jj][2 * i]);
+                        acc[jj][2 * i + 1] = fmaf(pw[jj], v1, acc[jj][2 * i + 1]);
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int jj = 0; jj < HG; ++jj)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[jj][e] += __shfl_xor_sync(0xffffffffu, acc[jj][e], 16);
+    __syncwarp();
+    if (rsel == 0) {
+#pragma unroll
+        for (int jj = 0; jj < HG; ++jj) {
+            float4 *dst = reinterpret_cast<float4 *>(sw + jj * kHeadDim + 8 * sub);
+            dst[0] = make_float4(acc[jj][0], acc[jj][1], acc[jj][2], acc[jj][3]);
+            dst[1] = make_float4(acc[jj][4], acc[jj][5], acc[jj][6], acc[jj][7]);
+        }
+    }
+    if (lane < HG) {
+        sml[warp][0][lane] = mloc;
+        sml[warp][1][lane] = lloc;
+    }
+    __syncthreads();
+
+    // ---- merge the four warps; thread tid owns element d = tid
+    const size_t slot0 = (static_cast<size_t>(b) * p.maxC + c) * p.H + static_cast<size_t>(g) * p.hpg;
+#pragma unroll 1
+    for (int jj = 0; jj < HG; ++jj) {
+        const int j = jbase + jj;
+        if (j >= p.hpg) break;
+        float M = sml[0][0][jj];
+#pragma unroll
+        for (int w = 1; w < 4; ++w) M = fmaxf(M, sml[w][0][jj]);
+        float O = 0.f, L = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float sc = ex2_approx(sml[w][0][jj] - M);
+            O = fmaf(sc, sbuf[w][jj * kHeadDim + tid], O);
+            L = fmaf(sc, sml[w][1][jj], L);
+        }
+        const size_t slot = slot0 + j;
+        p.part_o[slot * kHeadDim + tid] = O;
+        if (tid == 0) {
+            p.part_ml[2 * slot] = M;
+            p.part_ml[2 * slot + 1] = L;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(128) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
+    const int b = blockIdx.x / p.H;
+    const int hq = blockIdx.x % p.H;
+    const int d = threadIdx.x;
+    float *o = p.out + (static_cast<size_t>(b) * p.H + hq) * kHeadDim;
+    int len;
+    long long off;
+    if (!decode_seq_ok(p, b, len, off)) {
+        o[d] = __int_as_float(0x7fc00000);   // quiet NaN
+        return;
+    }
+    const int nch = (len + kChunk - 1) / kChunk;
+    const size_t slot0 = static_cast<size_t>(b) * p.maxC * p.H + hq;   // chunk c: slot0 + c * H
+    float M = -INFINITY;
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, p.part_ml[2 * (slot0 + static_cast<size_t>(c) * p.H)]);
+    float O = 0.f, L = 0.f;
+    for (int c = 0; c < nch; ++c) {
+        const size_t slot = slot0 + static_cast<size_t>(c) * p.H;
+        const float sc = ex2_approx(p.part_ml[2 * slot] - M);
+        O = fmaf(sc, p.part_o[slot * kHeadDim + d], O);
+        L = fmaf(sc, p.part_ml[2 * slot + 1], L);
+    }
+    o[d] = O / L;
+}
+
+}  // namespace gqa

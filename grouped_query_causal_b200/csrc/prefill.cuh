@@ -1,0 +1,449 @@
+// prefill.cuh -- prefill kernels for sm_100a.
+//
+//  (1) k_prologue_kernel: RMSNorm + RoPE of every K head vector, written once as
+//      bf16 k-hat.  Every K tile is read by all later query blocks of its sequence and
+//      by every query head of its group, so transforming it once is cheaper than
+//      redoing it in each reader (that would multiply the work by h * (T/128) / 2).
+//  (2) attn_fwd_kernel: flash-style causal GQA attention.  One CTA owns one
+//      (batch, KV head, 128-token query block, pair of query heads of the group).
+//      The raw Q tiles are loaded by TMA and normed + rotated in registers in place
+//      (the fused q prologue); K-hat/V tiles stream through a TMA ring and serve both
+//      query heads of the pair; S = Q K^T and O += P V run on the 5th-generation
+//      tensor cores (tcgen05.mma, fp32 accumulators in TMEM); the online softmax
+//      runs in two warpgroups (one per head of the pair, ping-ponging with the tensor
+//      core) with one query row per thread; causal tiles above the diagonal are never
+//      loaded.
+//
+// Sources, by page title and section: "Qwen3系列1-理论基础&真实结构" D1-2 (stable
+// softmax), D1-4 (softmax(QK^T/sqrt(d)+M)V), D1-5 (causal mask), D2-1 (RMSNorm), D2-2
+// (QK-Norm then RoPE, V untouched), D2-3 (GQA); "深入剖析Qwen3模型架构" 3.1.2 (K/V
+// shared by the h = H/Hkv consecutive query heads, RoPE pairs), 3.4.1 (frequencies);
+// "Qwen3" walkthrough, "Attention 的 Forward 流程" (norm, rotary, then attention).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+#include "rope.cuh"
+
+namespace gqa {
+
+// ============================================================================ K prologue
+struct KPrologueParams {
+    const uint16_t *k;     // bf16 [ntok, Hkv, D]
+    const int32_t *pos;    // [ntok]
+    const float *wk;       // [D]
+    uint16_t *khat;        // bf16 [ntok, Hkv, D]
+    long long ntok;
+    int Hkv;
+    float eps;
+    RopeFreqs rf;
+};
+
+// One warp per token at a time; each half-warp transforms one head vector, each lane
+// eight consecutive elements (four RoPE pairs).  cos/sin are evaluated once per token
+// and reused for all of its KV heads.
+__global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__ KPrologueParams p) {
+    const int lane = threadIdx.x & 31;
+    const int half = lane >> 4;
+    const int sub = lane & 15;
+    const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    long long tok = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+
+    const float4 wa = reinterpret_cast<const float4 *>(p.wk)[2 * sub];
+    const float4 wb = reinterpret_cast<const float4 *>(p.wk)[2 * sub + 1];
+    const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+
+    for (; tok < p.ntok; tok += nwarps) {
+        const int ps = p.pos[tok];
+        float cs[4], sn[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rope_cos_sin(ps, p.rf.inv_freq[4 * sub + i], cs[i], sn[i]);
+        for (int h0 = 0; h0 < p.Hkv; h0 += 2) {
+            const int hh = h0 + half;
+            const bool act = hh < p.Hkv;
+            const size_t off = (static_cast<size_t>(tok) * p.Hkv + hh) * kHeadDim + 8 * sub;
+            uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+            if (act) raw = *reinterpret_cast<const uint4 *>(p.k + off);
+            const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                x[2 * i] = bf16lo(rw[i]);
+                x[2 * i + 1] = bf16hi(rw[i]);
+            }
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+            for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + p.eps);
+            uint32_t outw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float a = w[2 * i] * x[2 * i] * inv;
+                const float b = w[2 * i + 1] * x[2 * i + 1] * inv;
+                outw[i] = pack_bf16x2(a * cs[i] - b * sn[i], a * sn[i] + b * cs[i]);
+            }
+            if (act) *reinterpret_cast<uint4 *>(p.khat + off) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+        }
+    }
+}
+
+// ============================================================================ attention
+constexpr int kBM = 128;                       // query rows per tile (one per softmax thread)
+constexpr int kBN = 128;                       // keys per K/V tile
+constexpr int kStages = 3;                     // K/V ring depth (tiles)
+constexpr uint32_t kTileBytes = 128 * 128 * 2; // one bf16 128x128 tile
+constexpr uint32_t kBoxBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-byte swizzle span)
+constexpr uint32_t kOffQ = 0;                                   // 2 tiles
+constexpr uint32_t kOffP = kOffQ + 2 * kTileBytes;              // 2 tiles
+constexpr uint32_t kOffKV = kOffP + 2 * kTileBytes;             // kStages tiles
+constexpr uint32_t kOffBar = kOffKV + kStages * kTileBytes;
+enum {
+    BAR_Q_FULL = 0,    // [2] TMA -> softmax WG: raw Q tile landed
+    BAR_Q_READY = 2,   // [2] softmax WG -> MMA: Q tile normed + rotated in place (128 arrivals)
+    BAR_KV_FULL = 4,   // [kStages] TMA -> MMA
+    BAR_KV_EMPTY = 4 + kStages,      // [kStages] MMA (commit) -> TMA
+    BAR_S_FULL = 4 + 2 * kStages,    // [2] MMA (commit) -> softmax WG
+    BAR_P_FULL = 6 + 2 * kStages,    // [2] softmax WG -> MMA (128 arrivals)
+    BAR_O_FULL = 8 + 2 * kStages,    // [2] MMA (commit) -> softmax WG: last P V done
+    BAR_DRAIN = 10 + 2 * kStages,    // MMA drains its own work before TMEM is released
+    NUM_BARS = 11 + 2 * kStages
+};
+constexpr uint32_t kOffTmemSlot = kOffBar + NUM_BARS * 8;
+constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align the base to 1024
+constexpr uint32_t kTmemCols = 512;   // S0 | S1 | O0 | O1, 128 fp32 columns each
+constexpr int kAttnThreads = 384;     // warp 0 TMA, warp 1 MMA, warps 4-7 / 8-11 softmax
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+struct AttnParams {
+    const int32_t *pos;    // [B, T]
+    const float *wq;       // [D]
+    float *out;            // fp32 [B, T, H, D]
+    unsigned *err;
+    int B, T, H, Hkv, hpg, nqb, npairs;
+    float eps;
+    float scale_log2;      // log2(e) / sqrt(D): softmax runs in base 2
+    RopeFreqs rf;
+};
+
+// Shared-memory address of 16-byte chunk c (0..15, i.e. elements 8c..8c+7) of row r of
+// a 128x128 bf16 tile stored as two 128B-swizzled boxes of 64 columns.
+__device__ __forceinline__ uint32_t tile_chunk_addr(uint32_t tile, int r, int c) {
+    return tile + static_cast<uint32_t>(c >> 3) * kBoxBytes + static_cast<uint32_t>(r) * 128u +
+           (static_cast<uint32_t>((c & 7) ^ (r & 7)) << 4);
+}
+
+// S = Q K^T for one 128x128 tile: eight K=16 steps over the head dimension.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t sk, uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = static_cast<uint32_t>(kk >> 2) * kBoxBytes + static_cast<uint32_t>(kk & 3) * 32u;
+        umma_bf16_ss(d_tmem, sw128_desc(sq + off, 16, 1024), sw128_desc(sk + off, 16, 1024), idesc,
+                     kk > 0 ? 1u : 0u);
+    }
+}
+
+// O (+)= P V: eight K=16 steps over the keys.  P is K-major (keys contiguous); V is
+// MN-major (head dim contiguous): its two 64-column boxes are kBoxBytes apart (LBO)
+// and 8-key groups are 1024 bytes apart (SBO).
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t sp, uint32_t sv, uint32_t idesc,
+                                         bool accumulate) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t offp = static_cast<uint32_t>(kk >> 2) * kBoxBytes + static_cast<uint32_t>(kk & 3) * 32u;
+        const uint32_t offv = static_cast<uint32_t>(kk) * 2048u;
+        umma_bf16_ss(d_tmem, sw128_desc(sp + offp, 16, 1024), sw128_desc(sv + offv, kBoxBytes, 1024), idesc,
+                     (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+// RMSNorm (w_q, eps) and RoPE (position ps) of query row r of a raw Q tile, in place.
+__device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, const float *wq, float eps,
+                                                const RopeFreqs &rf) {
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        const uint4 v = ld_shared_v4(tile_chunk_addr(sq, r, c));
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float a = bf16lo(u[i]), b = bf16hi(u[i]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+        }
+    }
+    const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + eps);
+#pragma unroll 2
+    for (int c = 0; c < 16; ++c) {
+        const uint32_t addr = tile_chunk_addr(sq, r, c);
+        const uint4 v = ld_shared_v4(addr);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        const float4 wa = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c);
+        const float4 wb = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c + 1);
+        const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float cs, sn;
+            rope_cos_sin(ps, rf.inv_freq[4 * c + i], cs, sn);
+            const float a = w[2 * i] * bf16lo(u[i]) * inv;
+            const float b = w[2 * i + 1] * bf16hi(u[i]) * inv;
+            o[i] = pack_bf16x2(a * cs - b * sn, a * sn + b * cs);
+        }
+        st_shared_v4(addr, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw_base & 1023u)) & 1023u;
+    uint8_t *smem = smem_raw + pad;
+    const uint32_t sbase = raw_base + pad;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    // ---- work unit: heaviest (latest) query blocks are scheduled first
+    const int per_qb = p.B * p.Hkv * p.npairs;
+    const int job = blockIdx.x;
+    const int qb = p.nqb - 1 - job / per_qb;
+    int rem = job % per_qb;
+    const int pair = rem % p.npairs;
+    rem /= p.npairs;
+    const int g = rem % p.Hkv;
+    const int b = rem / p.Hkv;
+    const int j0 = 2 * pair;
+    const int nslots = min(2, p.hpg - j0);
+    const int hq0 = g * p.hpg + j0;
+    const int n_kv = qb + 1;  // causal: K/V tiles 0 .. qb
+
+    const uint32_t sQ0 = sbase + kOffQ, sP0 = sbase + kOffP, sKV0 = sbase + kOffKV;
+    const uint32_t bar0 = sbase + kOffBar;
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(BAR(BAR_Q_FULL + s), 1);
+            mbar_init(BAR(BAR_Q_READY + s), kBM);
+            mbar_init(BAR(BAR_S_FULL + s), 1);
+            mbar_init(BAR(BAR_P_FULL + s), kBM);
+            mbar_init(BAR(BAR_O_FULL + s), 1);
+        }
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(BAR(BAR_KV_FULL + i), 1);
+            mbar_init(BAR(BAR_KV_EMPTY + i), 1);
+        }
+        mbar_init(BAR(BAR_DRAIN), 1);
+        fence_mbarrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(sbase + kOffTmemSlot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            for (int s = 0; s < nslots; ++s) {
+                const uint32_t dst = sQ0 + s * kTileBytes;
+                mbar_arrive_expect_tx(BAR(BAR_Q_FULL + s), kTileBytes);
+                tma_load_4d(dst, &tm_q, 0, hq0 + s, qb * kBM, b, BAR(BAR_Q_FULL + s));
+                tma_load_4d(dst + kBoxBytes, &tm_q, 64, hq0 + s, qb * kBM, b, BAR(BAR_Q_FULL + s));
+            }
+            int issued = 0;
+            for (int it = 0; it < 2 * n_kv; ++it) {   // K0, V0, K1, V1, ...
+                const int buf = it % kStages, use = it / kStages;
+                if (use > 0 && !mbar_wait(BAR(BAR_KV_EMPTY + buf), (use - 1) & 1, p.err)) {
+                    ok = false;
+                    break;
+                }
+                const CUtensorMap *m = (it & 1) ? &tm_v : &tm_k;
+                const uint32_t dst = sKV0 + buf * kTileBytes;
+                const int row0 = (it >> 1) * kBN;
+                mbar_arrive_expect_tx(BAR(BAR_KV_FULL + buf), kTileBytes);
+                tma_load_4d(dst, m, 0, g, row0, b, BAR(BAR_KV_FULL + buf));
+                tma_load_4d(dst + kBoxBytes, m, 64, g, row0, b, BAR(BAR_KV_FULL + buf));
+                issued = it + 1;
+            }
+            if (!ok) {
+                // Failure path: let every copy still in flight land before the CTA exits.
+                for (int s = 0; s < nslots; ++s) mbar_wait(BAR(BAR_Q_FULL + s), 0, p.err);
+                for (int it = max(0, issued - kStages); it < issued; ++it)
+                    mbar_wait(BAR(BAR_KV_FULL + it % kStages), (it / kStages) & 1, p.err);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_qk = idesc_bf16_f32(kBM, kBN, false);
+            const uint32_t id_pv = idesc_bf16_f32(kBM, kHeadDim, true);
+            bool ok = true;
+            for (int s = 0; s < nslots && ok; ++s) ok = mbar_wait(BAR(BAR_Q_READY + s), 0, p.err);
+            if (ok) ok = mbar_wait(BAR(BAR_KV_FULL + 0), 0, p.err);   // K0
+            if (ok) {
+                tc_fence_after();
+                for (int s = 0; s < nslots; ++s) {
+                    issue_qk(tmem + s * 128, sQ0 + s * kTileBytes, sKV0, id_qk);
+                    umma_commit(BAR(BAR_S_FULL + s));
+                }
+                umma_commit(BAR(BAR_KV_EMPTY + 0));
+            }
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int itv = 2 * j + 1, bv = itv % kStages;
+                const int itk = 2 * j + 2, bk = itk % kStages;
+                const bool more = j + 1 < n_kv;
+                if (!mbar_wait(BAR(BAR_KV_FULL + bv), (itv / kStages) & 1, p.err)) { ok = false; break; }
+                for (int s = 0; s < nslots; ++s) {
+                    if (!mbar_wait(BAR(BAR_P_FULL + s), j & 1, p.err)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(tmem + 256 + s * 128, sP0 + s * kTileBytes, sKV0 + bv * kTileBytes, id_pv, j > 0);
+                    if (more) {
+                        if (s == 0) {
+                            if (!mbar_wait(BAR(BAR_KV_FULL + bk), (itk / kStages) & 1, p.err)) { ok = false; break; }
+                            tc_fence_after();
+                        }
+                        issue_qk(tmem + s * 128, sQ0 + s * kTileBytes, sKV0 + bk * kTileBytes, id_qk);
+                        umma_commit(BAR(BAR_S_FULL + s));
+                    } else {
+                        umma_commit(BAR(BAR_O_FULL + s));
+                    }
+                }
+                if (!ok) break;
+                umma_commit(BAR(BAR_KV_EMPTY + bv));
+                if (more) umma_commit(BAR(BAR_KV_EMPTY + bk));
+            }
+            // Every MMA issued above must finish before TMEM can be released.
+            umma_commit(BAR(BAR_DRAIN));
+            mbar_wait(BAR(BAR_DRAIN), 0, p.err);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int s = (warp - 4) >> 2;
+        const int r = tid - 128 * (1 + s);   // query row in the tile == TMEM lane
+        if (s < nslots) {
+            const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+            const uint32_t tS = tmem + lane_base + s * 128;
+            const uint32_t tO = tmem + lane_base + 256 + s * 128;
+            const uint32_t sQ = sQ0 + s * kTileBytes;
+            const uint32_t sP = sP0 + s * kTileBytes;
+            const int t = qb * kBM + r;
+            const bool valid = t < p.T;
+            const int hq = hq0 + s;
+
+            bool ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_Q_FULL + s), 0, p.err));
+            if (ok) {
+                const int ps = valid ? p.pos[static_cast<size_t>(b) * p.T + t] : 0;
+                transform_q_row(sQ, r, ps, p.wq, p.eps, p.rf);
+                fence_proxy_async_smem();
+                mbar_arrive(BAR(BAR_Q_READY + s));
+            }
+
+            float m_run = -INFINITY;   // running max of scaled scores (base 2), possibly stale by < 8
+            float l_run = 0.f;         // running sum of 2^(score - m_run)
+            for (int j = 0; j < n_kv && ok; ++j) {
+                ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_S_FULL + s), j & 1, p.err));
+                if (!ok) break;
+                tc_fence_after();
+                float x[128];
+                tmem_ld32(tS, x);
+                tmem_ld32(tS + 32, x + 32);
+                tmem_ld32(tS + 64, x + 64);
+                tmem_ld32(tS + 96, x + 96);
+                tmem_wait_ld();
+                if (j == qb) {   // diagonal tile: key c is visible to row r iff c <= r
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (c > r) x[c] = -INFINITY;
+                }
+                float mx = x[0];
+#pragma unroll
+                for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+                const float m_new = fmaxf(m_run, mx * p.scale_log2);
+                // Only move the reference max when it grows by more than 2^8; the final
+                // O / l is exact either way because O and l always share the reference.
+                const bool need = m_new > m_run + 8.0f;
+                const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
+                if (need) m_run = m_new;
+                l_run *= alpha;
+                float lsum = 0.f;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    float e[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        e[u] = ex2_approx(fmaf(x[8 * c + u], p.scale_log2, -m_run));
+                        lsum += e[u];
+                    }
+                    st_shared_v4(tile_chunk_addr(sP, r, c),
+                                 make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
+                                            pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7])));
+                }
+                l_run += lsum;
+                // Rescale this row of O if the reference moved.  Safe: the P V of tile j-1
+                // finished before S of tile j was signalled, and the P V of tile j waits
+                // for P_FULL below.
+                if (__any_sync(0xffffffffu, need) && j > 0) {
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        float o[32];
+                        tmem_ld32(tO + 32 * c, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) o[u] *= alpha;
+                        tmem_st32(tO + 32 * c, o);
+                    }
+                    tmem_wait_st();
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(BAR(BAR_P_FULL + s));
+            }
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_O_FULL + s), 0, p.err));
+            if (ok) {
+                tc_fence_after();
+                const float inv_l = 1.0f / l_run;
+                float *orow = p.out + ((static_cast<size_t>(b) * p.T + t) * p.H + hq) * kHeadDim;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float o[32];
+                    tmem_ld32(tO + 32 * c, o);
+                    tmem_wait_ld();
+                    if (valid) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            reinterpret_cast<float4 *>(orow + 32 * c)[u] =
+                                make_float4(o[4 * u] * inv_l, o[4 * u + 1] * inv_l, o[4 * u + 2] * inv_l,
+                                            o[4 * u + 3] * inv_l);
+                    }
+                }
+            }
+            tc_fence_before();
+        }
+    }
+#undef BAR
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace gqa

@@ -1,0 +1,163 @@
+/*
+ * gqa_attn.h -- C ABI of libgqa_attn.so: the attention sub-block of a Qwen3-style
+ * decoder layer on one NVIDIA B200 (sm_100a):
+ *
+ *     q-hat = RoPE(RMSNorm(q; w_q, eps); pos)      k-hat = RoPE(RMSNorm(k; w_k, eps); pos)
+ *     out   = softmax(q-hat k-hat^T / sqrt(D) + M) V       (M: causal mask, GQA sharing)
+ *
+ * Sources, by page title and section:
+ *   "Qwen3系列1-理论基础&真实结构": D1-4 (softmax(QK^T/sqrt(d_k) + M) V, one softmax per
+ *       row), D1-5 (causal mask: row i sees keys j <= i), D2-1 (RMSNorm), D2-2 (QK-Norm
+ *       per head, then RoPE; V untouched; one weight vector for all Q heads and one for
+ *       all K heads; RoPE as 2x2 rotations of adjacent pairs), D2-3 (GQA; prefill writes
+ *       K/V to the cache and is compute-bound; decode feeds one token and is
+ *       bandwidth-bound).
+ *   "深入剖析Qwen3模型架构": 3.1.2 (GQA via repeat_interleave of K/V over query heads,
+ *       so query head hq reads KV head hq / (H/Hkv); RoPE pairs x[2i], x[2i+1]),
+ *       3.4.1 (RoPE frequencies base^(-2i/D), base raised to 1e6).
+ *   "Qwen3学习日志" section 一 (H query heads in groups of h = H/Hkv sharing a K/V head;
+ *       Hkv = H is MHA, Hkv = 1 is MQA).
+ *   "Qwen3" (nano-vllm walkthrough), "Attention 的 Forward 流程": q/k norm, then rotary
+ *       embedding, then attention that reads and writes the KV cache.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc'd or equivalent) owned by the
+ *     caller; the library allocates nothing, keeps no per-call state and never frees.
+ *   - bf16 tensors are IEEE bfloat16, row-major, contiguous, 16-byte aligned.
+ *   - D (head_dim) must be 128; other values return GQA_ERR_UNSUPPORTED.
+ *   - H % Hkv == 0 is required (GQA_ERR_INVALID_ARG otherwise).
+ *   - RoPE rotates adjacent pairs (x[2i], x[2i+1]) by pos * theta^(-2i/D), i = 0..D/2-1.
+ *   - RMSNorm: w_d * x_d / sqrt(mean(x^2) + eps), over one head vector.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Calls are asynchronous on that stream: they validate host-visible arguments,
+ *     enqueue kernels and return.  They never throw and never synchronize.
+ *   - Argument errors are reported before anything is launched.  Launch failures
+ *     return GQA_ERR_CUDA.  Conditions only the GPU can see (a bounded wait that ran
+ *     out, a device-side length outside its bound) set a device error word, read and
+ *     cleared by gqa_attn_device_status().
+ */
+#ifndef GQA_ATTN_H
+#define GQA_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GQA_OK = 0,
+    GQA_ERR_INVALID_ARG = -1,    /* bad pointer, shape, alignment or value */
+    GQA_ERR_UNSUPPORTED = -2,    /* valid but not implemented (D != 128) */
+    GQA_ERR_WORKSPACE = -3,      /* workspace missing, misaligned or too small */
+    GQA_ERR_CUDA = -4,           /* a CUDA runtime/driver call or a launch failed */
+    GQA_ERR_DEVICE_TIMEOUT = -5, /* a kernel gave up a bounded wait (device status) */
+    GQA_ERR_DEVICE_INPUT = -6    /* a device-side length was out of range (device status) */
+} gqa_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *gqa_status_string(gqa_status status);
+
+/* Workspace bytes gqa_attn_prefill needs for these sizes (k-hat, bf16 [B,T,Hkv,D],
+ * plus alignment).  Returns 0 for an empty problem or invalid sizes. */
+size_t gqa_attn_prefill_workspace_size(int B, int T, int H, int Hkv, int D);
+
+/*
+ * Prefill: causal grouped-query self-attention over whole sequences, with the q/k
+ * RMSNorm and RoPE applied inside ("Qwen3" walkthrough forward steps 4-6;
+ * "Qwen3系列1" D1-4, D1-5, D2-1, D2-2; "深入剖析Qwen3模型架构" 3.1.2, 3.4.1).
+ *
+ *   q        bf16 [B, T, H,   D]   raw (pre-norm, pre-RoPE) queries
+ *   k, v     bf16 [B, T, Hkv, D]   raw keys (normed and rotated here) and values
+ *   pos      int32 [B, T]          RoPE position of every token (only RoPE reads it;
+ *                                  the causal mask is on the token index t)
+ *   qnorm_w, knorm_w  fp32 [D]     RMSNorm weights shared by all Q heads / all K heads
+ *   theta    RoPE base (> 0), e.g. 1e6;   eps  RMSNorm epsilon (>= 0), e.g. 1e-6
+ *   out      fp32 [B, T, H, D]     out[b,t,hq] = sum_{j<=t} p_j v[b,j,hq/(H/Hkv)]
+ *   workspace  device buffer of >= gqa_attn_prefill_workspace_size(...) bytes,
+ *              256-byte aligned; fully overwritten; may be reused between calls
+ *              issued on the same stream.
+ *
+ * B = 0 or T = 0 is a no-op returning GQA_OK.  Calls that overlap on the GPU must not
+ * share a workspace.
+ */
+gqa_status gqa_attn_prefill(const void *q, const void *k, const void *v, const int32_t *pos,
+                            const float *qnorm_w, const float *knorm_w, float theta, float eps,
+                            float *out, int B, int T, int H, int Hkv, int D, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
+ * The two stages of gqa_attn_prefill, callable on their own (gqa_attn_prefill is
+ * exactly gqa_attn_k_norm_rope into its workspace followed by gqa_attn_prefill_khat).
+ *
+ * gqa_attn_k_norm_rope: k_hat = RoPE(RMSNorm(k; knorm_w, eps); pos), written as bf16
+ * in the layout of k.  These are the keys the KV cache holds ("Qwen3系列1" D2-3: K is
+ * written to the cache after its norm and rotation, before attention), so the output
+ * can be a decode cache directly.
+ *   k      bf16 [N, Hkv, D] (N = B*T tokens, any token order); pos int32 [N]
+ *   k_hat  bf16 [N, Hkv, D], must not overlap k.   N = 0 is a no-op.
+ */
+gqa_status gqa_attn_k_norm_rope(const void *k, const int32_t *pos, const float *knorm_w, float theta,
+                                float eps, void *k_hat, int64_t N, int Hkv, int D, void *stream);
+
+/*
+ * gqa_attn_prefill_khat: the attention stage of gqa_attn_prefill on keys that are
+ * already normed and rotated (k_hat, e.g. from gqa_attn_k_norm_rope): the raw q tiles
+ * are normed (qnorm_w, eps) and rotated (pos, theta) inside the attention kernel.
+ * Arguments as for gqa_attn_prefill; k_hat is bf16 [B, T, Hkv, D].  Needs no workspace.
+ */
+gqa_status gqa_attn_prefill_khat(const void *q, const void *k_hat, const void *v, const int32_t *pos,
+                                 const float *qnorm_w, float theta, float eps, float *out, int B, int T,
+                                 int H, int Hkv, int D, void *stream);
+
+/* Workspace bytes gqa_attn_decode needs: split-KV partial results for up to max_len
+ * cached tokens per sequence.  Returns 0 for an empty problem or invalid sizes. */
+size_t gqa_attn_decode_workspace_size(int B, int H, int Hkv, int D, int max_len);
+
+/*
+ * Decode: one new query token per sequence attends to that sequence's KV cache
+ * ("Qwen3系列1" D2-3: the cache holds K and V per KV head, written before attention;
+ * decode feeds a single token and is bound by reading the cache).
+ *
+ *   q         bf16 [B, H, D]        raw query of the new token; RMSNorm(qnorm_w, eps) and
+ *                                   RoPE at position q_pos[b] are applied here
+ *   k_cache   bf16 [rows, Hkv, D]   cached keys, already normed and rotated
+ *   v_cache   bf16 [rows, Hkv, D]   cached values
+ *   cache_offsets int64 [B + 1]     sequence b owns rows cache_offsets[b] ..
+ *                                   cache_offsets[b+1]-1 (non-decreasing)
+ *   seqlens   int32 [B]             number of valid cached rows of sequence b:
+ *                                   1 <= seqlens[b] <= max_len and
+ *                                   seqlens[b] <= cache_offsets[b+1] - cache_offsets[b];
+ *                                   every one of them is visible to the query
+ *   q_pos     int32 [B] or NULL     RoPE position of the query (NULL: seqlens[b])
+ *   out       fp32 [B, H, D]
+ *   max_len   host-side upper bound on seqlens (sizes the workspace)
+ *   workspace >= gqa_attn_decode_workspace_size(B, H, Hkv, D, max_len) bytes,
+ *             256-byte aligned; fully overwritten each call.
+ *
+ * cache_offsets, seqlens and q_pos live on the device, so their values are checked on
+ * the device: a sequence that breaks the bounds above gets NaN output, reads nothing
+ * outside its rows, and sets GQA_ERR_DEVICE_INPUT in the device status word.
+ * B = 0 is a no-op returning GQA_OK.
+ */
+gqa_status gqa_attn_decode(const void *q, const void *k_cache, const void *v_cache,
+                           const int64_t *cache_offsets, const int32_t *seqlens,
+                           const int32_t *q_pos, const float *qnorm_w, float theta, float eps,
+                           float *out, int B, int H, int Hkv, int D, int max_len,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Device status: waits for `stream` (a cudaStream_t as void*, NULL = legacy default
+ * stream), then reads and clears the library's device error word on the current
+ * device.  Returns GQA_OK, GQA_ERR_DEVICE_TIMEOUT (a kernel gave up a bounded wait and
+ * returned early; its outputs are invalid), GQA_ERR_DEVICE_INPUT (a decode sequence
+ * broke its length bounds), or GQA_ERR_CUDA.  This is the only synchronizing call.
+ */
+gqa_status gqa_attn_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_ATTN_H */

@@ -1,0 +1,118 @@
+"""The C-ABI library loads, exports every symbol its header declares, and rejects bad
+arguments on the host before anything reaches a GPU (no compute calls: CPU only)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from grouped_query_causal_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqa_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def _declared():
+    text = open(HEADER, encoding="utf-8").read()
+    return sorted(set(re.findall(r"\b(gqa_\w+)\s*\(", text)))
+
+
+def test_header_declares_what_the_binding_names():
+    assert _declared() == sorted(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in _declared():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+    # nothing but the C ABI is exported
+    assert {n for n in exported if n.startswith("gqa")} == set(_declared())
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS_NAMES.items():
+        assert lib.gqa_status_string(code).decode() == name
+
+
+def test_workspace_sizes(lib):
+    assert lib.gqa_attn_prefill_workspace_size(4, 4096, 32, 8, 128) == 4 * 4096 * 8 * 128 * 2
+    assert lib.gqa_attn_prefill_workspace_size(1, 3, 2, 1, 128) == 3 * 128 * 2
+    assert lib.gqa_attn_prefill_workspace_size(1, 128, 16, 8, 64) == 0
+    assert lib.gqa_attn_prefill_workspace_size(1, 128, 16, 3, 128) == 0
+    assert lib.gqa_attn_prefill_workspace_size(0, 128, 16, 8, 128) == 0
+    slots = 64 * 64 * 32
+    assert lib.gqa_attn_decode_workspace_size(64, 32, 8, 128, 32768) == slots * 128 * 4 + slots * 2 * 4
+    assert lib.gqa_attn_decode_workspace_size(2, 8, 2, 128, 1) == 2 * 8 * 128 * 4 + 256
+    assert lib.gqa_attn_decode_workspace_size(2, 8, 3, 128, 100) == 0
+    assert lib.gqa_attn_decode_workspace_size(2, 8, 2, 128, 0) == 0
+
+
+def _prefill(lib, **kw):
+    a = dict(q=16, k=16, v=16, pos=16, wq=16, wk=16, theta=1e6, eps=1e-6, out=16, B=1, T=8, H=4, Hkv=2, D=128,
+             ws=256, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return lib.gqa_attn_prefill(a["q"], a["k"], a["v"], a["pos"], a["wq"], a["wk"], a["theta"], a["eps"],
+                                a["out"], a["B"], a["T"], a["H"], a["Hkv"], a["D"], a["ws"], a["wsb"],
+                                a["stream"])
+
+
+def test_prefill_argument_errors_are_caught_on_the_host(lib):
+    # these return before any CUDA call (the pointers are never dereferenced)
+    assert _prefill(lib, D=64) == -2
+    assert _prefill(lib, D=0) == -1
+    assert _prefill(lib, H=5, Hkv=2) == -1
+    assert _prefill(lib, Hkv=0) == -1
+    assert _prefill(lib, B=-1) == -1
+    assert _prefill(lib, theta=0.0) == -1
+    assert _prefill(lib, theta=float("nan")) == -1
+    assert _prefill(lib, eps=-1.0) == -1
+    assert _prefill(lib, q=None) == -1
+    assert _prefill(lib, out=None) == -1
+    assert _prefill(lib, k=24) == -1        # misaligned
+    assert _prefill(lib, ws=None) == -3
+    assert _prefill(lib, ws=128) == -3      # workspace not 256-aligned
+    assert _prefill(lib, wsb=100) == -3     # too small
+    assert _prefill(lib, B=0) == 0          # empty: no-op
+    assert _prefill(lib, T=0, q=None) == 0
+
+
+def _decode(lib, **kw):
+    a = dict(q=16, kc=16, vc=16, offs=16, sl=16, qpos=None, wq=16, theta=1e6, eps=1e-6, out=16, B=2, H=8,
+             Hkv=2, D=128, max_len=100, ws=256, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return lib.gqa_attn_decode(a["q"], a["kc"], a["vc"], a["offs"], a["sl"], a["qpos"], a["wq"], a["theta"],
+                               a["eps"], a["out"], a["B"], a["H"], a["Hkv"], a["D"], a["max_len"], a["ws"],
+                               a["wsb"], a["stream"])
+
+
+def test_decode_argument_errors_are_caught_on_the_host(lib):
+    assert _decode(lib, D=256) == -2
+    assert _decode(lib, H=8, Hkv=3) == -1
+    assert _decode(lib, max_len=0) == -1
+    assert _decode(lib, max_len=1 << 30) == -1   # more chunks than a grid dimension holds
+    assert _decode(lib, kc=None) == -1
+    assert _decode(lib, offs=20) == -1          # int64 offsets must be 8-byte aligned
+    assert _decode(lib, qpos=18) == -1
+    assert _decode(lib, eps=float("inf")) == -1
+    assert _decode(lib, wsb=10) == -3
+    assert _decode(lib, B=0) == 0
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    saved = binding._lib
+    binding._lib = None
+    try:
+        with pytest.raises(RuntimeError):
+            binding.load(str(tmp_path / "missing.so"))
+    finally:
+        binding._lib = saved

@@ -1,0 +1,129 @@
+"""GPU parity of gqa_attn_prefill against the fp64 oracle (called through the C ABI
+via the ctypes binding).  Tolerance: max-abs 2e-2 and mean-abs 2e-3 per element."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle
+from grouped_query_causal_b200 import synthetic
+from tests.gpu_helpers import (assert_close, bits as bits_of, oracle_prefill_args, sample_rows, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def gqa():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu tests")
+    from grouped_query_causal_b200 import binding
+    binding.load()
+    return binding
+
+
+def _run(gqa, inp):
+    d = to_dev(inp)
+    out = gqa.prefill(d["q"], d["k"], d["v"], d["pos"], d["qnorm_w"], d["knorm_w"], d["theta"], d["eps"])
+    torch.cuda.synchronize()
+    gqa.check_device_status()
+    return out.cpu().numpy()
+
+
+def test_prefill_correctness_config(gqa):
+    """B=1, T=128, H=16, Hkv=8 (one query block, one diagonal tile) in full."""
+    inp = synthetic.make("prefill_correctness")
+    got = _run(gqa, inp)
+    ref = oracle.prefill(*oracle_prefill_args(inp))
+    assert_close(got, ref, "prefill_correctness")
+
+
+@pytest.mark.parametrize("name", ["gqa_sweep_mha", "gqa_sweep_hkv8", "gqa_sweep_hkv4", "gqa_sweep_mqa"])
+def test_gqa_degeneracy_sweep(gqa, name):
+    """B=2, T=512, H=16 with Hkv in {16 (MHA), 8, 4, 1 (MQA)}, every output element."""
+    inp = synthetic.make(name)
+    got = _run(gqa, inp)
+    ref = oracle.prefill(*oracle_prefill_args(inp))
+    assert_close(got, ref, name)
+
+
+@pytest.mark.parametrize("B,T,H,Hkv", [(1, 1, 2, 1), (2, 7, 4, 2), (1, 129, 6, 2), (2, 200, 3, 1),
+                                       (1, 383, 8, 8), (3, 130, 10, 2), (1, 257, 16, 2)])
+def test_ragged_and_odd_groups(gqa, B, T, H, Hkv):
+    """Ragged T (partial last query/key tile), odd heads per group, single token."""
+    inp = synthetic.prefill_inputs(B, T, H, Hkv, seed=B * 1000 + T)
+    got = _run(gqa, inp)
+    ref = oracle.prefill(*oracle_prefill_args(inp))
+    assert_close(got, ref, f"B{B} T{T} H{H} Hkv{Hkv}")
+
+
+def test_positions_drive_rope_only(gqa):
+    """Arbitrary (non-contiguous, large) positions: RoPE uses pos, the mask uses the index."""
+    inp = synthetic.prefill_inputs(2, 160, 8, 2, seed=77)
+    g = torch.Generator().manual_seed(78)
+    inp.pos = torch.randint(0, 32768, (2, 160), generator=g, dtype=torch.int32)
+    got = _run(gqa, inp)
+    ref = oracle.prefill(*oracle_prefill_args(inp))
+    assert_close(got, ref, "random positions")
+
+
+def test_deterministic(gqa):
+    inp = synthetic.prefill_inputs(1, 300, 8, 2, seed=5)
+    a = _run(gqa, inp)
+    b = _run(gqa, inp)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_large_prefill_sampled_rows(gqa):
+    """B=4, T=4096, H=32, Hkv=8, inputs x0.5, in the launch configuration the benchmark
+    times; checked on sampled rows the oracle computes one by one."""
+    inp = synthetic.make("large_prefill")
+    got = _run(gqa, inp)
+    rows = sample_rows(4, 4096, 32, n_random=96, seed=1)
+    ref = oracle.prefill_rows(*oracle_prefill_args(inp), rows)
+    assert_close(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, "large_prefill rows")
+    assert np.isfinite(got).all()
+
+
+def test_long_context_prefill_sampled_rows(gqa):
+    """B=1, T=32768, H=64, Hkv=8: sampled rows (incl. the last, longest ones)."""
+    inp = synthetic.make("long_context_prefill")
+    got = _run(gqa, inp)
+    rows = sample_rows(1, 32768, 64, n_random=24, seed=2)
+    ref = oracle.prefill_rows(*oracle_prefill_args(inp), rows)
+    assert_close(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, "long_context rows")
+    assert np.isfinite(got).all()
+
+
+def test_empty_problem_is_noop(gqa):
+    dev = "cuda"
+    q = torch.empty((0, 5, 4, 128), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((0, 5, 2, 128), dtype=torch.bfloat16, device=dev)
+    pos = torch.empty((0, 5), dtype=torch.int32, device=dev)
+    w = torch.ones(128, device=dev)
+    out = gqa.prefill(q, k, k, pos, w, w)
+    assert out.shape == (0, 5, 4, 128)
+
+
+def test_k_norm_rope_matches_oracle_k_hat(gqa):
+    """The k-hat stage on its own (the decode-cache writer): bf16 output within one bf16
+    rounding of the oracle's k-hat, at positions up to 32767."""
+    inp = synthetic.prefill_inputs(2, 300, 4, 4, seed=31)
+    g = torch.Generator().manual_seed(32)
+    inp.pos = torch.randint(0, 32768, (2, 300), generator=g, dtype=torch.int32)
+    khat = gqa.k_norm_rope(inp.k.cuda(), inp.pos.cuda(), inp.wk.cuda(), inp.theta, inp.eps)
+    torch.cuda.synchronize()
+    ntok = 2 * 300
+    ref = oracle.qk_transform(bits_of(inp.k).reshape(ntok, 4, 128), inp.pos.numpy().reshape(ntok), inp.wk.numpy(),
+                              inp.theta, inp.eps).reshape(2, 300, 4, 128)
+    got = khat.float().cpu().numpy()
+    # one bf16 rounding (2^-9 relative) plus fp32 arithmetic
+    assert (np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-5).all()
+
+
+def test_two_stage_prefill_equals_one_call(gqa):
+    inp = synthetic.prefill_inputs(2, 190, 8, 2, seed=33)
+    d = to_dev(inp)
+    one = gqa.prefill(d["q"], d["k"], d["v"], d["pos"], d["qnorm_w"], d["knorm_w"], d["theta"], d["eps"])
+    khat = gqa.k_norm_rope(d["k"], d["pos"], d["knorm_w"], d["theta"], d["eps"])
+    two = gqa.prefill_khat(d["q"], khat, d["v"], d["pos"], d["qnorm_w"], d["theta"], d["eps"])
+    torch.cuda.synchronize()
+    assert torch.equal(one, two)
