@@ -23,7 +23,9 @@ STATUS_NAMES = {
 # Every symbol the header declares.
 EXPORTS = ("gqa_status_string", "gqa_attn_prefill_workspace_size", "gqa_attn_prefill",
            "gqa_attn_k_norm_rope", "gqa_attn_prefill_khat", "gqa_attn_decode_workspace_size",
-           "gqa_attn_decode", "gqa_attn_device_status")
+           "gqa_attn_decode", "gqa_attn_decode_noalloc", "gqa_attn_device_status")
+# Size of the library's built-in scratch used by gqa_attn_decode_noalloc.
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class GqaError(RuntimeError):
@@ -58,6 +60,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_attn_decode_workspace_size.restype = Z
     lib.gqa_attn_decode.argtypes = [P, P, P, P, P, P, P, F, F, P, I, I, I, I, I, P, Z, P]
     lib.gqa_attn_decode.restype = I
+    lib.gqa_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, P, F, F, P, I, I, I, I, I, P]
+    lib.gqa_attn_decode_noalloc.restype = I
     lib.gqa_attn_device_status.argtypes = [P]
     lib.gqa_attn_device_status.restype = I
     _lib = lib
@@ -207,6 +211,34 @@ def decode(q, k_cache, v_cache, cache_offsets, seqlens, qnorm_w, max_len: int,
                              int(max_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
                              _stream_handle(stream))
     _raise(st, "gqa_attn_decode")
+    return out
+
+
+def decode_noalloc(q, k_cache, v_cache, cache_offsets, seqlens, qnorm_w, max_len: int,
+                   q_pos: Optional[torch.Tensor] = None, theta: float = 1.0e6, eps: float = 1e-6,
+                   out: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """decode() without a workspace, for callers that cannot allocate one: the library's
+    built-in scratch (NOALLOC_SCRATCH_BYTES per GPU) holds the partial results.  Calls
+    that overlap on the GPU share that scratch and must be serialized."""
+    lib = load()
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 3)
+    _check(v_cache, "v_cache", torch.bfloat16, 3)
+    _check(cache_offsets, "cache_offsets", torch.int64, 1)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    _check(qnorm_w, "qnorm_w", torch.float32, 1)
+    if q_pos is not None:
+        _check(q_pos, "q_pos", torch.int32, 1)
+    B, H, D = q.shape
+    Hkv = k_cache.shape[1]
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 3)
+    st = lib.gqa_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_offsets), _ptr(seqlens),
+                                     _ptr(q_pos), _ptr(qnorm_w), float(theta), float(eps), _ptr(out), B, H, Hkv, D,
+                                     int(max_len), _stream_handle(stream))
+    _raise(st, "gqa_attn_decode_noalloc")
     return out
 
 

@@ -325,6 +325,46 @@ extern "C" gqa_status gqa_attn_decode(const void *q, const void *k_cache, const 
     return launch_decode<8>(p, (h + 7) / 8, st);
 }
 
+namespace {
+
+// Scratch for gqa_attn_decode_noalloc: part of the library's own device image, so no
+// call ever allocates.  Host code must not use the symbol's host-side address; the
+// device address comes from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GQA_NOALLOC_SCRATCH_BYTES];
+
+void *noalloc_scratch_address() {
+    static std::atomic<void *> cache[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0) return nullptr;
+    void *p = cache[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || addr == nullptr) return nullptr;
+    cache[dev].store(addr, std::memory_order_release);
+    return addr;
+}
+
+}  // namespace
+
+extern "C" gqa_status gqa_attn_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                              const int64_t *cache_offsets, const int32_t *seqlens,
+                                              const int32_t *q_pos, const float *qnorm_w, float theta, float eps,
+                                              float *out, int B, int H, int Hkv, int D, int max_len,
+                                              void *stream) {
+    if (D == kHeadDim && B > 0 && H > 0 && Hkv > 0 && H % Hkv == 0 && max_len > 0 &&
+        gqa_attn_decode_workspace_size(B, H, Hkv, D, max_len) > GQA_NOALLOC_SCRATCH_BYTES)
+        return GQA_ERR_WORKSPACE;
+    // Every other argument check is gqa_attn_decode's; the scratch address is only
+    // looked up when there is work to launch.
+    if (D != kHeadDim || B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0 || max_len <= 0)
+        return gqa_attn_decode(q, k_cache, v_cache, cache_offsets, seqlens, q_pos, qnorm_w, theta, eps, out, B, H,
+                               Hkv, D, max_len, nullptr, 0, stream);
+    void *scratch = noalloc_scratch_address();
+    if (!scratch) return GQA_ERR_CUDA;
+    return gqa_attn_decode(q, k_cache, v_cache, cache_offsets, seqlens, q_pos, qnorm_w, theta, eps, out, B, H, Hkv,
+                           D, max_len, scratch, GQA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 extern "C" gqa_status gqa_attn_device_status(void *stream) {
     unsigned *err = device_error_word();
     if (!err) return GQA_ERR_CUDA;

@@ -147,6 +147,36 @@ gqa_status gqa_attn_decode(const void *q, const void *k_cache, const void *v_cac
                            float *out, int B, int H, int Hkv, int D, int max_len,
                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* Size of the library's built-in decode scratch used by gqa_attn_decode_noalloc. */
+#define GQA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * gqa_attn_decode_noalloc: gqa_attn_decode for callers that cannot hand the library a
+ * workspace and cannot allocate one, for example a plugin running inside a host
+ * framework that owns every byte of device memory, or a latency-critical serving loop
+ * that must not call cudaMalloc (which may synchronize the device).  The pages have no
+ * counterpart of this entry point; it exists only for such callers.
+ *
+ * Same arguments, results and device-side checks as gqa_attn_decode, minus the
+ * workspace: the split-KV partial results go to a scratch array that is part of the
+ * library itself (GQA_NOALLOC_SCRATCH_BYTES of device memory that every GPU which
+ * loads the library holds until the process exits).  No call allocates or frees.
+ *   - Problems whose partials need more than GQA_NOALLOC_SCRATCH_BYTES, i.e.
+ *     gqa_attn_decode_workspace_size(B, H, Hkv, D, max_len) > GQA_NOALLOC_SCRATCH_BYTES,
+ *     are rejected with GQA_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the scratch array's device address (once per
+ *     device, with that device current); make that first call before any stream capture.
+ *   - All calls on a device share the one scratch array, and it keeps the last call's
+ *     contents (nothing in it has to start at zero).  Calls that overlap on the GPU
+ *     (different streams without ordering between them) race on it and give undefined
+ *     results: serialize them.
+ */
+gqa_status gqa_attn_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                   const int64_t *cache_offsets, const int32_t *seqlens,
+                                   const int32_t *q_pos, const float *qnorm_w, float theta,
+                                   float eps, float *out, int B, int H, int Hkv, int D,
+                                   int max_len, void *stream);
+
 /*
  * Device status: waits for `stream` (a cudaStream_t as void*, NULL = legacy default
  * stream), then reads and clears the library's device error word on the current
