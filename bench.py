@@ -163,6 +163,7 @@ def run_ours(args, rank, world, local_rank):
     q, k, v, pos = pin.q.to(dev), pin.k.to(dev), pin.v.to(dev), pin.pos.to(dev)
     wq, wk = pin.wq.to(dev), pin.wk.to(dev)
     khat = torch.empty_like(k)
+    rope_cs = torch.empty((B, T, D), dtype=torch.float32, device=dev)
     out = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
     dq, kc, vc = dec.q.to(dev), dec.k_cache.to(dev), dec.v_cache.to(dev)
     offs, sl, dwq = dec.offsets.to(dev), dec.seqlens.to(dev), dec.wq.to(dev)
@@ -173,11 +174,12 @@ def run_ours(args, rank, world, local_rank):
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        st = lib.gqa_attn_k_norm_rope(ptr(k), ptr(pos), ptr(wk), pin.theta, pin.eps, ptr(khat), B * T, Hkv, D, sh)
+        st = lib.gqa_attn_k_norm_rope(ptr(k), ptr(pos), ptr(wk), pin.theta, pin.eps, ptr(khat), ptr(rope_cs), B * T,
+                                      Hkv, D, sh)
         if ev:
             ev[1].record(stream)
-        st |= lib.gqa_attn_prefill_khat(ptr(q), ptr(khat), ptr(v), ptr(pos), ptr(wq), pin.theta, pin.eps, ptr(out),
-                                        B, T, H, Hkv, D, sh)
+        st |= lib.gqa_attn_prefill_khat(ptr(q), ptr(khat), ptr(v), ptr(pos), ptr(rope_cs), ptr(wq), pin.theta,
+                                        pin.eps, ptr(out), B, T, H, Hkv, D, sh)
         if ev:
             ev[2].record(stream)
         st |= lib.gqa_attn_decode(ptr(dq), ptr(kc), ptr(vc), ptr(offs), ptr(sl), None, ptr(dwq), dec.theta, dec.eps,

@@ -52,9 +52,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_attn_prefill_workspace_size.restype = Z
     lib.gqa_attn_prefill.argtypes = [P, P, P, P, P, P, F, F, P, I, I, I, I, I, P, Z, P]
     lib.gqa_attn_prefill.restype = I
-    lib.gqa_attn_k_norm_rope.argtypes = [P, P, P, F, F, P, ctypes.c_int64, I, I, P]
+    lib.gqa_attn_k_norm_rope.argtypes = [P, P, P, F, F, P, P, ctypes.c_int64, I, I, P]
     lib.gqa_attn_k_norm_rope.restype = I
-    lib.gqa_attn_prefill_khat.argtypes = [P, P, P, P, P, F, F, P, I, I, I, I, I, P]
+    lib.gqa_attn_prefill_khat.argtypes = [P, P, P, P, P, P, F, F, P, I, I, I, I, I, P]
     lib.gqa_attn_prefill_khat.restype = I
     lib.gqa_attn_decode_workspace_size.argtypes = [I, I, I, I, I]
     lib.gqa_attn_decode_workspace_size.restype = Z
@@ -135,10 +135,12 @@ def prefill(q, k, v, pos, qnorm_w, knorm_w, theta: float = 1.0e6, eps: float = 1
 
 
 def k_norm_rope(k, pos, knorm_w, theta: float = 1.0e6, eps: float = 1e-6,
-                out: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, rope_cs: Optional[torch.Tensor] = None,
                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """k-hat = RoPE(RMSNorm(k)) in bf16.  k [..., Hkv, D] bf16 with one position per
-    token (pos has the leading shape of k) -> k_hat of k's shape (a decode cache)."""
+    token (pos has the leading shape of k) -> k_hat of k's shape (a decode cache).
+    rope_cs (fp32 [..., D/2, 2] over the same tokens), when given, receives the tokens'
+    RoPE cos/sin for prefill_khat to reuse."""
     lib = load()
     if k.dtype != torch.bfloat16 or not k.is_cuda or not k.is_contiguous() or k.dim() < 2:
         raise ValueError("k must be a contiguous CUDA bf16 tensor [..., Hkv, D]")
@@ -147,18 +149,22 @@ def k_norm_rope(k, pos, knorm_w, theta: float = 1.0e6, eps: float = 1e-6,
     N = k.numel() // (Hkv * D) if k.numel() else 0
     if pos.dtype != torch.int32 or not pos.is_cuda or not pos.is_contiguous() or pos.numel() != N:
         raise ValueError("pos must be a contiguous CUDA int32 tensor with one entry per token")
+    if rope_cs is not None and (rope_cs.dtype != torch.float32 or not rope_cs.is_cuda or not rope_cs.is_contiguous()
+                                or rope_cs.numel() != N * D):
+        raise ValueError("rope_cs must be a contiguous CUDA fp32 tensor of N * D elements")
     if out is None:
         out = torch.empty_like(k)
-    st = lib.gqa_attn_k_norm_rope(_ptr(k), _ptr(pos), _ptr(knorm_w), float(theta), float(eps), _ptr(out), N,
-                                  Hkv, D, _stream_handle(stream))
+    st = lib.gqa_attn_k_norm_rope(_ptr(k), _ptr(pos), _ptr(knorm_w), float(theta), float(eps), _ptr(out),
+                                  _ptr(rope_cs), N, Hkv, D, _stream_handle(stream))
     _raise(st, "gqa_attn_k_norm_rope")
     return out
 
 
 def prefill_khat(q, k_hat, v, pos, qnorm_w, theta: float = 1.0e6, eps: float = 1e-6,
-                 out: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None, rope_cs: Optional[torch.Tensor] = None,
                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """Attention stage of prefill on already normed + rotated keys (k_hat [B,T,Hkv,D])."""
+    """Attention stage of prefill on already normed + rotated keys (k_hat [B,T,Hkv,D]);
+    rope_cs is the cos/sin table k_norm_rope wrote for the same tokens, or None."""
     lib = load()
     _check(q, "q", torch.bfloat16, 4)
     _check(k_hat, "k_hat", torch.bfloat16, 4)
@@ -172,8 +178,11 @@ def prefill_khat(q, k_hat, v, pos, qnorm_w, theta: float = 1.0e6, eps: float = 1
     if out is None:
         out = torch.empty((B, T, H, D), dtype=torch.float32, device=q.device)
     _check(out, "out", torch.float32, 4)
-    st = lib.gqa_attn_prefill_khat(_ptr(q), _ptr(k_hat), _ptr(v), _ptr(pos), _ptr(qnorm_w), float(theta),
-                                   float(eps), _ptr(out), B, T, H, Hkv, D, _stream_handle(stream))
+    if rope_cs is not None and (rope_cs.dtype != torch.float32 or not rope_cs.is_cuda or not rope_cs.is_contiguous()
+                                or rope_cs.numel() != B * T * D):
+        raise ValueError("rope_cs must be a contiguous CUDA fp32 tensor of B * T * D elements")
+    st = lib.gqa_attn_prefill_khat(_ptr(q), _ptr(k_hat), _ptr(v), _ptr(pos), _ptr(rope_cs), _ptr(qnorm_w),
+                                   float(theta), float(eps), _ptr(out), B, T, H, Hkv, D, _stream_handle(stream))
     _raise(st, "gqa_attn_prefill_khat")
     return out
 

@@ -137,9 +137,16 @@ extern "C" const char *gqa_status_string(gqa_status status) {
     return "GQA_UNKNOWN_STATUS";
 }
 
+namespace {
+// Workspace of gqa_attn_prefill: k-hat (bf16 [B,T,Hkv,D]), then the per-token RoPE
+// cos/sin table (fp32 [B,T,D/2,2]).
+size_t khat_bytes(int B, int T, int Hkv) { return round_up(static_cast<size_t>(B) * T * Hkv * kHeadDim * 2, 256); }
+size_t rope_table_bytes(int B, int T) { return round_up(static_cast<size_t>(B) * T * kHeadDim * sizeof(float), 256); }
+}  // namespace
+
 extern "C" size_t gqa_attn_prefill_workspace_size(int B, int T, int H, int Hkv, int D) {
     if (D != kHeadDim || !prefill_shape_ok(B, T, H, Hkv) || B == 0 || T == 0) return 0;
-    return round_up(static_cast<size_t>(B) * T * Hkv * kHeadDim * 2, 256);
+    return khat_bytes(B, T, Hkv) + rope_table_bytes(B, T);
 }
 
 namespace {
@@ -150,12 +157,13 @@ bool params_ok(float theta, float eps) {
 
 // Enqueue the k-hat prologue (arguments already validated).
 gqa_status launch_k_norm_rope(const void *k, const int32_t *pos, const float *knorm_w, const RopeFreqs &rf,
-                              float eps, void *k_hat, long long ntok, int Hkv, cudaStream_t st) {
+                              float eps, void *k_hat, float *rope_cs, long long ntok, int Hkv, cudaStream_t st) {
     KPrologueParams kp;
     kp.k = static_cast<const uint16_t *>(k);
     kp.pos = pos;
     kp.wk = knorm_w;
     kp.khat = static_cast<uint16_t *>(k_hat);
+    kp.rope_cs = rope_cs;
     kp.ntok = ntok;
     kp.Hkv = Hkv;
     kp.eps = eps;
@@ -169,8 +177,8 @@ gqa_status launch_k_norm_rope(const void *k, const int32_t *pos, const float *kn
 
 // Enqueue the attention kernel (arguments already validated).
 gqa_status launch_attention(const void *q, const void *k_hat, const void *v, const int32_t *pos,
-                            const float *qnorm_w, const RopeFreqs &rf, float eps, float *out, int B, int T,
-                            int H, int Hkv, cudaStream_t st) {
+                            const float *rope_cs, const float *qnorm_w, const RopeFreqs &rf, float eps, float *out,
+                            int B, int T, int H, int Hkv, cudaStream_t st) {
     unsigned *err = device_error_word();
     if (!err) return GQA_ERR_CUDA;
     CUtensorMap tm_q, tm_k, tm_v;
@@ -180,6 +188,7 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
     if (!attn_smem_attr_set()) return GQA_ERR_CUDA;
     AttnParams ap;
     ap.pos = pos;
+    ap.rope_cs = rope_cs;
     ap.wq = qnorm_w;
     ap.out = out;
     ap.err = err;
@@ -202,34 +211,41 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
 }  // namespace
 
 extern "C" gqa_status gqa_attn_k_norm_rope(const void *k, const int32_t *pos, const float *knorm_w, float theta,
-                                           float eps, void *k_hat, int64_t N, int Hkv, int D, void *stream) {
+                                           float eps, void *k_hat, float *rope_cs, int64_t N, int Hkv, int D,
+                                           void *stream) {
     if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
     if (N < 0 || Hkv <= 0 || N > (1LL << 31)) return GQA_ERR_INVALID_ARG;
     if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
     if (N == 0) return GQA_OK;
     if (!k || !pos || !knorm_w || !k_hat) return GQA_ERR_INVALID_ARG;
-    if (!aligned(k, 16) || !aligned(k_hat, 16) || !aligned(knorm_w, 16) || !aligned(pos, 4))
+    if (!aligned(k, 16) || !aligned(k_hat, 16) || !aligned(knorm_w, 16) || !aligned(pos, 4) ||
+        (rope_cs && !aligned(rope_cs, 16)))
         return GQA_ERR_INVALID_ARG;
     const size_t bytes = static_cast<size_t>(N) * Hkv * kHeadDim * 2;
     const uintptr_t a = reinterpret_cast<uintptr_t>(k), b = reinterpret_cast<uintptr_t>(k_hat);
     if (a < b + bytes && b < a + bytes) return GQA_ERR_INVALID_ARG;   // overlapping buffers
-    return launch_k_norm_rope(k, pos, knorm_w, rope_freqs(static_cast<double>(theta)), eps, k_hat, N, Hkv,
+    if (rope_cs) {
+        const uintptr_t c = reinterpret_cast<uintptr_t>(rope_cs);
+        const size_t tb = static_cast<size_t>(N) * kHeadDim * sizeof(float);
+        if ((c < b + bytes && b < c + tb) || (c < a + bytes && a < c + tb)) return GQA_ERR_INVALID_ARG;
+    }
+    return launch_k_norm_rope(k, pos, knorm_w, rope_freqs(static_cast<double>(theta)), eps, k_hat, rope_cs, N, Hkv,
                               static_cast<cudaStream_t>(stream));
 }
 
 extern "C" gqa_status gqa_attn_prefill_khat(const void *q, const void *k_hat, const void *v, const int32_t *pos,
-                                            const float *qnorm_w, float theta, float eps, float *out, int B,
-                                            int T, int H, int Hkv, int D, void *stream) {
+                                            const float *rope_cs, const float *qnorm_w, float theta, float eps,
+                                            float *out, int B, int T, int H, int Hkv, int D, void *stream) {
     if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
     if (!prefill_shape_ok(B, T, H, Hkv)) return GQA_ERR_INVALID_ARG;
     if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
     if (B == 0 || T == 0) return GQA_OK;
     if (!q || !k_hat || !v || !pos || !qnorm_w || !out) return GQA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k_hat, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(qnorm_w, 16) ||
-        !aligned(pos, 4))
+        !aligned(pos, 4) || (rope_cs && !aligned(rope_cs, 16)))
         return GQA_ERR_INVALID_ARG;
-    return launch_attention(q, k_hat, v, pos, qnorm_w, rope_freqs(static_cast<double>(theta)), eps, out, B, T, H,
-                            Hkv, static_cast<cudaStream_t>(stream));
+    return launch_attention(q, k_hat, v, pos, rope_cs, qnorm_w, rope_freqs(static_cast<double>(theta)), eps, out, B,
+                            T, H, Hkv, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" gqa_status gqa_attn_prefill(const void *q, const void *k, const void *v, const int32_t *pos,
@@ -249,9 +265,11 @@ extern "C" gqa_status gqa_attn_prefill(const void *q, const void *k, const void 
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const RopeFreqs rf = rope_freqs(static_cast<double>(theta));
-    gqa_status s = launch_k_norm_rope(k, pos, knorm_w, rf, eps, workspace, static_cast<long long>(B) * T, Hkv, st);
+    float *table = reinterpret_cast<float *>(static_cast<char *>(workspace) + khat_bytes(B, T, Hkv));
+    gqa_status s =
+        launch_k_norm_rope(k, pos, knorm_w, rf, eps, workspace, table, static_cast<long long>(B) * T, Hkv, st);
     if (s != GQA_OK) return s;
-    return launch_attention(q, workspace, v, pos, qnorm_w, rf, eps, out, B, T, H, Hkv, st);
+    return launch_attention(q, workspace, v, pos, table, qnorm_w, rf, eps, out, B, T, H, Hkv, st);
 }
 
 extern "C" size_t gqa_attn_decode_workspace_size(int B, int H, int Hkv, int D, int max_len) {

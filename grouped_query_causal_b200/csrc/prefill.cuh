@@ -34,6 +34,7 @@ struct KPrologueParams {
     const int32_t *pos;    // [ntok]
     const float *wk;       // [D]
     uint16_t *khat;        // bf16 [ntok, Hkv, D]
+    float *rope_cs;        // [ntok, D/2, 2] (cos, sin) of every token's RoPE angles, or nullptr
     long long ntok;
     int Hkv;
     float eps;
@@ -41,8 +42,9 @@ struct KPrologueParams {
 };
 
 // One warp per token at a time; each half-warp transforms one head vector, each lane
-// eight consecutive elements (four RoPE pairs).  cos/sin are evaluated once per token
-// and reused for all of its KV heads.
+// eight consecutive elements (four RoPE pairs).  cos/sin are evaluated once per token,
+// reused for all of its KV heads, and optionally stored so the query side (same
+// positions) can read them instead of evaluating them again.
 __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__ KPrologueParams p) {
     const int lane = threadIdx.x & 31;
     const int half = lane >> 4;
@@ -59,6 +61,11 @@ __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__
         float cs[4], sn[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) rope_cos_sin(ps, p.rf.inv_freq[4 * sub + i], cs[i], sn[i]);
+        if (p.rope_cs != nullptr && half == 0) {
+            float4 *dst = reinterpret_cast<float4 *>(p.rope_cs + static_cast<size_t>(tok) * kHeadDim + 8 * sub);
+            dst[0] = make_float4(cs[0], sn[0], cs[1], sn[1]);
+            dst[1] = make_float4(cs[2], sn[2], cs[3], sn[3]);
+        }
         for (int h0 = 0; h0 < p.Hkv; h0 += 2) {
             const int hh = h0 + half;
             const bool act = hh < p.Hkv;
@@ -93,32 +100,34 @@ __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__
 // ============================================================================ attention
 constexpr int kBM = 128;                       // query rows per tile (one per softmax thread)
 constexpr int kBN = 128;                       // keys per K/V tile
-constexpr int kStages = 3;                     // K/V ring depth (tiles)
+constexpr int kStages = 5;                     // K/V ring depth (tiles)
 constexpr uint32_t kTileBytes = 128 * 128 * 2; // one bf16 128x128 tile
 constexpr uint32_t kBoxBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr uint32_t kOffQ = 0;                                   // 2 tiles
-constexpr uint32_t kOffP = kOffQ + 2 * kTileBytes;              // 2 tiles
-constexpr uint32_t kOffKV = kOffP + 2 * kTileBytes;             // kStages tiles
+constexpr uint32_t kOffKV = kOffQ + 2 * kTileBytes;             // kStages tiles
 constexpr uint32_t kOffBar = kOffKV + kStages * kTileBytes;
 enum {
     BAR_Q_FULL = 0,    // [2] TMA -> softmax WG: raw Q tile landed
     BAR_Q_READY = 2,   // [2] softmax WG -> MMA: Q tile normed + rotated in place (128 arrivals)
     BAR_KV_FULL = 4,   // [kStages] TMA -> MMA
     BAR_KV_EMPTY = 4 + kStages,      // [kStages] MMA (commit) -> TMA
-    BAR_S_FULL = 4 + 2 * kStages,    // [2] MMA (commit) -> softmax WG
-    BAR_P_FULL = 6 + 2 * kStages,    // [2] softmax WG -> MMA (128 arrivals)
-    BAR_O_FULL = 8 + 2 * kStages,    // [2] MMA (commit) -> softmax WG: last P V done
+    BAR_S_FULL = 4 + 2 * kStages,    // [2] MMA (commit) -> softmax WG: S of the next tile is in TMEM
+    BAR_P_FULL = 6 + 2 * kStages,    // [2] softmax WG -> MMA: P written over S in TMEM, O rescaled (128 arrivals)
+    BAR_O_FULL = 8 + 2 * kStages,    // [2] MMA (commit) -> softmax WG: last P V finished
     BAR_DRAIN = 10 + 2 * kStages,    // MMA drains its own work before TMEM is released
     NUM_BARS = 11 + 2 * kStages
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + NUM_BARS * 8;
 constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align the base to 1024
-constexpr uint32_t kTmemCols = 512;   // S0 | S1 | O0 | O1, 128 fp32 columns each
+// TMEM: S0 | S1 | O0 | O1, 128 fp32 columns each.  P of a tile (bf16, two per column)
+// is written over the first 64 columns of its S once S has been read.
+constexpr uint32_t kTmemCols = 512;
 constexpr int kAttnThreads = 384;     // warp 0 TMA, warp 1 MMA, warps 4-7 / 8-11 softmax
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct AttnParams {
     const int32_t *pos;    // [B, T]
+    const float *rope_cs;  // [B, T, D/2, 2] cos/sin of the RoPE angles, or nullptr (evaluate here)
     const float *wq;       // [D]
     float *out;            // fp32 [B, T, H, D]
     unsigned *err;
@@ -135,7 +144,8 @@ __device__ __forceinline__ uint32_t tile_chunk_addr(uint32_t tile, int r, int c)
            (static_cast<uint32_t>((c & 7) ^ (r & 7)) << 4);
 }
 
-// S = Q K^T for one 128x128 tile: eight K=16 steps over the head dimension.
+// S = Q K^T for one 128x128 tile: eight K=16 steps over the head dimension, both
+// operands K-major in shared memory.
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t sk, uint32_t idesc) {
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
@@ -145,23 +155,24 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t 
     }
 }
 
-// O (+)= P V: eight K=16 steps over the keys.  P is K-major (keys contiguous); V is
-// MN-major (head dim contiguous): its two 64-column boxes are kBoxBytes apart (LBO)
-// and 8-key groups are 1024 bytes apart (SBO).
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t sp, uint32_t sv, uint32_t idesc,
+// O (+)= P V: eight K=16 steps over the keys.  P (bf16, K-major) is read from tensor
+// memory, 8 columns per step; V is MN-major in shared memory (head dim contiguous):
+// its two 64-column boxes are kBoxBytes apart (LBO) and 8-key groups 1024 bytes (SBO).
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t sv, uint32_t idesc,
                                          bool accumulate) {
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t offp = static_cast<uint32_t>(kk >> 2) * kBoxBytes + static_cast<uint32_t>(kk & 3) * 32u;
         const uint32_t offv = static_cast<uint32_t>(kk) * 2048u;
-        umma_bf16_ss(d_tmem, sw128_desc(sp + offp, 16, 1024), sw128_desc(sv + offv, kBoxBytes, 1024), idesc,
+        umma_bf16_ts(d_tmem, p_tmem + 8u * kk, sw128_desc(sv + offv, kBoxBytes, 1024), idesc,
                      (accumulate || kk > 0) ? 1u : 0u);
     }
 }
 
-// RMSNorm (w_q, eps) and RoPE (position ps) of query row r of a raw Q tile, in place.
-__device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, const float *wq, float eps,
-                                                const RopeFreqs &rf) {
+// RMSNorm (w_q, eps) and RoPE of query row r of a raw Q tile, in place.  The rotation
+// uses the token's cos/sin row `cs` ([D/2][2], from the K prologue) when given, else
+// evaluates them from the position ps.
+__device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, const float *cs_row, const float *wq,
+                                                float eps, const RopeFreqs &rf) {
     float ss = 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
@@ -183,16 +194,37 @@ __device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, cons
         const float4 wa = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c);
         const float4 wb = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c + 1);
         const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+        float cs[4], sn[4];
+        if (cs_row != nullptr) {
+            const float4 t0 = __ldg(reinterpret_cast<const float4 *>(cs_row) + 2 * c);
+            const float4 t1 = __ldg(reinterpret_cast<const float4 *>(cs_row) + 2 * c + 1);
+            cs[0] = t0.x; sn[0] = t0.y; cs[1] = t0.z; sn[1] = t0.w;
+            cs[2] = t1.x; sn[2] = t1.y; cs[3] = t1.z; sn[3] = t1.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rope_cos_sin(ps, rf.inv_freq[4 * c + i], cs[i], sn[i]);
+        }
         uint32_t o[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            float cs, sn;
-            rope_cos_sin(ps, rf.inv_freq[4 * c + i], cs, sn);
             const float a = w[2 * i] * bf16lo(u[i]) * inv;
             const float b = w[2 * i + 1] * bf16hi(u[i]) * inv;
-            o[i] = pack_bf16x2(a * cs - b * sn, a * sn + b * cs);
+            o[i] = pack_bf16x2(a * cs[i] - b * sn[i], a * sn[i] + b * cs[i]);
         }
         st_shared_v4(addr, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+}
+
+// 2^(x*scale + negm) of 64 consecutive scores, packed as bf16 pairs into 32 words; their
+// (unrounded) sum goes into eight partial sums.
+__device__ __forceinline__ void exp_pack64(const float *x, float scale, float negm, uint32_t *pk, float (&sp)[8]) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const float e0 = ex2_approx(fmaf(x[2 * c], scale, negm));
+        const float e1 = ex2_approx(fmaf(x[2 * c + 1], scale, negm));
+        sp[(2 * c) & 7] += e0;
+        sp[(2 * c + 1) & 7] += e1;
+        pk[c] = pack_bf16x2(e0, e1);
     }
 }
 
@@ -223,7 +255,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int hq0 = g * p.hpg + j0;
     const int n_kv = qb + 1;  // causal: K/V tiles 0 .. qb
 
-    const uint32_t sQ0 = sbase + kOffQ, sP0 = sbase + kOffP, sKV0 = sbase + kOffKV;
+    const uint32_t sQ0 = sbase + kOffQ, sKV0 = sbase + kOffKV;
     const uint32_t bar0 = sbase + kOffBar;
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
 
@@ -291,12 +323,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // In-order program with blocking (suspending) waits, heads interleaved:
+        //   Q K_0^T (both heads), then for every tile j and head s: P_j V_j as soon as
+        //   the softmax has written P_j over S_j, immediately followed by Q K_{j+1}^T
+        //   (which overwrites P_j: tcgen05.mma operations of one thread run in issue
+        //   order).  While head 0's softmax works on S_{j+1}, the tensor core runs head
+        //   1's P V and Q K^T, and vice versa.
+        // The issuing thread is on the critical path, so its waits carry a short suspend
+        // hint: a default try_wait can wake up ~900 cycles after the phase completes.
+#define MMA_WAIT(b_, par_, e_) mbar_wait_hint((b_), (par_), 20u, (e_))
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16_f32(kBM, kBN, false);
             const uint32_t id_pv = idesc_bf16_f32(kBM, kHeadDim, true);
             bool ok = true;
             for (int s = 0; s < nslots && ok; ++s) ok = mbar_wait(BAR(BAR_Q_READY + s), 0, p.err);
-            if (ok) ok = mbar_wait(BAR(BAR_KV_FULL + 0), 0, p.err);   // K0
+            if (ok) ok = mbar_wait(BAR(BAR_KV_FULL + 0), 0, p.err);   // K_0 is ring item 0
             if (ok) {
                 tc_fence_after();
                 for (int s = 0; s < nslots; ++s) {
@@ -306,33 +347,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 umma_commit(BAR(BAR_KV_EMPTY + 0));
             }
             for (int j = 0; j < n_kv && ok; ++j) {
-                const int itv = 2 * j + 1, bv = itv % kStages;
-                const int itk = 2 * j + 2, bk = itk % kStages;
+                const int iv = 2 * j + 1, ik = 2 * j + 2;   // ring items of V_j and K_{j+1}
                 const bool more = j + 1 < n_kv;
-                if (!mbar_wait(BAR(BAR_KV_FULL + bv), (itv / kStages) & 1, p.err)) { ok = false; break; }
+                if (!MMA_WAIT(BAR(BAR_KV_FULL + iv % kStages), (iv / kStages) & 1, p.err)) { ok = false; break; }
                 for (int s = 0; s < nslots; ++s) {
-                    if (!mbar_wait(BAR(BAR_P_FULL + s), j & 1, p.err)) { ok = false; break; }
+                    if (!MMA_WAIT(BAR(BAR_P_FULL + s), j & 1, p.err)) { ok = false; break; }
                     tc_fence_after();
-                    issue_pv(tmem + 256 + s * 128, sP0 + s * kTileBytes, sKV0 + bv * kTileBytes, id_pv, j > 0);
+                    issue_pv(tmem + 256 + s * 128, tmem + s * 128, sKV0 + (iv % kStages) * kTileBytes, id_pv, j > 0);
                     if (more) {
-                        if (s == 0) {
-                            if (!mbar_wait(BAR(BAR_KV_FULL + bk), (itk / kStages) & 1, p.err)) { ok = false; break; }
-                            tc_fence_after();
+                        if (s == 0 && !MMA_WAIT(BAR(BAR_KV_FULL + ik % kStages), (ik / kStages) & 1, p.err)) {
+                            ok = false;
+                            break;
                         }
-                        issue_qk(tmem + s * 128, sQ0 + s * kTileBytes, sKV0 + bk * kTileBytes, id_qk);
+                        issue_qk(tmem + s * 128, sQ0 + s * kTileBytes, sKV0 + (ik % kStages) * kTileBytes, id_qk);
                         umma_commit(BAR(BAR_S_FULL + s));
                     } else {
                         umma_commit(BAR(BAR_O_FULL + s));
                     }
                 }
                 if (!ok) break;
-                umma_commit(BAR(BAR_KV_EMPTY + bv));
-                if (more) umma_commit(BAR(BAR_KV_EMPTY + bk));
+                umma_commit(BAR(BAR_KV_EMPTY + iv % kStages));
+                if (more) umma_commit(BAR(BAR_KV_EMPTY + ik % kStages));
             }
             // Every MMA issued above must finish before TMEM can be released.
             umma_commit(BAR(BAR_DRAIN));
             mbar_wait(BAR(BAR_DRAIN), 0, p.err);
         }
+#undef MMA_WAIT
         __syncwarp();
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax warpgroups
@@ -343,15 +384,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint32_t tS = tmem + lane_base + s * 128;
             const uint32_t tO = tmem + lane_base + 256 + s * 128;
             const uint32_t sQ = sQ0 + s * kTileBytes;
-            const uint32_t sP = sP0 + s * kTileBytes;
             const int t = qb * kBM + r;
             const bool valid = t < p.T;
             const int hq = hq0 + s;
 
             bool ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_Q_FULL + s), 0, p.err));
             if (ok) {
-                const int ps = valid ? p.pos[static_cast<size_t>(b) * p.T + t] : 0;
-                transform_q_row(sQ, r, ps, p.wq, p.eps, p.rf);
+                const size_t tok = static_cast<size_t>(b) * p.T + t;
+                const int ps = valid ? p.pos[tok] : 0;
+                const float *cs_row = (valid && p.rope_cs != nullptr) ? p.rope_cs + tok * kHeadDim : nullptr;
+                transform_q_row(sQ, r, ps, cs_row, p.wq, p.eps, p.rf);
                 fence_proxy_async_smem();
                 mbar_arrive(BAR(BAR_Q_READY + s));
             }
@@ -359,6 +401,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             float m_run = -INFINITY;   // running max of scaled scores (base 2), possibly stale by < 8
             float l_run = 0.f;         // running sum of 2^(score - m_run)
             for (int j = 0; j < n_kv && ok; ++j) {
+                // S_FULL of tile j also means P_{j-1} V_{j-1} has finished (issued before Q K_j^T).
                 ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_S_FULL + s), j & 1, p.err));
                 if (!ok) break;
                 tc_fence_after();
@@ -373,9 +416,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     for (int c = 0; c < 128; ++c)
                         if (c > r) x[c] = -INFINITY;
                 }
-                float mx = x[0];
+                // row max with eight independent partial maxima (short dependency chains)
+                float mp[8];
 #pragma unroll
-                for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+                for (int u = 0; u < 8; ++u) mp[u] = x[u];
+#pragma unroll
+                for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+                const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
                 const float m_new = fmaxf(m_run, mx * p.scale_log2);
                 // Only move the reference max when it grows by more than 2^8; the final
                 // O / l is exact either way because O and l always share the reference.
@@ -383,23 +431,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
                 if (need) m_run = m_new;
                 l_run *= alpha;
-                float lsum = 0.f;
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    float e[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        e[u] = ex2_approx(fmaf(x[8 * c + u], p.scale_log2, -m_run));
-                        lsum += e[u];
-                    }
-                    st_shared_v4(tile_chunk_addr(sP, r, c),
-                                 make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
-                                            pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7])));
+                const float negm = -m_run;
+                float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                {
+                    uint32_t pk[32];
+                    exp_pack64(x, p.scale_log2, negm, pk, sp);
+                    tmem_st32(tS, reinterpret_cast<const float *>(pk));          // P keys 0..63
                 }
-                l_run += lsum;
-                // Rescale this row of O if the reference moved.  Safe: the P V of tile j-1
-                // finished before S of tile j was signalled, and the P V of tile j waits
-                // for P_FULL below.
+                {
+                    uint32_t pk[32];
+                    exp_pack64(x + 64, p.scale_log2, negm, pk, sp);
+                    tmem_st32(tS + 32, reinterpret_cast<const float *>(pk));     // P keys 64..127
+                }
+                // Rescale this row of O if the reference moved (rare after the first tiles).
+                // O is stable: P_{j-1} V_{j-1} finished before S_j was signalled.
                 if (__any_sync(0xffffffffu, need) && j > 0) {
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
@@ -410,11 +455,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         for (int u = 0; u < 32; ++u) o[u] *= alpha;
                         tmem_st32(tO + 32 * c, o);
                     }
-                    tmem_wait_st();
                 }
-                fence_proxy_async_smem();
+                tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(BAR(BAR_P_FULL + s));
+                l_run += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
             }
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_O_FULL + s), 0, p.err));
             if (ok) {

@@ -59,8 +59,9 @@ typedef enum {
 /* Human-readable name of a status code (static string, never NULL). */
 const char *gqa_status_string(gqa_status status);
 
-/* Workspace bytes gqa_attn_prefill needs for these sizes (k-hat, bf16 [B,T,Hkv,D],
- * plus alignment).  Returns 0 for an empty problem or invalid sizes. */
+/* Workspace bytes gqa_attn_prefill needs for these sizes: k-hat (bf16 [B,T,Hkv,D]) and
+ * the per-token RoPE cos/sin table (fp32 [B,T,D/2,2]), each rounded up to 256 bytes.
+ * Returns 0 for an empty problem or invalid sizes. */
 size_t gqa_attn_prefill_workspace_size(int B, int T, int H, int Hkv, int D);
 
 /*
@@ -95,21 +96,27 @@ gqa_status gqa_attn_prefill(const void *q, const void *k, const void *v, const i
  * in the layout of k.  These are the keys the KV cache holds ("Qwen3系列1" D2-3: K is
  * written to the cache after its norm and rotation, before attention), so the output
  * can be a decode cache directly.
- *   k      bf16 [N, Hkv, D] (N = B*T tokens, any token order); pos int32 [N]
- *   k_hat  bf16 [N, Hkv, D], must not overlap k.   N = 0 is a no-op.
+ *   k        bf16 [N, Hkv, D] (N = B*T tokens, any token order); pos int32 [N]
+ *   k_hat    bf16 [N, Hkv, D], must not overlap k.   N = 0 is a no-op.
+ *   rope_cs  fp32 [N, D/2, 2] or NULL: when given, receives (cos, sin) of every token's
+ *            RoPE angles pos * theta^(-2i/D), for gqa_attn_prefill_khat to reuse.
  */
 gqa_status gqa_attn_k_norm_rope(const void *k, const int32_t *pos, const float *knorm_w, float theta,
-                                float eps, void *k_hat, int64_t N, int Hkv, int D, void *stream);
+                                float eps, void *k_hat, float *rope_cs, int64_t N, int Hkv, int D,
+                                void *stream);
 
 /*
  * gqa_attn_prefill_khat: the attention stage of gqa_attn_prefill on keys that are
  * already normed and rotated (k_hat, e.g. from gqa_attn_k_norm_rope): the raw q tiles
  * are normed (qnorm_w, eps) and rotated (pos, theta) inside the attention kernel.
- * Arguments as for gqa_attn_prefill; k_hat is bf16 [B, T, Hkv, D].  Needs no workspace.
+ * Arguments as for gqa_attn_prefill; k_hat is bf16 [B, T, Hkv, D].  rope_cs is the
+ * fp32 [B, T, D/2, 2] table gqa_attn_k_norm_rope wrote for the same positions and
+ * theta, or NULL (the kernel then evaluates cos/sin itself, which is slower).
+ * Needs no workspace.
  */
 gqa_status gqa_attn_prefill_khat(const void *q, const void *k_hat, const void *v, const int32_t *pos,
-                                 const float *qnorm_w, float theta, float eps, float *out, int B, int T,
-                                 int H, int Hkv, int D, void *stream);
+                                 const float *rope_cs, const float *qnorm_w, float theta, float eps,
+                                 float *out, int B, int T, int H, int Hkv, int D, void *stream);
 
 /* Workspace bytes gqa_attn_decode needs: split-KV partial results for up to max_len
  * cached tokens per sequence.  Returns 0 for an empty problem or invalid sizes. */

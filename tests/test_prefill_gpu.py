@@ -123,7 +123,33 @@ def test_two_stage_prefill_equals_one_call(gqa):
     inp = synthetic.prefill_inputs(2, 190, 8, 2, seed=33)
     d = to_dev(inp)
     one = gqa.prefill(d["q"], d["k"], d["v"], d["pos"], d["qnorm_w"], d["knorm_w"], d["theta"], d["eps"])
-    khat = gqa.k_norm_rope(d["k"], d["pos"], d["knorm_w"], d["theta"], d["eps"])
-    two = gqa.prefill_khat(d["q"], khat, d["v"], d["pos"], d["qnorm_w"], d["theta"], d["eps"])
+    table = torch.empty((2, 190, 128), dtype=torch.float32, device="cuda")
+    khat = gqa.k_norm_rope(d["k"], d["pos"], d["knorm_w"], d["theta"], d["eps"], rope_cs=table)
+    two = gqa.prefill_khat(d["q"], khat, d["v"], d["pos"], d["qnorm_w"], d["theta"], d["eps"], rope_cs=table)
     torch.cuda.synchronize()
     assert torch.equal(one, two)
+
+
+def test_q_rope_without_table_matches_oracle(gqa):
+    """The attention stage alone, evaluating the query cos/sin itself (no table)."""
+    inp = synthetic.prefill_inputs(1, 300, 8, 4, seed=34)
+    g = torch.Generator().manual_seed(35)
+    inp.pos = torch.randint(0, 32768, (1, 300), generator=g, dtype=torch.int32)
+    d = to_dev(inp)
+    khat = gqa.k_norm_rope(d["k"], d["pos"], d["knorm_w"], d["theta"], d["eps"])
+    got = gqa.prefill_khat(d["q"], khat, d["v"], d["pos"], d["qnorm_w"], d["theta"], d["eps"])
+    torch.cuda.synchronize()
+    gqa.check_device_status()
+    assert_close(got.cpu().numpy(), oracle.prefill(*oracle_prefill_args(inp)), "no table")
+
+
+def test_rope_table_matches_closed_form(gqa):
+    """The cos/sin table the K prologue writes: cos/sin(pos * theta^(-2i/D))."""
+    pos = torch.tensor([0, 1, 7, 4095, 32767], dtype=torch.int32)
+    k = torch.zeros((5, 1, 128), dtype=torch.bfloat16)
+    table = torch.empty((5, 128), dtype=torch.float32, device="cuda")
+    gqa.k_norm_rope(k.cuda(), pos.cuda(), torch.ones(128, device="cuda"), 1e6, 1e-6, rope_cs=table)
+    torch.cuda.synchronize()
+    ang = pos.double()[:, None] * (1e6 ** (-torch.arange(0, 128, 2, dtype=torch.float64) / 128))
+    ref = torch.stack([torch.cos(ang), torch.sin(ang)], -1).reshape(5, 128)
+    assert (table.cpu().double() - ref).abs().max().item() < 2e-6
