@@ -237,7 +237,9 @@ def run_ours(args, rank, world, local_rank):
         return None
     pk, pk_kind = peaks()
     hbm = float(pk["hbm_gbs"])
-    tc = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    # The burst figure: the step runs at the maximum SM clock (see "clocks"), like the burst
+    # cuBLAS measurement; the power-capped sustained figure is reported for context.
+    tc = float(pk["bf16_tflops"])
     attn_tflops = flops * K / (attn_ms / 1e3) / 1e12
     dec_gbs = dbytes * K / dec_s / 1e9
     traffic_attn = traffic_from_profiles("attn_fwd_kernel")
@@ -278,8 +280,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": tc, "unit": "TFLOP/s",
                      "frac": round(attn_tflops / tc, 4), "traffic": traffic_attn, "kernel": "attn_fwd_kernel",
                      "attn_ms": round(attn_ms / K, 4), "k_prologue_ms": round(pro_ms / K, 4),
-                     "peak_source": f"bf16_tflops_sustained of {pk_kind}",
-                     "peak_burst": float(pk["bf16_tflops"])},
+                     "peak_source": f"bf16_tflops (burst) of {pk_kind}",
+                     "peak_sustained": float(pk.get("bf16_tflops_sustained", tc))},
         "e2e": e2e["prefill"],
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
