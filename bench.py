@@ -163,7 +163,7 @@ def run_ours(args, rank, world, local_rank):
     q, k, v, pos = pin.q.to(dev), pin.k.to(dev), pin.v.to(dev), pin.pos.to(dev)
     wq, wk = pin.wq.to(dev), pin.wk.to(dev)
     khat = torch.empty_like(k)
-    rope_cs = torch.empty((B, T, D), dtype=torch.float32, device=dev)
+    rope_cs = torch.empty(gqa.rope_table_numel(B * T, D), dtype=torch.float32, device=dev)
     out = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
     dq, kc, vc = dec.q.to(dev), dec.k_cache.to(dev), dec.v_cache.to(dev)
     offs, sl, dwq = dec.offsets.to(dev), dec.seqlens.to(dev), dec.wq.to(dev)

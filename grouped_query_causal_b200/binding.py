@@ -95,6 +95,18 @@ def _raise(status: int, what: str):
         raise GqaError(status, what)
 
 
+def rope_table_numel(n_tokens: int, D: int = 128) -> int:
+    """fp32 elements of the RoPE cos/sin table for n_tokens (GQA_ROPE_TABLE_BYTES / 4)."""
+    return (n_tokens + 127) // 128 * 128 * D
+
+
+def rope_table_entry(table: torch.Tensor, n: int, pair: int):
+    """(cos, sin) of RoPE pair `pair` of flattened token n in a table k_norm_rope wrote."""
+    i2, k = divmod(pair, 2)
+    base = (((n >> 7) * 32 + i2) * 128 + (n & 127)) * 4 + 2 * k
+    return float(table[base]), float(table[base + 1])
+
+
 def prefill_workspace_size(B: int, T: int, H: int, Hkv: int, D: int = 128) -> int:
     return int(load().gqa_attn_prefill_workspace_size(B, T, H, Hkv, D))
 
@@ -139,8 +151,8 @@ def k_norm_rope(k, pos, knorm_w, theta: float = 1.0e6, eps: float = 1e-6,
                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """k-hat = RoPE(RMSNorm(k)) in bf16.  k [..., Hkv, D] bf16 with one position per
     token (pos has the leading shape of k) -> k_hat of k's shape (a decode cache).
-    rope_cs (fp32 [..., D/2, 2] over the same tokens), when given, receives the tokens'
-    RoPE cos/sin for prefill_khat to reuse."""
+    rope_cs (fp32, rope_table_numel(N) elements), when given, receives the tokens' RoPE
+    cos/sin (an opaque blocked table) for prefill_khat to reuse."""
     lib = load()
     if k.dtype != torch.bfloat16 or not k.is_cuda or not k.is_contiguous() or k.dim() < 2:
         raise ValueError("k must be a contiguous CUDA bf16 tensor [..., Hkv, D]")
@@ -150,8 +162,8 @@ def k_norm_rope(k, pos, knorm_w, theta: float = 1.0e6, eps: float = 1e-6,
     if pos.dtype != torch.int32 or not pos.is_cuda or not pos.is_contiguous() or pos.numel() != N:
         raise ValueError("pos must be a contiguous CUDA int32 tensor with one entry per token")
     if rope_cs is not None and (rope_cs.dtype != torch.float32 or not rope_cs.is_cuda or not rope_cs.is_contiguous()
-                                or rope_cs.numel() != N * D):
-        raise ValueError("rope_cs must be a contiguous CUDA fp32 tensor of N * D elements")
+                                or rope_cs.numel() < rope_table_numel(N)):
+        raise ValueError("rope_cs must be a contiguous CUDA fp32 tensor of rope_table_numel(N) elements")
     if out is None:
         out = torch.empty_like(k)
     st = lib.gqa_attn_k_norm_rope(_ptr(k), _ptr(pos), _ptr(knorm_w), float(theta), float(eps), _ptr(out),
@@ -179,8 +191,8 @@ def prefill_khat(q, k_hat, v, pos, qnorm_w, theta: float = 1.0e6, eps: float = 1
         out = torch.empty((B, T, H, D), dtype=torch.float32, device=q.device)
     _check(out, "out", torch.float32, 4)
     if rope_cs is not None and (rope_cs.dtype != torch.float32 or not rope_cs.is_cuda or not rope_cs.is_contiguous()
-                                or rope_cs.numel() != B * T * D):
-        raise ValueError("rope_cs must be a contiguous CUDA fp32 tensor of B * T * D elements")
+                                or rope_cs.numel() < rope_table_numel(B * T)):
+        raise ValueError("rope_cs must be a contiguous CUDA fp32 tensor of rope_table_numel(B * T) elements")
     st = lib.gqa_attn_prefill_khat(_ptr(q), _ptr(k_hat), _ptr(v), _ptr(pos), _ptr(rope_cs), _ptr(qnorm_w),
                                    float(theta), float(eps), _ptr(out), B, T, H, Hkv, D, _stream_handle(stream))
     _raise(st, "gqa_attn_prefill_khat")

@@ -138,10 +138,10 @@ extern "C" const char *gqa_status_string(gqa_status status) {
 }
 
 namespace {
-// Workspace of gqa_attn_prefill: k-hat (bf16 [B,T,Hkv,D]), then the per-token RoPE
-// cos/sin table (fp32 [B,T,D/2,2]).
+// Workspace of gqa_attn_prefill: k-hat (bf16 [B,T,Hkv,D]), then the RoPE cos/sin table
+// (round_up(B*T, 128) tokens x D fp32, blocked layout of rope_table_index).
 size_t khat_bytes(int B, int T, int Hkv) { return round_up(static_cast<size_t>(B) * T * Hkv * kHeadDim * 2, 256); }
-size_t rope_table_bytes(int B, int T) { return round_up(static_cast<size_t>(B) * T * kHeadDim * sizeof(float), 256); }
+size_t rope_table_bytes(int B, int T) { return round_up(static_cast<size_t>(B) * T, 128) * kHeadDim * sizeof(float); }
 }  // namespace
 
 extern "C" size_t gqa_attn_prefill_workspace_size(int B, int T, int H, int Hkv, int D) {
@@ -226,7 +226,7 @@ extern "C" gqa_status gqa_attn_k_norm_rope(const void *k, const int32_t *pos, co
     if (a < b + bytes && b < a + bytes) return GQA_ERR_INVALID_ARG;   // overlapping buffers
     if (rope_cs) {
         const uintptr_t c = reinterpret_cast<uintptr_t>(rope_cs);
-        const size_t tb = static_cast<size_t>(N) * kHeadDim * sizeof(float);
+        const size_t tb = round_up(static_cast<size_t>(N), 128) * kHeadDim * sizeof(float);
         if ((c < b + bytes && b < c + tb) || (c < a + bytes && a < c + tb)) return GQA_ERR_INVALID_ARG;
     }
     return launch_k_norm_rope(k, pos, knorm_w, rope_freqs(static_cast<double>(theta)), eps, k_hat, rope_cs, N, Hkv,

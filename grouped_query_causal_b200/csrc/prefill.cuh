@@ -29,12 +29,20 @@
 namespace gqa {
 
 // ============================================================================ K prologue
+// RoPE cos/sin table: float4 entry (cos, sin, cos, sin) of RoPE pairs 2*i2 and 2*i2+1 of
+// flattened token n.  Blocked by 128 tokens, pair-major inside a block, so the 32 threads
+// of a warp (consecutive tokens) read 512 contiguous bytes per load in the q prologue.
+// Size: round_up(N, 128) * 32 float4.
+__host__ __device__ __forceinline__ size_t rope_table_index(long long n, int i2) {
+    return (static_cast<size_t>(n >> 7) * 32 + static_cast<size_t>(i2)) * 128 + static_cast<size_t>(n & 127);
+}
+
 struct KPrologueParams {
     const uint16_t *k;     // bf16 [ntok, Hkv, D]
     const int32_t *pos;    // [ntok]
     const float *wk;       // [D]
     uint16_t *khat;        // bf16 [ntok, Hkv, D]
-    float *rope_cs;        // [ntok, D/2, 2] (cos, sin) of every token's RoPE angles, or nullptr
+    float *rope_cs;        // RoPE cos/sin of every token in the blocked table layout (rope_table_index), or nullptr
     long long ntok;
     int Hkv;
     float eps;
@@ -62,37 +70,49 @@ __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__
 #pragma unroll
         for (int i = 0; i < 4; ++i) rope_cos_sin(ps, p.rf.inv_freq[4 * sub + i], cs[i], sn[i]);
         if (p.rope_cs != nullptr && half == 0) {
-            float4 *dst = reinterpret_cast<float4 *>(p.rope_cs + static_cast<size_t>(tok) * kHeadDim + 8 * sub);
-            dst[0] = make_float4(cs[0], sn[0], cs[1], sn[1]);
-            dst[1] = make_float4(cs[2], sn[2], cs[3], sn[3]);
+            float4 *tab = reinterpret_cast<float4 *>(p.rope_cs);
+            tab[rope_table_index(tok, 2 * sub)] = make_float4(cs[0], sn[0], cs[1], sn[1]);
+            tab[rope_table_index(tok, 2 * sub + 1)] = make_float4(cs[2], sn[2], cs[3], sn[3]);
         }
-        for (int h0 = 0; h0 < p.Hkv; h0 += 2) {
-            const int hh = h0 + half;
-            const bool act = hh < p.Hkv;
-            const size_t off = (static_cast<size_t>(tok) * p.Hkv + hh) * kHeadDim + 8 * sub;
-            uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-            if (act) raw = *reinterpret_cast<const uint4 *>(p.k + off);
-            const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
-            float x[8];
+        // up to 8 head pairs per batch: all loads first, so they are in flight together
+        for (int h0 = 0; h0 < p.Hkv; h0 += 16) {
+            constexpr int kPairs = 8;
+            uint4 raw[kPairs];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                x[2 * i] = bf16lo(rw[i]);
-                x[2 * i + 1] = bf16hi(rw[i]);
+            for (int u = 0; u < kPairs; ++u) {
+                const int hh = h0 + 2 * u + half;
+                raw[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (hh < p.Hkv)
+                    raw[u] = *reinterpret_cast<const uint4 *>(p.k + (static_cast<size_t>(tok) * p.Hkv + hh) * kHeadDim + 8 * sub);
             }
-            float ss = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+            for (int u = 0; u < kPairs; ++u) {
+                const int hh = h0 + 2 * u + half;
+                if (h0 + 2 * u >= p.Hkv) break;   // warp-uniform
+                const uint32_t rw[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+                float x[8];
 #pragma unroll
-            for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + p.eps);
-            uint32_t outw[4];
+                for (int i = 0; i < 4; ++i) {
+                    x[2 * i] = bf16lo(rw[i]);
+                    x[2 * i + 1] = bf16hi(rw[i]);
+                }
+                float ss = 0.f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float a = w[2 * i] * x[2 * i] * inv;
-                const float b = w[2 * i + 1] * x[2 * i + 1] * inv;
-                outw[i] = pack_bf16x2(a * cs[i] - b * sn[i], a * sn[i] + b * cs[i]);
+                for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + p.eps);
+                uint32_t outw[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float a = w[2 * i] * x[2 * i] * inv;
+                    const float b = w[2 * i + 1] * x[2 * i + 1] * inv;
+                    outw[i] = pack_bf16x2(a * cs[i] - b * sn[i], a * sn[i] + b * cs[i]);
+                }
+                if (hh < p.Hkv)
+                    *reinterpret_cast<uint4 *>(p.khat + (static_cast<size_t>(tok) * p.Hkv + hh) * kHeadDim + 8 * sub) =
+                        make_uint4(outw[0], outw[1], outw[2], outw[3]);
             }
-            if (act) *reinterpret_cast<uint4 *>(p.khat + off) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
         }
     }
 }
@@ -127,7 +147,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct AttnParams {
     const int32_t *pos;    // [B, T]
-    const float *rope_cs;  // [B, T, D/2, 2] cos/sin of the RoPE angles, or nullptr (evaluate here)
+    const float *rope_cs;  // RoPE cos/sin table over the B*T tokens (rope_table_index), or nullptr (evaluate here)
     const float *wq;       // [D]
     float *out;            // fp32 [B, T, H, D]
     unsigned *err;
@@ -168,11 +188,12 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
     }
 }
 
-// RMSNorm (w_q, eps) and RoPE of query row r of a raw Q tile, in place.  The rotation
-// uses the token's cos/sin row `cs` ([D/2][2], from the K prologue) when given, else
-// evaluates them from the position ps.
-__device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, const float *cs_row, const float *wq,
-                                                float eps, const RopeFreqs &rf) {
+// RMSNorm (w_q, eps) and RoPE of query row r (flattened token n) of a raw Q tile, in
+// place.  The rotation uses the K prologue's cos/sin table when given (coalesced across
+// the warp: consecutive rows are consecutive tokens), fetched in two batches of 16
+// loads, else evaluates cos/sin from the position ps.
+__device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, const float *table, long long n,
+                                                const float *wq, float eps, const RopeFreqs &rf) {
     float ss = 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
@@ -186,32 +207,41 @@ __device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, cons
         }
     }
     const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + eps);
-#pragma unroll 2
-    for (int c = 0; c < 16; ++c) {
-        const uint32_t addr = tile_chunk_addr(sq, r, c);
-        const uint4 v = ld_shared_v4(addr);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-        const float4 wa = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c);
-        const float4 wb = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c + 1);
-        const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-        float cs[4], sn[4];
-        if (cs_row != nullptr) {
-            const float4 t0 = __ldg(reinterpret_cast<const float4 *>(cs_row) + 2 * c);
-            const float4 t1 = __ldg(reinterpret_cast<const float4 *>(cs_row) + 2 * c + 1);
-            cs[0] = t0.x; sn[0] = t0.y; cs[1] = t0.z; sn[1] = t0.w;
-            cs[2] = t1.x; sn[2] = t1.y; cs[3] = t1.z; sn[3] = t1.w;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        float4 tb[16];   // (cos, sin) of pairs 32*half .. 32*half+31, two pairs per float4
+        if (table != nullptr) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                tb[i] = __ldg(reinterpret_cast<const float4 *>(table) + rope_table_index(n, 16 * half + i));
         } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) rope_cos_sin(ps, rf.inv_freq[4 * c + i], cs[i], sn[i]);
+            for (int i = 0; i < 16; ++i) {
+                const int pr = 32 * half + 2 * i;
+                rope_cos_sin(ps, rf.inv_freq[pr], tb[i].x, tb[i].y);
+                rope_cos_sin(ps, rf.inv_freq[pr + 1], tb[i].z, tb[i].w);
+            }
         }
-        uint32_t o[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float a = w[2 * i] * bf16lo(u[i]) * inv;
-            const float b = w[2 * i + 1] * bf16hi(u[i]) * inv;
-            o[i] = pack_bf16x2(a * cs[i] - b * sn[i], a * sn[i] + b * cs[i]);
+        for (int c8 = 0; c8 < 8; ++c8) {
+            const int c = 8 * half + c8;   // elements 8c..8c+7 = RoPE pairs 4c..4c+3
+            const uint32_t addr = tile_chunk_addr(sq, r, c);
+            const uint4 v = ld_shared_v4(addr);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+            const float4 wa = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c);
+            const float4 wb = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c + 1);
+            const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            const float cs[4] = {tb[2 * c8].x, tb[2 * c8].z, tb[2 * c8 + 1].x, tb[2 * c8 + 1].z};
+            const float sn[4] = {tb[2 * c8].y, tb[2 * c8].w, tb[2 * c8 + 1].y, tb[2 * c8 + 1].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float a = w[2 * i] * bf16lo(u[i]) * inv;
+                const float b = w[2 * i + 1] * bf16hi(u[i]) * inv;
+                o[i] = pack_bf16x2(a * cs[i] - b * sn[i], a * sn[i] + b * cs[i]);
+            }
+            st_shared_v4(addr, make_uint4(o[0], o[1], o[2], o[3]));
         }
-        st_shared_v4(addr, make_uint4(o[0], o[1], o[2], o[3]));
     }
 }
 
@@ -292,6 +322,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             bool ok = true;
+            if (p.rope_cs != nullptr) {   // the table blocks holding this query block's tokens
+                const long long n0 = static_cast<long long>(b) * p.T + qb * kBM;
+                const long long n1 = n0 + min(kBM, p.T - qb * kBM) - 1;
+                for (long long blk = n0 >> 7; blk <= (n1 >> 7); ++blk)
+                    prefetch_l2_bulk(p.rope_cs + rope_table_index(blk << 7, 0) * 4, 32 * 128 * 16);
+            }
             for (int s = 0; s < nslots; ++s) {
                 const uint32_t dst = sQ0 + s * kTileBytes;
                 mbar_arrive_expect_tx(BAR(BAR_Q_FULL + s), kTileBytes);
@@ -383,17 +419,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
             const uint32_t tS = tmem + lane_base + s * 128;
             const uint32_t tO = tmem + lane_base + 256 + s * 128;
-            const uint32_t sQ = sQ0 + s * kTileBytes;
             const int t = qb * kBM + r;
             const bool valid = t < p.T;
             const int hq = hq0 + s;
 
             bool ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_Q_FULL + s), 0, p.err));
             if (ok) {
-                const size_t tok = static_cast<size_t>(b) * p.T + t;
+                const long long tok = static_cast<long long>(b) * p.T + t;
                 const int ps = valid ? p.pos[tok] : 0;
-                const float *cs_row = (valid && p.rope_cs != nullptr) ? p.rope_cs + tok * kHeadDim : nullptr;
-                transform_q_row(sQ, r, ps, cs_row, p.wq, p.eps, p.rf);
+                transform_q_row(sQ0 + s * kTileBytes, r, ps, valid ? p.rope_cs : nullptr, tok, p.wq, p.eps, p.rf);
                 fence_proxy_async_smem();
                 mbar_arrive(BAR(BAR_Q_READY + s));
             }

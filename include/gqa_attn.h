@@ -59,9 +59,12 @@ typedef enum {
 /* Human-readable name of a status code (static string, never NULL). */
 const char *gqa_status_string(gqa_status status);
 
-/* Workspace bytes gqa_attn_prefill needs for these sizes: k-hat (bf16 [B,T,Hkv,D]) and
- * the per-token RoPE cos/sin table (fp32 [B,T,D/2,2]), each rounded up to 256 bytes.
- * Returns 0 for an empty problem or invalid sizes. */
+/* Bytes of the RoPE cos/sin table for n tokens: round_up(n, 128) * D * 4, with D = 128. */
+#define GQA_ROPE_TABLE_BYTES(n) ((((size_t)(n) + 127) / 128) * 128 * 128 * 4)
+
+/* Workspace bytes gqa_attn_prefill needs for these sizes: k-hat (bf16 [B,T,Hkv,D],
+ * rounded up to 256 bytes) and the RoPE cos/sin table of the B*T tokens
+ * (GQA_ROPE_TABLE_BYTES(B*T)).  Returns 0 for an empty problem or invalid sizes. */
 size_t gqa_attn_prefill_workspace_size(int B, int T, int H, int Hkv, int D);
 
 /*
@@ -98,8 +101,9 @@ gqa_status gqa_attn_prefill(const void *q, const void *k, const void *v, const i
  * can be a decode cache directly.
  *   k        bf16 [N, Hkv, D] (N = B*T tokens, any token order); pos int32 [N]
  *   k_hat    bf16 [N, Hkv, D], must not overlap k.   N = 0 is a no-op.
- *   rope_cs  fp32 [N, D/2, 2] or NULL: when given, receives (cos, sin) of every token's
- *            RoPE angles pos * theta^(-2i/D), for gqa_attn_prefill_khat to reuse.
+ *   rope_cs  NULL, or GQA_ROPE_TABLE_BYTES(N) bytes (16-byte aligned) that receive the
+ *            cos/sin of every token's RoPE angles pos * theta^(-2i/D) in the library's
+ *            blocked layout (an opaque intermediate), for gqa_attn_prefill_khat to reuse.
  */
 gqa_status gqa_attn_k_norm_rope(const void *k, const int32_t *pos, const float *knorm_w, float theta,
                                 float eps, void *k_hat, float *rope_cs, int64_t N, int Hkv, int D,
@@ -110,8 +114,8 @@ gqa_status gqa_attn_k_norm_rope(const void *k, const int32_t *pos, const float *
  * already normed and rotated (k_hat, e.g. from gqa_attn_k_norm_rope): the raw q tiles
  * are normed (qnorm_w, eps) and rotated (pos, theta) inside the attention kernel.
  * Arguments as for gqa_attn_prefill; k_hat is bf16 [B, T, Hkv, D].  rope_cs is the
- * fp32 [B, T, D/2, 2] table gqa_attn_k_norm_rope wrote for the same positions and
- * theta, or NULL (the kernel then evaluates cos/sin itself, which is slower).
+ * table gqa_attn_k_norm_rope wrote for the same B*T tokens (flattened b*T + t),
+ * positions and theta, or NULL (the kernel then evaluates cos/sin itself, slower).
  * Needs no workspace.
  */
 gqa_status gqa_attn_prefill_khat(const void *q, const void *k_hat, const void *v, const int32_t *pos,

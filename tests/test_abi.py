@@ -45,9 +45,9 @@ def test_status_strings(lib):
 
 
 def test_workspace_sizes(lib):
-    # k-hat (bf16 [B,T,Hkv,D]) + RoPE table (fp32 [B,T,D/2,2]), each rounded up to 256 bytes
+    # k-hat (bf16 [B,T,Hkv,D], rounded to 256 B) + RoPE table (round_up(B*T, 128) tokens x 512 B)
     assert lib.gqa_attn_prefill_workspace_size(4, 4096, 32, 8, 128) == 4 * 4096 * 8 * 128 * 2 + 4 * 4096 * 128 * 4
-    assert lib.gqa_attn_prefill_workspace_size(1, 3, 2, 1, 128) == 3 * 128 * 2 + 3 * 128 * 4
+    assert lib.gqa_attn_prefill_workspace_size(1, 3, 2, 1, 128) == 3 * 128 * 2 + 128 * 128 * 4
     assert lib.gqa_attn_prefill_workspace_size(1, 128, 16, 8, 64) == 0
     assert lib.gqa_attn_prefill_workspace_size(1, 128, 16, 3, 128) == 0
     assert lib.gqa_attn_prefill_workspace_size(0, 128, 16, 8, 128) == 0

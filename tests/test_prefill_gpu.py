@@ -123,7 +123,7 @@ def test_two_stage_prefill_equals_one_call(gqa):
     inp = synthetic.prefill_inputs(2, 190, 8, 2, seed=33)
     d = to_dev(inp)
     one = gqa.prefill(d["q"], d["k"], d["v"], d["pos"], d["qnorm_w"], d["knorm_w"], d["theta"], d["eps"])
-    table = torch.empty((2, 190, 128), dtype=torch.float32, device="cuda")
+    table = torch.empty(gqa.rope_table_numel(2 * 190), dtype=torch.float32, device="cuda")
     khat = gqa.k_norm_rope(d["k"], d["pos"], d["knorm_w"], d["theta"], d["eps"], rope_cs=table)
     two = gqa.prefill_khat(d["q"], khat, d["v"], d["pos"], d["qnorm_w"], d["theta"], d["eps"], rope_cs=table)
     torch.cuda.synchronize()
@@ -145,11 +145,18 @@ def test_q_rope_without_table_matches_oracle(gqa):
 
 def test_rope_table_matches_closed_form(gqa):
     """The cos/sin table the K prologue writes: cos/sin(pos * theta^(-2i/D))."""
-    pos = torch.tensor([0, 1, 7, 4095, 32767], dtype=torch.int32)
-    k = torch.zeros((5, 1, 128), dtype=torch.bfloat16)
-    table = torch.empty((5, 128), dtype=torch.float32, device="cuda")
+    g = torch.Generator().manual_seed(36)
+    pos = torch.cat([torch.tensor([0, 1, 7, 4095, 32767]), torch.randint(0, 32768, (200,), generator=g)]).to(torch.int32)
+    n = pos.numel()
+    k = torch.zeros((n, 1, 128), dtype=torch.bfloat16)
+    table = torch.empty(gqa.rope_table_numel(n), dtype=torch.float32, device="cuda")
     gqa.k_norm_rope(k.cuda(), pos.cuda(), torch.ones(128, device="cuda"), 1e6, 1e-6, rope_cs=table)
     torch.cuda.synchronize()
-    ang = pos.double()[:, None] * (1e6 ** (-torch.arange(0, 128, 2, dtype=torch.float64) / 128))
-    ref = torch.stack([torch.cos(ang), torch.sin(ang)], -1).reshape(5, 128)
-    assert (table.cpu().double() - ref).abs().max().item() < 2e-6
+    tab = table.cpu()
+    worst = 0.0
+    for i in range(n):
+        for pair in (0, 1, 31, 62, 63):
+            c, s_ = gqa.rope_table_entry(tab, i, pair)
+            ang = float(pos[i]) * 1e6 ** (-2.0 * pair / 128)
+            worst = max(worst, abs(c - np.cos(ang)), abs(s_ - np.sin(ang)))
+    assert worst < 2e-6, worst
