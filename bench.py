@@ -39,7 +39,11 @@ from grouped_query_causal_b200 import synthetic  # noqa: E402
 METRIC = "prefill attn TFLOPS and decode KV-read GB/s on 1 B200, % of roofline"
 PREFILL = "large_prefill"
 DECODE = "batched_decode"
-KERNEL_SOURCES = ["prefill.cuh", "decode.cuh", "ptx.cuh", "rope.cuh", "gqa_attn.cu"]
+# The sources each kernel is compiled from; its ncu traffic figure is stale once they change.
+KERNEL_SOURCES = {
+    "attn_fwd_kernel": ["prefill.cuh", "ptx.cuh", "rope.cuh", "gqa_attn.cu"],
+    "decode_split_kernel": ["decode.cuh", "ptx.cuh", "rope.cuh", "gqa_attn.cu"],
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -67,9 +71,9 @@ def peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "grouped_query_causal_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -85,7 +89,7 @@ def traffic_from_profiles(kernel):
     except (OSError, ValueError):
         return None
     e = t.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or kernel not in KERNEL_SOURCES or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
