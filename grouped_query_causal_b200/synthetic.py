@@ -109,6 +109,48 @@ def decode_inputs(B: int = 64, H: int = 32, Hkv: int = 8, D: int = HEAD_DIM, see
     return DecodeInputs(q, k_cache, v_cache, offsets, seqlens.to(torch.int32), wq)
 
 
+@dataclass
+class DecodeAppendInputs:
+    q: torch.Tensor        # bf16 [B,H,D], the new token's raw query
+    k_new: torch.Tensor    # bf16 [B,Hkv,D], the new token's raw key
+    v_new: torch.Tensor    # bf16 [B,Hkv,D], the new token's value
+    k_cache: torch.Tensor  # bf16 [rows,Hkv,D]; rows past a sequence's length hold stale data
+    v_cache: torch.Tensor  # bf16 [rows,Hkv,D]
+    offsets: torch.Tensor  # int64 [B+1]; sequence b owns rows offsets[b] .. offsets[b+1]-1
+    seqlens: torch.Tensor  # int32 [B], cached rows before the step (>= 0)
+    wq: torch.Tensor       # fp32 [D]
+    wk: torch.Tensor       # fp32 [D]
+    theta: float = THETA
+    eps: float = EPS
+
+    @property
+    def max_len(self) -> int:
+        """Keys attended after the append: the longest length + 1."""
+        return int(self.seqlens.max()) + 1 if self.seqlens.numel() else 0
+
+
+def decode_append_inputs(B: int = 64, H: int = 32, Hkv: int = 8, D: int = HEAD_DIM, seed: int = 0,
+                         len_lo: int = 1023, len_hi: int = 32767, seqlens=None,
+                         spare: int = 1) -> DecodeAppendInputs:
+    """A cache with `spare` free rows after each sequence's cached rows, plus one new token
+    per sequence.  Lengths U{len_lo..len_hi} unless given; every other value as in
+    decode_inputs."""
+    if seqlens is None:
+        seqlens = torch.randint(len_lo, len_hi + 1, (B,), generator=_gen(seed + 10), dtype=torch.int64)
+    seqlens = torch.as_tensor(seqlens, dtype=torch.int64).reshape(B)
+    offsets = torch.zeros(B + 1, dtype=torch.int64)
+    offsets[1:] = torch.cumsum(seqlens + spare, 0)
+    rows = int(offsets[-1])
+    q = _normal_bf16((B, H, D), seed)
+    k_cache = _normal_bf16((rows, Hkv, D), seed + 1)
+    v_cache = _normal_bf16((rows, Hkv, D), seed + 2)
+    wq = _uniform((D,), seed + 3, 0.5, 1.5)
+    wk = _uniform((D,), seed + 4, 0.5, 1.5)
+    k_new = _normal_bf16((B, Hkv, D), seed + 5)
+    v_new = _normal_bf16((B, Hkv, D), seed + 6)
+    return DecodeAppendInputs(q, k_new, v_new, k_cache, v_cache, offsets, seqlens.to(torch.int32), wq, wk)
+
+
 # The documented workloads, by name.
 WORKLOADS = {
     "prefill_correctness": dict(kind="prefill", B=1, T=128, H=16, Hkv=8),
@@ -119,6 +161,7 @@ WORKLOADS = {
     "large_prefill": dict(kind="prefill", B=4, T=4096, H=32, Hkv=8, scale=0.5),
     "batched_decode": dict(kind="decode", B=64, H=32, Hkv=8, len_lo=1024, len_hi=32768),
     "long_context_prefill": dict(kind="prefill", B=1, T=32768, H=64, Hkv=8),
+    "batched_decode_append": dict(kind="decode_append", B=64, H=32, Hkv=8, len_lo=1023, len_hi=32767),
 }
 
 
@@ -127,4 +170,6 @@ def make(name: str, seed: int = 0):
     kind = w.pop("kind")
     if kind == "prefill":
         return prefill_inputs(seed=seed, **w)
+    if kind == "decode_append":
+        return decode_append_inputs(seed=seed, **w)
     return decode_inputs(seed=seed, **w)

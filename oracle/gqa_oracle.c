@@ -319,6 +319,94 @@ void oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v
 }
 
 /* Number of threads the OpenMP runtime will use (reported beside the CPU timing). */
+/* One decode step with the new token appended to the cache first.  [A] D2-3: the new
+ * token's K and V go into the KV cache, and the token then attends to the whole cache;
+ * [C] "Attention 的 Forward 流程": q and k are normed, then rotated, before attention.
+ * Sequence b holds len_b = seqlens[b] >= 0 cached rows from row offsets[b] on (already
+ * normed and rotated K, raw V).  Its new token brings raw q [H, D], k_new [Hkv, D] and
+ * v_new [Hkv, D] (bf16 bits) and sits at position qpos[b] (default len_b).  The appended
+ * key of KV head g is k-hat = RoPE(RMSNorm(k_new[g]; w_k), position), the appended value
+ * is v_new[g] unchanged, and query head hq attends to the len_b cached rows of KV head
+ * hq / (H/Hkv) followed by that appended row: len_b + 1 keys, none masked.  khat_out
+ * [B, Hkv, D] receives the appended keys (fp64, before any storage rounding). */
+void oracle_decode_append(const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
+                          const uint16_t *k_cache, const uint16_t *v_cache,
+                          const int64_t *offsets, const int32_t *seqlens, const int32_t *qpos,
+                          const float *wq, const float *wk, double base, double eps, int B,
+                          int H, int Hkv, int D, double *out, double *khat_out)
+{
+    int h_per_kv = H / Hkv;
+    double inv_sqrt_d = 1.0 / sqrt((double)D);
+    int32_t maxkeys = 1;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] + 1 > maxkeys)
+            maxkeys = seqlens[b] + 1;
+    double *wqd = (double *)malloc(sizeof(double) * D);
+    double *wkd = (double *)malloc(sizeof(double) * D);
+    for (int d = 0; d < D; ++d) {
+        wqd[d] = (double)wq[d];
+        wkd[d] = (double)wk[d];
+    }
+    /* the appended keys first: one per (sequence, KV head) */
+    {
+        double *tmp = (double *)malloc(sizeof(double) * D);
+        for (int b = 0; b < B; ++b) {
+            int32_t position = qpos ? qpos[b] : seqlens[b];
+            for (int g = 0; g < Hkv; ++g)
+                norm_then_rope(k_new + ((int64_t)b * Hkv + g) * D, wkd, position, base, eps, D, tmp,
+                               khat_out + ((int64_t)b * Hkv + g) * D);
+        }
+        free(tmp);
+    }
+#pragma omp parallel
+    {
+        double *tmp = (double *)malloc(sizeof(double) * D);
+        double *qi = (double *)malloc(sizeof(double) * D);
+        double *s = (double *)malloc(sizeof(double) * maxkeys);
+        double *p = (double *)malloc(sizeof(double) * maxkeys);
+        double *vbuf = (double *)malloc(sizeof(double) * (size_t)maxkeys * D);
+        const double **vr = (const double **)malloc(sizeof(double *) * maxkeys);
+#pragma omp for collapse(2) schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b)
+            for (int hq = 0; hq < H; ++hq) {
+                int g = hq / h_per_kv;
+                int32_t len = seqlens[b];
+                int32_t position = qpos ? qpos[b] : len;
+                norm_then_rope(q + ((int64_t)b * H + hq) * D, wqd, position, base, eps, D, tmp, qi);
+                for (int32_t j = 0; j <= len; ++j) {
+                    double dot = 0.0;
+                    if (j < len) {
+                        int64_t row = offsets[b] + j;
+                        const uint16_t *kj = k_cache + (row * Hkv + g) * D;
+                        const uint16_t *vj = v_cache + (row * Hkv + g) * D;
+                        for (int d = 0; d < D; ++d) {
+                            dot += qi[d] * bf16_bits_to_double(kj[d]);
+                            vbuf[(int64_t)j * D + d] = bf16_bits_to_double(vj[d]);
+                        }
+                    } else {
+                        const double *kj = khat_out + ((int64_t)b * Hkv + g) * D;
+                        const uint16_t *vj = v_new + ((int64_t)b * Hkv + g) * D;
+                        for (int d = 0; d < D; ++d) {
+                            dot += qi[d] * kj[d];
+                            vbuf[(int64_t)j * D + d] = bf16_bits_to_double(vj[d]);
+                        }
+                    }
+                    s[j] = dot * inv_sqrt_d;
+                    vr[j] = vbuf + (int64_t)j * D;
+                }
+                softmax_weighted_sum(s, len + 1, vr, D, p, out + ((int64_t)b * H + hq) * D);
+            }
+        free(tmp);
+        free(qi);
+        free(s);
+        free(p);
+        free(vbuf);
+        free(vr);
+    }
+    free(wqd);
+    free(wkd);
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -53,6 +53,8 @@ def _load():
             lib.oracle_prefill_rows.argtypes = [P, P, P, P, P, P, Dd, Dd, I, I, I, I, I,
                                                 L, P, P]
             lib.oracle_decode.argtypes = [P, P, P, P, P, P, P, Dd, Dd, I, I, I, I, P]
+            lib.oracle_decode_append.argtypes = [P, P, P, P, P, P, P, P, P, P, Dd, Dd, I, I, I, I,
+                                                 P, P]
             lib.oracle_num_threads.restype = I
             _lib = lib
     return _lib
@@ -167,3 +169,31 @@ def decode(q_bits, k_cache_bits, v_cache_bits, offsets, seqlens, qpos, wq, theta
                           _p(seqlens), _p(qpos_a), _p(wq), theta, eps, B, H, Hkv, D,
                           _p(out))
     return out
+
+
+def decode_append(q_bits, k_new_bits, v_new_bits, k_cache_bits, v_cache_bits, offsets, seqlens,
+                  qpos, wq, wk, theta: float, eps: float):
+    """Decode step that appends the new token first: q [B,H,D], k_new / v_new [B,Hkv,D] bf16
+    bits; caches [rows,Hkv,D] bf16 bits; offsets [B(+1)] int64; seqlens [B] int32 (>= 0);
+    qpos [B] int32 or None (then qpos = seqlens).  Returns (out [B,H,D], k-hat of the
+    appended rows [B,Hkv,D]), both fp64."""
+    q_bits = _c(q_bits, np.uint16)
+    k_new_bits = _c(k_new_bits, np.uint16)
+    v_new_bits = _c(v_new_bits, np.uint16)
+    k_cache_bits = _c(k_cache_bits, np.uint16)
+    v_cache_bits = _c(v_cache_bits, np.uint16)
+    B, H, D = q_bits.shape
+    Hkv = k_new_bits.shape[1]
+    assert k_new_bits.shape == (B, Hkv, D) and v_new_bits.shape == (B, Hkv, D)
+    offsets = _c(offsets, np.int64)
+    seqlens = _c(seqlens, np.int32)
+    assert (seqlens >= 0).all()
+    qpos_a = None if qpos is None else _c(qpos, np.int32)
+    wq = _c(wq, np.float32)
+    wk = _c(wk, np.float32)
+    out = np.empty((B, H, D), np.float64)
+    khat = np.empty((B, Hkv, D), np.float64)
+    _load().oracle_decode_append(_p(q_bits), _p(k_new_bits), _p(v_new_bits), _p(k_cache_bits),
+                                 _p(v_cache_bits), _p(offsets), _p(seqlens), _p(qpos_a), _p(wq),
+                                 _p(wk), theta, eps, B, H, Hkv, D, _p(out), _p(khat))
+    return out, khat

@@ -383,3 +383,103 @@ def test_decode_matches_torch_fp64_on_ragged_cache():
         p = torch.softmax((kc @ qh[b][:, :, None])[..., 0] / math.sqrt(D), -1)                # [H,n]
         ref = (p[:, :, None] * vc).sum(1)
         np.testing.assert_allclose(got[b], ref.numpy(), rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------------------
+# Decode step with the new token appended to the cache first
+# --------------------------------------------------------------------------------------
+
+def test_decode_append_equals_the_last_row_of_prefill():
+    """Appending token L (normed, rotated K at position L; raw V) to a cache holding the
+    k-hat / v of tokens 0..L-1, then attending, is row L of the causal computation over
+    L + 1 tokens ("Qwen3系列1" D2-3: the new K/V enter the cache before attention)."""
+    B, L, H, Hkv, D = 3, 20, 8, 2, 32
+    inp = synthetic.prefill_inputs(B, L + 1, H, Hkv, D=D, seed=21)
+    ntok = B * (L + 1)
+    pos = inp.pos.numpy().reshape(ntok)
+    kh = oracle.qk_transform(_bits(inp.k).reshape(ntok, Hkv, D), pos, inp.wk.numpy(), inp.theta, inp.eps)
+    qh = oracle.qk_transform(_bits(inp.q).reshape(ntok, H, D), pos, inp.wq.numpy(), inp.theta, inp.eps)
+    kh = kh.reshape(B, L + 1, Hkv, D)
+    kh_cache = torch.from_numpy(kh[:, :L].copy()).to(torch.bfloat16)   # the cache stores bf16
+    # reference keys: cached rows as stored, the appended row exact
+    k_ref = np.concatenate([kh_cache.double().numpy(), kh[:, L:]], axis=1)
+    ref = oracle.sdpa_gqa(qh.reshape(B, L + 1, H, D), k_ref, inp.v.double().numpy())[:, L]
+    # the cache has one free row after each sequence
+    kc = torch.zeros(B, L + 1, Hkv, D, dtype=torch.bfloat16)
+    kc[:, :L] = kh_cache
+    vc = torch.zeros(B, L + 1, Hkv, D, dtype=torch.bfloat16)
+    vc[:, :L] = inp.v[:, :L]
+    offsets = np.arange(B + 1, dtype=np.int64) * (L + 1)
+    seqlens = np.full(B, L, np.int32)
+    got, khat = oracle.decode_append(_bits(inp.q)[:, L], _bits(inp.k)[:, L], _bits(inp.v)[:, L],
+                                     _bits(kc).reshape(-1, Hkv, D), _bits(vc).reshape(-1, Hkv, D),
+                                     offsets, seqlens, None, inp.wq.numpy(), inp.wk.numpy(), inp.theta, inp.eps)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(khat, kh[:, L])
+    # an explicit query position equal to the length is the default
+    got2, _ = oracle.decode_append(_bits(inp.q)[:, L], _bits(inp.k)[:, L], _bits(inp.v)[:, L],
+                                   _bits(kc).reshape(-1, Hkv, D), _bits(vc).reshape(-1, Hkv, D),
+                                   offsets, seqlens, seqlens, inp.wq.numpy(), inp.wk.numpy(), inp.theta,
+                                   inp.eps)
+    np.testing.assert_array_equal(got, got2)
+
+
+def test_decode_append_to_an_empty_cache_returns_the_new_value():
+    """With no cached rows the token attends only to itself: one key, weight 1, so every
+    query head of a group returns that group's new value exactly."""
+    B, H, Hkv, D = 3, 6, 3, 16
+    inp = synthetic.decode_append_inputs(B, H, Hkv, D, seed=22, seqlens=[0, 0, 0])
+    got, _ = oracle.decode_append(_bits(inp.q), _bits(inp.k_new), _bits(inp.v_new), _bits(inp.k_cache),
+                                  _bits(inp.v_cache), inp.offsets.numpy(), inp.seqlens.numpy(), None,
+                                  inp.wq.numpy(), inp.wk.numpy(), inp.theta, inp.eps)
+    v = inp.v_new.double().numpy()
+    for hq in range(H):
+        np.testing.assert_array_equal(got[:, hq], v[:, hq // (H // Hkv)])
+
+
+def test_decode_append_matches_torch_fp64_on_ragged_cache():
+    rng = np.random.default_rng(23)
+    B, H, Hkv, D = 4, 8, 2, 16
+    seqlens = np.array([0, 5, 17, 2], np.int32)
+    inp = synthetic.decode_append_inputs(B, H, Hkv, D, seed=23, seqlens=seqlens, spare=3)
+    qpos = rng.integers(0, 1000, B).astype(np.int32)
+    got, khat = oracle.decode_append(_bits(inp.q), _bits(inp.k_new), _bits(inp.v_new), _bits(inp.k_cache),
+                                     _bits(inp.v_cache), inp.offsets.numpy(), inp.seqlens.numpy(), qpos,
+                                     inp.wq.numpy(), inp.wk.numpy(), inp.theta, inp.eps)
+    inv_freq = 1.0 / (inp.theta ** (torch.arange(0, D, 2, dtype=torch.float64) / D))
+
+    def norm_rope(x, w, p):   # x [..., D] at positions p (broadcast over leading dims)
+        x = x.double()
+        xn = w.double() * x / torch.sqrt(x.pow(2).mean(-1, keepdim=True) + inp.eps)
+        ang = p[..., None] * inv_freq
+        c, s = torch.cos(ang), torch.sin(ang)
+        return torch.stack([xn[..., ::2] * c - xn[..., 1::2] * s, xn[..., ::2] * s + xn[..., 1::2] * c], -1).flatten(-2)
+
+    pq = torch.from_numpy(qpos).double()
+    qh = norm_rope(inp.q, inp.wq, pq[:, None])          # [B,H,D]
+    kn = norm_rope(inp.k_new, inp.wk, pq[:, None])      # [B,Hkv,D]
+    np.testing.assert_allclose(khat, kn.numpy(), rtol=0, atol=1e-13)
+    for b in range(B):
+        o0, n = int(inp.offsets[b]), int(seqlens[b])
+        kc = torch.cat([inp.k_cache[o0:o0 + n].double(), kn[b][None]], 0)          # [n+1,Hkv,D]
+        vc = torch.cat([inp.v_cache[o0:o0 + n].double(), inp.v_new[b][None].double()], 0)
+        kc = kc.permute(1, 0, 2).repeat_interleave(H // Hkv, 0)
+        vc = vc.permute(1, 0, 2).repeat_interleave(H // Hkv, 0)
+        p = torch.softmax((kc @ qh[b][:, :, None])[..., 0] / math.sqrt(D), -1)
+        np.testing.assert_allclose(got[b], (p[:, :, None] * vc).sum(1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_decode_append_ignores_rows_past_the_length():
+    """Stale rows after a sequence's cached rows (where the append writes) play no part."""
+    B, H, Hkv, D = 2, 4, 2, 16
+    inp = synthetic.decode_append_inputs(B, H, Hkv, D, seed=24, seqlens=[7, 3], spare=4)
+    args = (inp.offsets.numpy(), inp.seqlens.numpy(), None, inp.wq.numpy(), inp.wk.numpy(), inp.theta, inp.eps)
+    a, _ = oracle.decode_append(_bits(inp.q), _bits(inp.k_new), _bits(inp.v_new), _bits(inp.k_cache),
+                                _bits(inp.v_cache), *args)
+    kc, vc = inp.k_cache.clone(), inp.v_cache.clone()
+    for b in range(B):
+        lo = int(inp.offsets[b]) + int(inp.seqlens[b])
+        kc[lo:int(inp.offsets[b + 1])] = 7.0
+        vc[lo:int(inp.offsets[b + 1])] = -3.0
+    b_, _ = oracle.decode_append(_bits(inp.q), _bits(inp.k_new), _bits(inp.v_new), _bits(kc), _bits(vc), *args)
+    np.testing.assert_array_equal(a, b_)
