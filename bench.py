@@ -39,6 +39,7 @@ from grouped_query_causal_b200 import synthetic  # noqa: E402
 METRIC = "prefill attn TFLOPS and decode KV-read GB/s on 1 B200, % of roofline"
 PREFILL = "large_prefill"
 DECODE = "batched_decode"
+DECODE_APPEND = "batched_decode_append"
 # The sources each kernel is compiled from; its ncu traffic figure is stale once they change.
 KERNEL_SOURCES = {
     "attn_fwd_kernel": ["prefill.cuh", "ptx.cuh", "rope.cuh", "gqa_attn.cu"],
@@ -59,6 +60,13 @@ def decode_bytes(seqlens, H, Hkv, D=128):
     bf16 query and the fp32 output."""
     B = len(seqlens)
     return int(sum(int(s) for s in seqlens)) * Hkv * D * 2 * 2 + B * H * D * 2 + B * H * D * 4
+
+
+def decode_append_bytes(seqlens, H, Hkv, D=128):
+    """Algorithmic bytes of the append step: the new K/V rows read (bf16) and written into
+    the cache, then decode over seqlens[b] + 1 rows."""
+    B = len(seqlens)
+    return decode_bytes([int(s) + 1 for s in seqlens], H, Hkv, D) + 2 * B * Hkv * D * 2 * 2
 
 
 def peaks():
@@ -237,6 +245,9 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the public API with host buffers (pinned), copies timed
     e2e = run_e2e(gqa, pin, dec, dev, stream, rank, world, max(3, min(K, 10)))
 
+    # ---- the decode step that appends the new token first (its own timed region)
+    app = run_decode_append(gqa, dev, stream, world, K, args.warmup)
+
     if rank != 0:
         return None
     pk, pk_kind = peaks()
@@ -287,12 +298,65 @@ def run_ours(args, rank, world, local_rank):
                      "peak_source": f"bf16_tflops (burst) of {pk_kind}",
                      "peak_sustained": float(pk.get("bf16_tflops_sustained", tc))},
         "e2e": e2e["prefill"],
+        "decode_append": dict(app, roofline=dict(app["roofline"], peak=hbm,
+                                                 frac=round(app["roofline"]["achieved"] / hbm, 4),
+                                                 peak_source=f"hbm_gbs of {pk_kind}")),
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(pin, dec, budget_s=args.cpu_seconds)
     return line
+
+
+def run_decode_append(gqa, dev, stream, world, K, W):
+    """gqa_attn_decode_append on the batched append workload (64 sequences with
+    1023..32767 cached rows, one new token each), inputs resident, CUDA events around K
+    calls after W warm-up calls.  Every call writes the same rows with the same values."""
+    lib = gqa.load()
+    sh = stream.cuda_stream
+    w = synthetic.make(DECODE_APPEND)
+    B, H, D = w.q.shape
+    Hkv = w.k_cache.shape[1]
+    t = {n: getattr(w, n).to(dev) for n in ("q", "k_new", "v_new", "k_cache", "v_cache", "offsets", "seqlens",
+                                               "wq", "wk")}
+    out = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(gqa.decode_workspace_size(B, H, Hkv, w.max_len, D), dtype=torch.uint8, device=dev)
+    ptr = lambda x: x.data_ptr()  # noqa: E731
+
+    def call():
+        st = lib.gqa_attn_decode_append(ptr(t["q"]), ptr(t["k_new"]), ptr(t["v_new"]), ptr(t["k_cache"]),
+                                        ptr(t["v_cache"]), ptr(t["offsets"]), ptr(t["seqlens"]), None, ptr(t["wq"]),
+                                        ptr(t["wk"]), w.theta, w.eps, ptr(out), B, H, Hkv, D, w.max_len, ptr(ws),
+                                        ws.numel(), sh)
+        if st != 0:
+            raise RuntimeError(f"gqa_attn_decode_append failed with status {st}")
+
+    for _ in range(W):
+        call()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if gqa.device_status() != 0:
+        raise RuntimeError("device status error in the append-step timing")
+    ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
+    sec = float(ms.item()) / 1e3
+    nbytes = decode_append_bytes(w.seqlens.tolist(), H, Hkv, D)
+    gbs = nbytes * K / sec / 1e9
+    del t, out, ws
+    return {"value": round(world * gbs, 1), "unit": "GB/s", "ms": round(1e3 * sec / K, 4),
+            "workload": "64 sequences, cached rows U[1023,32767] + 1 appended, H32 Hkv8 D128",
+            "bytes_per_call": nbytes, "gpu_launches": 3 * K,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s", "traffic": None,
+                         "kernel": "decode_append_kernel + decode_split_kernel + decode_merge_kernel (one call)"}}
 
 
 def run_e2e(gqa, pin, dec, dev, stream, rank, world, steps):

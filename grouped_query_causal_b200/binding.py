@@ -23,7 +23,8 @@ STATUS_NAMES = {
 # Every symbol the header declares.
 EXPORTS = ("gqa_status_string", "gqa_attn_prefill_workspace_size", "gqa_attn_prefill",
            "gqa_attn_k_norm_rope", "gqa_attn_prefill_khat", "gqa_attn_decode_workspace_size",
-           "gqa_attn_decode", "gqa_attn_decode_noalloc", "gqa_attn_device_status")
+           "gqa_attn_decode", "gqa_attn_decode_append", "gqa_attn_decode_noalloc",
+           "gqa_attn_device_status")
 # Size of the library's built-in scratch used by gqa_attn_decode_noalloc.
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -60,6 +61,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_attn_decode_workspace_size.restype = Z
     lib.gqa_attn_decode.argtypes = [P, P, P, P, P, P, P, F, F, P, I, I, I, I, I, P, Z, P]
     lib.gqa_attn_decode.restype = I
+    lib.gqa_attn_decode_append.argtypes = [P, P, P, P, P, P, P, P, P, P, F, F, P, I, I, I, I, I, P, Z, P]
+    lib.gqa_attn_decode_append.restype = I
     lib.gqa_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, P, F, F, P, I, I, I, I, I, P]
     lib.gqa_attn_decode_noalloc.restype = I
     lib.gqa_attn_device_status.argtypes = [P]
@@ -232,6 +235,50 @@ def decode(q, k_cache, v_cache, cache_offsets, seqlens, qnorm_w, max_len: int,
                              int(max_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
                              _stream_handle(stream))
     _raise(st, "gqa_attn_decode")
+    return out
+
+
+def decode_append(q, k_new, v_new, k_cache, v_cache, cache_offsets, seqlens, qnorm_w, knorm_w,
+                  max_len: int, q_pos: Optional[torch.Tensor] = None, theta: float = 1.0e6,
+                  eps: float = 1e-6, out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Decode step that appends the new token first: k-hat of k_new [B,Hkv,D] (normed
+    with knorm_w, rotated at q_pos or seqlens[b]) and v_new [B,Hkv,D] go to row seqlens[b]
+    of each sequence in k_cache / v_cache (written in place), then q [B,H,D] attends to
+    rows 0..seqlens[b].  max_len bounds seqlens[b] + 1.  seqlens is not advanced."""
+    lib = load()
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_new, "k_new", torch.bfloat16, 3)
+    _check(v_new, "v_new", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 3)
+    _check(v_cache, "v_cache", torch.bfloat16, 3)
+    _check(cache_offsets, "cache_offsets", torch.int64, 1)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    _check(qnorm_w, "qnorm_w", torch.float32, 1)
+    _check(knorm_w, "knorm_w", torch.float32, 1)
+    if q_pos is not None:
+        _check(q_pos, "q_pos", torch.int32, 1)
+    B, H, D = q.shape
+    Hkv = k_cache.shape[1]
+    if k_cache.shape[2] != D or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape mismatch")
+    if k_new.shape != (B, Hkv, D) or v_new.shape != (B, Hkv, D):
+        raise ValueError("k_new and v_new must be [B, Hkv, D]")
+    if cache_offsets.shape != (B + 1,) or seqlens.shape != (B,):
+        raise ValueError("cache_offsets must be [B+1] and seqlens [B]")
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 3)
+    need = int(lib.gqa_attn_decode_workspace_size(B, H, Hkv, D, int(max_len)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib.gqa_attn_decode_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(cache_offsets), _ptr(seqlens), _ptr(q_pos), _ptr(qnorm_w),
+                                    _ptr(knorm_w), float(theta), float(eps), _ptr(out), B, H, Hkv, D,
+                                    int(max_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream_handle(stream))
+    _raise(st, "gqa_attn_decode_append")
     return out
 
 

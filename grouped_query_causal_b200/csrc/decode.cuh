@@ -12,6 +12,10 @@
 //    and the four warp partials are merged into one (m, l, O) per head.
 //  decode_merge_kernel: log-sum-exp combination of the chunk partials of each
 //    (sequence, query head):  O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c.
+//  decode_append_kernel: the decode step that first writes the new token into the
+//    cache ("Qwen3系列1" D2-3: K and V enter the per-layer cache before attention):
+//    k-hat = RoPE(RMSNorm(k_new; w_k)) at the token's position and v_new go to row
+//    len of each sequence; the split kernel then attends to len + 1 rows.
 #pragma once
 #include <cuda_runtime.h>
 
@@ -38,14 +42,16 @@ struct DecodeParams {
     float *out;               // [B, H, D]
     unsigned *err;
     int B, H, Hkv, hpg, maxC, max_len;
+    int len_add;              // rows attended beyond seqlens[b]: 1 after an append, else 0
     float eps;
     float scale_log2;         // log2(e) / sqrt(D)
     RopeFreqs rf;
 };
 
-// Device-side bounds of sequence b: 1 <= len <= max_len and len fits its rows.
+// Device-side bounds of sequence b, with len = seqlens[b] + len_add the rows attended:
+// 1 <= len <= max_len and len fits its rows.
 __device__ __forceinline__ bool decode_seq_ok(const DecodeParams &p, int b, int &len, long long &off) {
-    len = p.seqlens[b];
+    len = p.seqlens[b] + p.len_add;
     off = p.offsets[b];
     const long long cap = p.offsets[b + 1] - off;
     return len >= 1 && len <= p.max_len && static_cast<long long>(len) <= cap && off >= 0;
@@ -122,7 +128,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
 
     // ---- q prologue: RMSNorm + RoPE at the query position, scaled into base-2 logits
     {
-        const int ps = p.qpos ? p.qpos[b] : len;
+        const int ps = p.qpos ? p.qpos[b] : p.seqlens[b];
         float cs0, sn0, cs1, sn1;
         rope_cos_sin(ps, p.rf.inv_freq[2 * lane], cs0, sn0);
         rope_cos_sin(ps, p.rf.inv_freq[2 * lane + 1], cs1, sn1);
@@ -319,6 +325,60 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const __grid_constant
         L = fmaf(sc, p.part_ml[2 * slot + 1], L);
     }
     o[d] = O / L;
+}
+
+struct AppendParams {
+    const uint16_t *k_new;    // bf16 [B, Hkv, D]
+    const uint16_t *v_new;    // bf16 [B, Hkv, D]
+    uint16_t *kc;             // bf16 [rows, Hkv, D]
+    uint16_t *vc;             // bf16 [rows, Hkv, D]
+    const int64_t *offsets;   // [B + 1]
+    const int32_t *seqlens;   // [B], rows cached before the step
+    const int32_t *qpos;      // [B] or nullptr (position = seqlens[b])
+    const float *wk;          // [D]
+    unsigned *err;
+    int B, Hkv, max_len;
+    float eps;
+    RopeFreqs rf;
+};
+
+// One warp per (sequence, KV head): RMSNorm + RoPE of the new key at the token's
+// position, rounded to bf16, written to row seqlens[b] of the sequence; the new value
+// is copied next to it.  Lane l holds elements 4l .. 4l+3 (RoPE pairs 2l and 2l+1).
+// A sequence whose rows cannot take the new token is flagged and left untouched.
+__global__ void __launch_bounds__(128) decode_append_kernel(const __grid_constant__ AppendParams p) {
+    const int lane = threadIdx.x & 31;
+    const long long pair = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+    if (pair >= static_cast<long long>(p.B) * p.Hkv) return;
+    const int b = static_cast<int>(pair / p.Hkv);
+    const int g = static_cast<int>(pair % p.Hkv);
+    const int len = p.seqlens[b];
+    const long long off = p.offsets[b];
+    const long long cap = p.offsets[b + 1] - off;
+    if (!(len >= 0 && len + 1 <= p.max_len && static_cast<long long>(len) + 1 <= cap && off >= 0)) {
+        if (g == 0 && lane == 0) atomicOr(p.err, kErrInput);
+        return;
+    }
+    const int ps = p.qpos ? p.qpos[b] : len;
+    const size_t src = (static_cast<size_t>(b) * p.Hkv + g) * kHeadDim + 4 * lane;
+    const size_t dst = ((static_cast<size_t>(off) + len) * p.Hkv + g) * kHeadDim + 4 * lane;
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p.k_new + src);
+    const uint2 vraw = *reinterpret_cast<const uint2 *>(p.v_new + src);
+    const float x0 = bf16lo(raw.x), x1 = bf16hi(raw.x), x2 = bf16lo(raw.y), x3 = bf16hi(raw.y);
+    float ss = x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + p.eps);
+    const float4 w = reinterpret_cast<const float4 *>(p.wk)[lane];
+    const float a0 = w.x * x0 * inv, a1 = w.y * x1 * inv, a2 = w.z * x2 * inv, a3 = w.w * x3 * inv;
+    float cs0, sn0, cs1, sn1;
+    rope_cos_sin(ps, p.rf.inv_freq[2 * lane], cs0, sn0);
+    rope_cos_sin(ps, p.rf.inv_freq[2 * lane + 1], cs1, sn1);
+    uint2 o;
+    o.x = pack_bf16x2(a0 * cs0 - a1 * sn0, a0 * sn0 + a1 * cs0);
+    o.y = pack_bf16x2(a2 * cs1 - a3 * sn1, a2 * sn1 + a3 * cs1);
+    *reinterpret_cast<uint2 *>(p.kc + dst) = o;
+    *reinterpret_cast<uint2 *>(p.vc + dst) = vraw;
 }
 
 }  // namespace gqa

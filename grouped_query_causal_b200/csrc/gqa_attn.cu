@@ -290,11 +290,16 @@ gqa_status launch_decode(const DecodeParams &p, int npass, cudaStream_t st) {
 }
 }  // namespace
 
-extern "C" gqa_status gqa_attn_decode(const void *q, const void *k_cache, const void *v_cache,
-                                      const int64_t *cache_offsets, const int32_t *seqlens, const int32_t *q_pos,
-                                      const float *qnorm_w, float theta, float eps, float *out, int B, int H,
-                                      int Hkv, int D, int max_len, void *workspace, size_t workspace_bytes,
-                                      void *stream) {
+namespace {
+
+// Shared body of the decode entry points.  With k_new != nullptr the new token is first
+// appended to the cache (decode_append_kernel) and the split kernel attends to one row
+// more than seqlens[b].
+gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                       const int64_t *cache_offsets, const int32_t *seqlens, const int32_t *q_pos,
+                       const float *qnorm_w, const float *knorm_w, float theta, float eps, float *out, int B,
+                       int H, int Hkv, int D, int max_len, void *workspace, size_t workspace_bytes, void *stream) {
+    const bool append = k_new != nullptr || v_new != nullptr || knorm_w != nullptr;
     if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
     if (B < 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0) return GQA_ERR_INVALID_ARG;
     if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
@@ -307,10 +312,35 @@ extern "C" gqa_status gqa_attn_decode(const void *q, const void *k_cache, const 
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(qnorm_w, 16) ||
         !aligned(out, 4) || !aligned(cache_offsets, 8) || !aligned(seqlens, 4) || (q_pos && !aligned(q_pos, 4)))
         return GQA_ERR_INVALID_ARG;
+    if (append && (!k_new || !v_new || !knorm_w || !aligned(k_new, 8) || !aligned(v_new, 8) || !aligned(knorm_w, 16)))
+        return GQA_ERR_INVALID_ARG;
     const size_t need = gqa_attn_decode_workspace_size(B, H, Hkv, D, max_len);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
     unsigned *err = device_error_word();
     if (!err) return GQA_ERR_CUDA;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const RopeFreqs rf = rope_freqs(static_cast<double>(theta));
+    if (append) {
+        AppendParams ap;
+        ap.k_new = static_cast<const uint16_t *>(k_new);
+        ap.v_new = static_cast<const uint16_t *>(v_new);
+        ap.kc = static_cast<uint16_t *>(k_cache);
+        ap.vc = static_cast<uint16_t *>(v_cache);
+        ap.offsets = cache_offsets;
+        ap.seqlens = seqlens;
+        ap.qpos = q_pos;
+        ap.wk = knorm_w;
+        ap.err = err;
+        ap.B = B;
+        ap.Hkv = Hkv;
+        ap.max_len = max_len;
+        ap.eps = eps;
+        ap.rf = rf;
+        const long long warps = static_cast<long long>(B) * Hkv;
+        decode_append_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, st>>>(ap);
+        if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+    }
 
     const size_t slots = decode_slots(B, H, max_len);
     DecodeParams p;
@@ -331,16 +361,38 @@ extern "C" gqa_status gqa_attn_decode(const void *q, const void *k_cache, const 
     p.hpg = H / Hkv;
     p.maxC = static_cast<int>((static_cast<long long>(max_len) + kChunk - 1) / kChunk);
     p.max_len = max_len;
+    p.len_add = append ? 1 : 0;
     p.eps = eps;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim)));
-    p.rf = rope_freqs(static_cast<double>(theta));
+    p.rf = rf;
 
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int h = p.hpg;
     if (h == 1) return launch_decode<1>(p, 1, st);
     if (h == 2) return launch_decode<2>(p, 1, st);
     if (h <= 4) return launch_decode<4>(p, 1, st);
     return launch_decode<8>(p, (h + 7) / 8, st);
+}
+
+}  // namespace
+
+extern "C" gqa_status gqa_attn_decode(const void *q, const void *k_cache, const void *v_cache,
+                                      const int64_t *cache_offsets, const int32_t *seqlens, const int32_t *q_pos,
+                                      const float *qnorm_w, float theta, float eps, float *out, int B, int H,
+                                      int Hkv, int D, int max_len, void *workspace, size_t workspace_bytes,
+                                      void *stream) {
+    return decode_impl(q, nullptr, nullptr, const_cast<void *>(k_cache), const_cast<void *>(v_cache), cache_offsets,
+                       seqlens, q_pos, qnorm_w, nullptr, theta, eps, out, B, H, Hkv, D, max_len, workspace,
+                       workspace_bytes, stream);
+}
+
+extern "C" gqa_status gqa_attn_decode_append(const void *q, const void *k_new, const void *v_new, void *k_cache,
+                                             void *v_cache, const int64_t *cache_offsets, const int32_t *seqlens,
+                                             const int32_t *q_pos, const float *qnorm_w, const float *knorm_w,
+                                             float theta, float eps, float *out, int B, int H, int Hkv, int D,
+                                             int max_len, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!k_new || !v_new || !knorm_w) return GQA_ERR_INVALID_ARG;
+    return decode_impl(q, k_new, v_new, k_cache, v_cache, cache_offsets, seqlens, q_pos, qnorm_w, knorm_w, theta,
+                       eps, out, B, H, Hkv, D, max_len, workspace, workspace_bytes, stream);
 }
 
 namespace {

@@ -158,6 +158,40 @@ gqa_status gqa_attn_decode(const void *q, const void *k_cache, const void *v_cac
                            float *out, int B, int H, int Hkv, int D, int max_len,
                            void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Decode step that first appends the new token to the cache, then attends
+ * ("Qwen3系列1" D2-3: the new token's K and V are written into the per-layer cache
+ * before attention; "Qwen3" walkthrough, attention forward: q and k are normed, then
+ * rotated).  For sequence b with seqlens[b] = n cached rows:
+ *   row n of the sequence (row cache_offsets[b] + n) receives
+ *     K: RoPE(RMSNorm(k_new[b, g]; knorm_w, eps), position) rounded to bf16,
+ *     V: v_new[b, g] unchanged,
+ *   and the query, normed and rotated at the same position, attends to rows 0 .. n
+ *   (n + 1 keys).  position = q_pos[b], or n when q_pos is NULL.
+ *
+ *   q          bf16 [B, H, D]        raw query of the new token
+ *   k_new      bf16 [B, Hkv, D]      raw key of the new token (8-byte aligned)
+ *   v_new      bf16 [B, Hkv, D]      value of the new token (8-byte aligned)
+ *   k_cache, v_cache  bf16 [rows, Hkv, D]  written at row n of each sequence, read at 0 .. n
+ *   cache_offsets, q_pos, qnorm_w, theta, eps, out, workspace: as for gqa_attn_decode
+ *   seqlens    int32 [B]             rows cached before the step: 0 <= seqlens[b],
+ *                                    seqlens[b] + 1 <= max_len and
+ *                                    seqlens[b] + 1 <= cache_offsets[b+1] - cache_offsets[b]
+ *   knorm_w    fp32 [D]              k RMSNorm weight (16-byte aligned)
+ *   max_len    host-side upper bound on seqlens[b] + 1 (sizes the workspace)
+ *
+ * seqlens is not modified: the caller advances it after the step.  The K/V rows of the
+ * new token are in place when the call's work completes on the stream.  A sequence that
+ * breaks the bounds above is not written, gets NaN output and sets
+ * GQA_ERR_DEVICE_INPUT in the device status word.  Null k_new, v_new or knorm_w is
+ * GQA_ERR_INVALID_ARG; every other host-side check is gqa_attn_decode's.
+ */
+gqa_status gqa_attn_decode_append(const void *q, const void *k_new, const void *v_new, void *k_cache,
+                                  void *v_cache, const int64_t *cache_offsets, const int32_t *seqlens,
+                                  const int32_t *q_pos, const float *qnorm_w, const float *knorm_w,
+                                  float theta, float eps, float *out, int B, int H, int Hkv, int D,
+                                  int max_len, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Size of the library's built-in decode scratch used by gqa_attn_decode_noalloc. */
 #define GQA_NOALLOC_SCRATCH_BYTES (32u << 20)
 

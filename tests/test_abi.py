@@ -109,6 +109,28 @@ def test_decode_argument_errors_are_caught_on_the_host(lib):
     assert _decode(lib, B=0) == 0
 
 
+def _decode_append(lib, **kw):
+    a = dict(q=16, kn=16, vn=16, kc=16, vc=16, offs=16, sl=16, qpos=None, wq=16, wk=16, theta=1e6, eps=1e-6,
+             out=16, B=2, H=8, Hkv=2, D=128, max_len=100, ws=256, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return lib.gqa_attn_decode_append(a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["offs"], a["sl"], a["qpos"],
+                                      a["wq"], a["wk"], a["theta"], a["eps"], a["out"], a["B"], a["H"], a["Hkv"],
+                                      a["D"], a["max_len"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_decode_append_argument_errors_are_caught_on_the_host(lib):
+    assert _decode_append(lib, kn=None) == -1
+    assert _decode_append(lib, vn=None) == -1
+    assert _decode_append(lib, wk=None) == -1
+    assert _decode_append(lib, kn=20) == -1     # new rows must be 8-byte aligned
+    assert _decode_append(lib, wk=24) == -1     # knorm_w must be 16-byte aligned
+    assert _decode_append(lib, D=256) == -2
+    assert _decode_append(lib, H=8, Hkv=3) == -1
+    assert _decode_append(lib, max_len=0) == -1
+    assert _decode_append(lib, wsb=10) == -3
+    assert _decode_append(lib, B=0) == 0
+
+
 def test_binding_fails_loudly_without_the_library(tmp_path):
     saved = binding._lib
     binding._lib = None
