@@ -5,11 +5,14 @@
 // work is bandwidth-bound: every cached K/V row is read exactly once, shared by the
 // h = H/Hkv query heads of its group ("深入剖析Qwen3模型架构" 3.1.2).
 //
-//  decode_split_kernel: one CTA per (sequence, KV head, 512-key chunk, head pass).
+//  decode_split_kernel: one CTA per (sequence, KV head, 1024-key chunk, head pass).
 //    The h query vectors are normed + rotated at the query position in the prologue;
-//    each warp streams 128 keys of the chunk with 16-byte loads (a half-warp per
-//    256-byte key row), first K (scores for all h heads), then V (weighted sum),
-//    and the four warp partials are merged into one (m, l, O) per head.
+//    each warp streams 256 keys of the chunk with 16-byte loads (a half-warp per
+//    256-byte key row, 16 rows per batch, the next batch's loads issued before the
+//    current batch is used), first K (scores for all h heads), then V (weighted sum;
+//    its first batch is requested before the softmax of the scores), with packed
+//    two-lane fp32 FMAs (the kernel is otherwise issue-bound), and the four warp
+//    partials are merged into one (m, l, O) per head.
 //  decode_merge_kernel: log-sum-exp combination of the chunk partials of each
 //    (sequence, query head):  O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c.
 //  decode_append_kernel: the decode step that first writes the new token into the
@@ -24,9 +27,9 @@
 
 namespace gqa {
 
-constexpr int kChunk = 512;                // keys per split
+constexpr int kChunk = 1024;                // keys per split
 constexpr int kWarpKeys = kChunk / 4;      // keys per warp
-constexpr int kRowPairs = 8;               // row pairs in flight per warp (16 rows)
+constexpr int kRowPairs = 8;               // row pairs per batch (16 rows); two batches in flight
 constexpr int kMaxHeadsPerPass = 8;
 
 struct DecodeParams {
@@ -160,11 +163,11 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
 
     const int sub = lane & 15;    // elements 8*sub .. 8*sub+7 of a row
     const int rsel = lane >> 4;   // which row of the pair
-    float qr[HG][8];
+    float2 qr[HG][4];   // pairs of query elements, for packed two-lane FMAs
 #pragma unroll
     for (int jj = 0; jj < HG; ++jj)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) qr[jj][e] = sq[jj][8 * sub + e];
+        for (int e = 0; e < 4; ++e) qr[jj][e] = make_float2(sq[jj][8 * sub + 2 * e], sq[jj][8 * sub + 2 * e + 1]);
 
     const int kw0 = k0 + warp * kWarpKeys;
     const int kw1 = min(k1, kw0 + kWarpKeys);
@@ -177,34 +180,45 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     const int my_head = decode_head_of_lane<HG>(lane);
 
     // ---- K sweep: base-2 logits of the HG heads for each key of this warp
+    uint4 kn[kRowPairs];
+#pragma unroll
+    for (int u = 0; u < kRowPairs; ++u) {
+        const int row = kw0 + 2 * u + rsel;
+        kn[u] = row < kw1 ? ldg_stream_v4(kbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
+    }
     for (int base = kw0; base < kw1; base += 2 * kRowPairs) {
         uint4 kv[kRowPairs];
 #pragma unroll
+        for (int u = 0; u < kRowPairs; ++u) kv[u] = kn[u];
+#pragma unroll
         for (int u = 0; u < kRowPairs; ++u) {
-            const int row = base + 2 * u + rsel;
-            kv[u] = row < kw1 ? ldg_stream_v4(kbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
+            const int row = base + 2 * kRowPairs + 2 * u + rsel;
+            kn[u] = row < kw1 ? ldg_stream_v4(kbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int u = 0; u < kRowPairs; ++u) {
             const uint32_t rw[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
-            float x[8];
+            float2 x[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                x[2 * i] = bf16lo(rw[i]);
-                x[2 * i + 1] = bf16hi(rw[i]);
-            }
+            for (int i = 0; i < 4; ++i) x[i] = make_float2(bf16lo(rw[i]), bf16hi(rw[i]));
             float part[HG];
 #pragma unroll
             for (int jj = 0; jj < HG; ++jj) {
-                float acc = 0.f;
+                float2 acc = __fmul2_rn(qr[jj][0], x[0]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc = fmaf(qr[jj][e], x[e], acc);
-                part[jj] = acc;
+                for (int e = 1; e < 4; ++e) acc = __ffma2_rn(qr[jj][e], x[e], acc);
+                part[jj] = acc.x + acc.y;
             }
             const float sfull = decode_reduce_heads<HG>(part, lane);
             const int rl = base + 2 * u + rsel - kw0;   // < kWarpKeys by construction
             if (writer) sw[rl * HG + my_head] = sfull;
         }
+    }
+    uint4 vn[kRowPairs];
+#pragma unroll
+    for (int u = 0; u < kRowPairs; ++u) {
+        const int row = kw0 + 2 * u + rsel;
+        vn[u] = row < kw1 ? ldg_stream_v4(vbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
     }
     __syncwarp();
 
@@ -225,17 +239,19 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     __syncwarp();
 
     // ---- V sweep: weighted sum of this warp's value rows
-    float acc[HG][8];
+    float2 acc[HG][4];
 #pragma unroll
     for (int jj = 0; jj < HG; ++jj)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[jj][e] = 0.f;
+        for (int e = 0; e < 4; ++e) acc[jj][e] = make_float2(0.f, 0.f);
     for (int base = kw0; base < kw1; base += 2 * kRowPairs) {
         uint4 vv[kRowPairs];
 #pragma unroll
+        for (int u = 0; u < kRowPairs; ++u) vv[u] = vn[u];
+#pragma unroll
         for (int u = 0; u < kRowPairs; ++u) {
-            const int row = base + 2 * u + rsel;
-            vv[u] = row < kw1 ? ldg_stream_v4(vbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
+            const int row = base + 2 * kRowPairs + 2 * u + rsel;
+            vn[u] = row < kw1 ? ldg_stream_v4(vbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int u = 0; u < kRowPairs; ++u) {
@@ -248,12 +264,9 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
                 const uint32_t rw[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float v0 = bf16lo(rw[i]), v1 = bf16hi(rw[i]);
+                    const float2 vv2 = make_float2(bf16lo(rw[i]), bf16hi(rw[i]));
 #pragma unroll
-                    for (int jj = 0; jj < HG; ++jj) {
-                        acc[jj][2 * i] = fmaf(pw[jj], v0, acc[jj][2 * i]);
-                        acc[jj][2 * i + 1] = fmaf(pw[jj], v1, acc[jj][2 * i + 1]);
-                    }
+                    for (int jj = 0; jj < HG; ++jj) acc[jj][i] = __ffma2_rn(make_float2(pw[jj], pw[jj]), vv2, acc[jj][i]);
                 }
             }
         }
@@ -261,14 +274,17 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
 #pragma unroll
     for (int jj = 0; jj < HG; ++jj)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[jj][e] += __shfl_xor_sync(0xffffffffu, acc[jj][e], 16);
+        for (int e = 0; e < 4; ++e) {
+            acc[jj][e].x += __shfl_xor_sync(0xffffffffu, acc[jj][e].x, 16);
+            acc[jj][e].y += __shfl_xor_sync(0xffffffffu, acc[jj][e].y, 16);
+        }
     __syncwarp();
     if (rsel == 0) {
 #pragma unroll
         for (int jj = 0; jj < HG; ++jj) {
             float4 *dst = reinterpret_cast<float4 *>(sw + jj * kHeadDim + 8 * sub);
-            dst[0] = make_float4(acc[jj][0], acc[jj][1], acc[jj][2], acc[jj][3]);
-            dst[1] = make_float4(acc[jj][4], acc[jj][5], acc[jj][6], acc[jj][7]);
+            dst[0] = make_float4(acc[jj][0].x, acc[jj][0].y, acc[jj][1].x, acc[jj][1].y);
+            dst[1] = make_float4(acc[jj][2].x, acc[jj][2].y, acc[jj][3].x, acc[jj][3].y);
         }
     }
     if (lane < HG) {

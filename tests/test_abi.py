@@ -51,7 +51,7 @@ def test_workspace_sizes(lib):
     assert lib.gqa_attn_prefill_workspace_size(1, 128, 16, 8, 64) == 0
     assert lib.gqa_attn_prefill_workspace_size(1, 128, 16, 3, 128) == 0
     assert lib.gqa_attn_prefill_workspace_size(0, 128, 16, 8, 128) == 0
-    slots = 64 * 64 * 32
+    slots = 64 * 32 * 32   # sequences x 1024-key chunks of 32768 keys x query heads
     assert lib.gqa_attn_decode_workspace_size(64, 32, 8, 128, 32768) == slots * 128 * 4 + slots * 2 * 4
     assert lib.gqa_attn_decode_workspace_size(2, 8, 2, 128, 1) == 2 * 8 * 128 * 4 + 256
     assert lib.gqa_attn_decode_workspace_size(2, 8, 3, 128, 100) == 0

@@ -65,7 +65,7 @@ def _check_cache(inp, kc, vc, khat_ref, idx=None, q_pos=None):
 def test_ragged_lengths(gqa, H, Hkv):
     """Lengths 0 (empty cache: the token attends only to itself), 1, chunk edges and a
     ragged tail; two spare rows per sequence."""
-    seqlens = [0, 1, 511, 512, 1023, 1500, 37]
+    seqlens = [0, 1, 511, 512, 1023, 1024, 1500, 37, 2047]
     inp = synthetic.decode_append_inputs(len(seqlens), H, Hkv, seed=31, seqlens=seqlens, spare=2)
     out, kc, vc = _run(gqa, inp)
     gqa.check_device_status()

@@ -57,7 +57,8 @@ def test_batched_decode_config(gqa):
 
 @pytest.mark.parametrize("H,Hkv", [(16, 16), (16, 8), (16, 4), (16, 1), (12, 4), (10, 2), (32, 8)])
 def test_group_sizes(gqa, H, Hkv):
-    seqlens = [1, 511, 512, 513, 1500, 37]
+    # chunk edges (1024-key chunks, 16-row load batches) and ragged tails
+    seqlens = [1, 511, 512, 513, 1500, 37, 1023, 1024, 1025, 2049, 16, 17]
     inp = synthetic.decode_inputs(len(seqlens), H, Hkv, seed=H * 100 + Hkv, seqlens=seqlens)
     got = _run(gqa, inp)
     gqa.check_device_status()
