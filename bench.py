@@ -62,6 +62,21 @@ def decode_bytes(seqlens, H, Hkv, D=128):
     return int(sum(int(s) for s in seqlens)) * Hkv * D * 2 * 2 + B * H * D * 2 + B * H * D * 4
 
 
+def max_over_ranks(values, device, world):
+    """Element-wise maximum of `values` (durations) over all ranks of the process group;
+    the values themselves when there is one rank."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(units_per_rank, world, seconds):
+    """Throughput of the whole job: every rank processed `units_per_rank` in at most
+    `seconds` (the maximum over ranks)."""
+    return world * units_per_rank / seconds
+
+
 def decode_append_bytes(seqlens, H, Hkv, D=128):
     """Algorithmic bytes of the append step: the new K/V rows read (bf16) and written into
     the cache, then decode over seqlens[b] + 1 rows."""
@@ -234,10 +249,7 @@ def run_ours(args, rank, world, local_rank):
     attn_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
     dec_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
     # max over ranks of every duration
-    times = torch.tensor([total_ms, pro_ms, attn_ms, dec_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    total_ms, pro_ms, attn_ms, dec_ms = times.tolist()
+    total_ms, pro_ms, attn_ms, dec_ms = max_over_ranks([total_ms, pro_ms, attn_ms, dec_ms], dev, world)
     K = args.steps
     prefill_s = (pro_ms + attn_ms) / 1e3
     dec_s = dec_ms / 1e3
@@ -261,7 +273,7 @@ def run_ours(args, rank, world, local_rank):
     traffic_dec = traffic_from_profiles("decode_split_kernel")
     line = {
         "metric": METRIC,
-        "value": round(world * flops * K / prefill_s / 1e12, 2),
+        "value": round(whole_job_rate(flops * K, world, prefill_s) / 1e12, 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": K,
@@ -283,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
         },
         "prefill_ms": round(1e3 * prefill_s / K, 4),
         "decode": {
-            "value": round(world * dbytes * K / dec_s / 1e9, 1),
+            "value": round(whole_job_rate(dbytes * K, world, dec_s) / 1e9, 1),
             "unit": "GB/s",
             "ms": round(1e3 * dec_s / K, 4),
             "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
@@ -345,14 +357,12 @@ def run_decode_append(gqa, dev, stream, world, K, W):
     torch.cuda.synchronize()
     if gqa.device_status() != 0:
         raise RuntimeError("device status error in the append-step timing")
-    ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
-    sec = float(ms.item()) / 1e3
+    sec = max_over_ranks([e0.elapsed_time(e1)], dev, world)[0] / 1e3
     nbytes = decode_append_bytes(w.seqlens.tolist(), H, Hkv, D)
     gbs = nbytes * K / sec / 1e9
     del t, out, ws
-    return {"value": round(world * gbs, 1), "unit": "GB/s", "ms": round(1e3 * sec / K, 4),
+    return {"value": round(whole_job_rate(nbytes * K, world, sec) / 1e9, 1), "unit": "GB/s",
+            "ms": round(1e3 * sec / K, 4),
             "workload": "64 sequences, cached rows U[1023,32767] + 1 appended, H32 Hkv8 D128",
             "bytes_per_call": nbytes, "gpu_launches": 3 * K,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s", "traffic": None,
@@ -419,11 +429,8 @@ def run_e2e(gqa, pin, dec, dev, stream, rank, world, steps):
                 raise RuntimeError(f"e2e {name} failed")
         b.record(stream)
         torch.cuda.synchronize()
-        ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
-        sec = ms.item() / 1e3
-        res[name] = {"value": round(world * units * steps / sec / scale, 3), "unit": unit,
+        sec = max_over_ranks([a.elapsed_time(b)], dev, world)[0] / 1e3
+        res[name] = {"value": round(whole_job_rate(units * steps, world, sec) / scale, 3), "unit": unit,
                      "h2d_bytes_per_step": int(b_in), "d2h_bytes_per_step": int(b_out), "steps": steps}
     return res
 
