@@ -82,20 +82,96 @@ void oracle_rope(const double *x, double pos, double base, int D, double *out)
     }
 }
 
+/* ---- RoPE variants: the frequency table, the pairing and the logit multiplier ----
+ *
+ * Frequencies theta_i, i = 0 .. D/2-1, for a base b and an extension factor s >= 1:
+ *   none    b^(-2i/D)                                   ([B] 3.4.1)
+ *   linear  b^(-2i/D) / s: the position divided by s     (the linear interpolation of
+ *           "Qwen3 技术报告深度解读" 4.2, i.e. Position Interpolation, Chen et al. 2023)
+ *   ntk     (b * s^(D/(D-2)))^(-2i/D): the base raised so that the lowest frequency is
+ *           divided by s and the highest is kept ("NTK-aware" scaling; the page's own
+ *           formula in 4.2 is garbled, so the published form is used)
+ *   yarn    "NTK-by-parts" of YaRN (Peng, Quesnelle, Fan, Shippole 2023, sec. 3.2-3.4;
+ *           the page's 3.4.2 snippet is garbled): with wavelength lambda_i = 2 pi / theta_i
+ *           and r_i = L / lambda_i (L the training context length),
+ *           gamma_i = clamp((r_i - beta_slow) / (beta_fast - beta_slow), 0, 1) and
+ *           theta'_i = (1 - gamma_i) theta_i / s + gamma_i theta_i;
+ *           the logits are multiplied by (0.1 ln s + 1)^2 (YaRN's temperature, applied
+ *           as sqrt(1/t) = 0.1 ln s + 1 on both q and k).
+ * Pairing: adjacent rotates (x[2i], x[2i+1]) by pos * theta_i ([A] D2-2, [B] 3.1.2);
+ * half rotates (x[i], x[i + D/2]) by the same angle (the rotate-half layout). */
+void oracle_rope_inv_freq(double base, int D, int scaling, double factor, int orig_max_pos,
+                          double beta_fast, double beta_slow, double *inv_freq)
+{
+    const double two_pi = 6.283185307179586476925286766559;
+    for (int i = 0; i < D / 2; ++i) {
+        double th = pow(base, -2.0 * (double)i / (double)D);
+        if (scaling == 1) {
+            th = th / factor;
+        } else if (scaling == 2) {
+            double b2 = base * pow(factor, (double)D / (double)(D - 2));
+            th = pow(b2, -2.0 * (double)i / (double)D);
+        } else if (scaling == 3) {
+            double r = (double)orig_max_pos / (two_pi / th);
+            double gamma = (r - beta_slow) / (beta_fast - beta_slow);
+            if (gamma < 0.0)
+                gamma = 0.0;
+            if (gamma > 1.0)
+                gamma = 1.0;
+            th = (1.0 - gamma) * th / factor + gamma * th;
+        }
+        inv_freq[i] = th;
+    }
+}
+
+double oracle_rope_logit_mult(int scaling, double factor)
+{
+    if (scaling == 3) {
+        double m = 0.1 * log(factor) + 1.0;
+        return m * m;
+    }
+    return 1.0;
+}
+
+/* RoPE of one head vector with a given frequency table and pairing (0 adjacent, 1 half). */
+void oracle_rope_ex(const double *x, double pos, const double *inv_freq, int pairing, int D,
+                    double *out)
+{
+    for (int i = 0; i < D / 2; ++i) {
+        double phi = pos * inv_freq[i];
+        double c = cos(phi), s = sin(phi);
+        int ia = pairing ? i : 2 * i;
+        int ib = pairing ? i + D / 2 : 2 * i + 1;
+        double a = x[ia], b = x[ib];
+        out[ia] = a * c - b * s;
+        out[ib] = a * s + b * c;
+    }
+}
+
+/* The plain frequency table b^(-2i/D) of [B] 3.4.1 (as oracle_rope uses), caller frees. */
+static double *plain_inv_freq(double base, int D)
+{
+    double *f = (double *)malloc(sizeof(double) * (D / 2 > 0 ? D / 2 : 1));
+    oracle_rope_inv_freq(base, D, 0, 1.0, 1, 32.0, 1.0, f);
+    return f;
+}
+
 /* q-hat / k-hat of one head vector: RMSNorm, then RoPE ([A] D2-2, [C] forward steps 4-5). */
-static void norm_then_rope(const uint16_t *xbits, const double *w, int32_t pos, double base,
-                           double eps, int D, double *tmp, double *out)
+static void norm_then_rope(const uint16_t *xbits, const double *w, int32_t pos,
+                           const double *inv_freq, int pairing, double eps, int D, double *tmp,
+                           double *out)
 {
     for (int d = 0; d < D; ++d)
         out[d] = bf16_bits_to_double(xbits[d]);
     oracle_rmsnorm(out, w, eps, D, tmp);
-    oracle_rope(tmp, (double)pos, base, D, out);
+    oracle_rope_ex(tmp, (double)pos, inv_freq, pairing, D, out);
 }
 
 /* Apply norm + RoPE to every head vector of x [N, nheads, D] with positions pos [N].
  * Exposes the oracle's q-hat / k-hat (used by the tests to build a decode cache). */
-void oracle_qk_transform(const uint16_t *x, const int32_t *pos, const float *w, double base,
-                         double eps, int64_t N, int nheads, int D, double *out)
+void oracle_qk_transform_ex(const uint16_t *x, const int32_t *pos, const float *w,
+                            const double *inv_freq, int pairing, double eps, int64_t N, int nheads,
+                            int D, double *out)
 {
     double *wd = (double *)malloc(sizeof(double) * D);
     for (int d = 0; d < D; ++d)
@@ -106,11 +182,19 @@ void oracle_qk_transform(const uint16_t *x, const int32_t *pos, const float *w, 
 #pragma omp for schedule(static)
         for (int64_t n = 0; n < N; ++n)
             for (int h = 0; h < nheads; ++h)
-                norm_then_rope(x + (n * nheads + h) * D, wd, pos[n], base, eps, D, tmp,
+                norm_then_rope(x + (n * nheads + h) * D, wd, pos[n], inv_freq, pairing, eps, D, tmp,
                                out + (n * nheads + h) * D);
         free(tmp);
     }
     free(wd);
+}
+
+void oracle_qk_transform(const uint16_t *x, const int32_t *pos, const float *w, double base,
+                         double eps, int64_t N, int nheads, int D, double *out)
+{
+    double *f = plain_inv_freq(base, D);
+    oracle_qk_transform_ex(x, pos, w, f, 0, eps, N, nheads, D, out);
+    free(f);
 }
 
 /* One output row of attention, [A] D1-4 / D1-2: given the scores s_j of the visible
@@ -205,14 +289,15 @@ void oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
  * full on a CPU).  rows holds nrows triples (b, hq, i); out is [nrows, D].  Each row
  * is computed from scratch by the same definition as oracle_prefill: q-hat of row i,
  * k-hat of keys 0..i of KV head hq / (H/Hkv), causal softmax, weighted sum of V. */
-void oracle_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                         const int32_t *pos, const float *wq, const float *wk, double base,
-                         double eps, int B, int T, int H, int Hkv, int D, int64_t nrows,
-                         const int64_t *rows, double *out)
+void oracle_prefill_rows_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            const int32_t *pos, const float *wq, const float *wk,
+                            const double *inv_freq, int pairing, double logit_mult, double eps,
+                            int B, int T, int H, int Hkv, int D, int64_t nrows, const int64_t *rows,
+                            double *out)
 {
     (void)B;
     int h_per_kv = H / Hkv;
-    double inv_sqrt_d = 1.0 / sqrt((double)D);
+    double inv_sqrt_d = logit_mult / sqrt((double)D);
     double *wqd = (double *)malloc(sizeof(double) * D);
     double *wkd = (double *)malloc(sizeof(double) * D);
     for (int d = 0; d < D; ++d) {
@@ -232,9 +317,11 @@ void oracle_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v
         for (int64_t r = 0; r < nrows; ++r) {
             int64_t b = rows[3 * r], hq = rows[3 * r + 1], i = rows[3 * r + 2];
             int64_t g = hq / h_per_kv;
-            norm_then_rope(q + ((b * T + i) * H + hq) * D, wqd, pos[b * T + i], base, eps, D, tmp, qi);
+            norm_then_rope(q + ((b * T + i) * H + hq) * D, wqd, pos[b * T + i], inv_freq, pairing, eps, D,
+                           tmp, qi);
             for (int64_t j = 0; j <= i; ++j) {
-                norm_then_rope(k + ((b * T + j) * Hkv + g) * D, wkd, pos[b * T + j], base, eps, D, tmp, kj);
+                norm_then_rope(k + ((b * T + j) * Hkv + g) * D, wkd, pos[b * T + j], inv_freq, pairing, eps,
+                               D, tmp, kj);
                 double dot = 0.0;
                 for (int d = 0; d < D; ++d)
                     dot += qi[d] * kj[d];
@@ -258,6 +345,16 @@ void oracle_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v
     free(wkd);
 }
 
+void oracle_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         const int32_t *pos, const float *wq, const float *wk, double base,
+                         double eps, int B, int T, int H, int Hkv, int D, int64_t nrows,
+                         const int64_t *rows, double *out)
+{
+    double *f = plain_inv_freq(base, D);
+    oracle_prefill_rows_ex(q, k, v, pos, wq, wk, f, 0, 1.0, eps, B, T, H, Hkv, D, nrows, rows, out);
+    free(f);
+}
+
 /* Decode: one new query token per sequence against its KV cache ([A] D2-3: prefill
  * writes K/V to the cache, decode feeds one token and reads the cache).
  * q [B,H,D] bf16 bits (raw: normed and rotated here at position qpos[b], or at
@@ -265,13 +362,13 @@ void oracle_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v
  * sequence b owning rows offsets[b] .. offsets[b]+seqlens[b]-1, which are used as
  * already-normed, already-rotated K and raw V; all of them are visible (the cache
  * holds only earlier positions).  out [B,H,D] fp64. */
-void oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
-                   const int64_t *offsets, const int32_t *seqlens, const int32_t *qpos,
-                   const float *wq, double base, double eps, int B, int H, int Hkv, int D,
-                   double *out)
+void oracle_decode_ex(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                      const int64_t *offsets, const int32_t *seqlens, const int32_t *qpos,
+                      const float *wq, const double *inv_freq, int pairing, double logit_mult,
+                      double eps, int B, int H, int Hkv, int D, double *out)
 {
     int h_per_kv = H / Hkv;
-    double inv_sqrt_d = 1.0 / sqrt((double)D);
+    double inv_sqrt_d = logit_mult / sqrt((double)D);
     int32_t maxlen = 1;
     for (int b = 0; b < B; ++b)
         if (seqlens[b] > maxlen)
@@ -293,7 +390,8 @@ void oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v
                 int g = hq / h_per_kv;
                 int32_t len = seqlens[b];
                 int32_t position = qpos ? qpos[b] : len;
-                norm_then_rope(q + ((int64_t)b * H + hq) * D, wqd, position, base, eps, D, tmp, qi);
+                norm_then_rope(q + ((int64_t)b * H + hq) * D, wqd, position, inv_freq, pairing, eps, D, tmp,
+                               qi);
                 for (int32_t j = 0; j < len; ++j) {
                     int64_t row = offsets[b] + j;
                     const uint16_t *kj = k_cache + (row * Hkv + g) * D;
@@ -318,6 +416,16 @@ void oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v
     free(wqd);
 }
 
+void oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                   const int64_t *offsets, const int32_t *seqlens, const int32_t *qpos,
+                   const float *wq, double base, double eps, int B, int H, int Hkv, int D,
+                   double *out)
+{
+    double *f = plain_inv_freq(base, D);
+    oracle_decode_ex(q, k_cache, v_cache, offsets, seqlens, qpos, wq, f, 0, 1.0, eps, B, H, Hkv, D, out);
+    free(f);
+}
+
 /* Number of threads the OpenMP runtime will use (reported beside the CPU timing). */
 /* One decode step with the new token appended to the cache first.  [A] D2-3: the new
  * token's K and V go into the KV cache, and the token then attends to the whole cache;
@@ -329,14 +437,15 @@ void oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v
  * is v_new[g] unchanged, and query head hq attends to the len_b cached rows of KV head
  * hq / (H/Hkv) followed by that appended row: len_b + 1 keys, none masked.  khat_out
  * [B, Hkv, D] receives the appended keys (fp64, before any storage rounding). */
-void oracle_decode_append(const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
-                          const uint16_t *k_cache, const uint16_t *v_cache,
-                          const int64_t *offsets, const int32_t *seqlens, const int32_t *qpos,
-                          const float *wq, const float *wk, double base, double eps, int B,
-                          int H, int Hkv, int D, double *out, double *khat_out)
+void oracle_decode_append_ex(const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
+                             const uint16_t *k_cache, const uint16_t *v_cache,
+                             const int64_t *offsets, const int32_t *seqlens, const int32_t *qpos,
+                             const float *wq, const float *wk, const double *inv_freq, int pairing,
+                             double logit_mult, double eps, int B, int H, int Hkv, int D,
+                             double *out, double *khat_out)
 {
     int h_per_kv = H / Hkv;
-    double inv_sqrt_d = 1.0 / sqrt((double)D);
+    double inv_sqrt_d = logit_mult / sqrt((double)D);
     int32_t maxkeys = 1;
     for (int b = 0; b < B; ++b)
         if (seqlens[b] + 1 > maxkeys)
@@ -353,8 +462,8 @@ void oracle_decode_append(const uint16_t *q, const uint16_t *k_new, const uint16
         for (int b = 0; b < B; ++b) {
             int32_t position = qpos ? qpos[b] : seqlens[b];
             for (int g = 0; g < Hkv; ++g)
-                norm_then_rope(k_new + ((int64_t)b * Hkv + g) * D, wkd, position, base, eps, D, tmp,
-                               khat_out + ((int64_t)b * Hkv + g) * D);
+                norm_then_rope(k_new + ((int64_t)b * Hkv + g) * D, wkd, position, inv_freq, pairing, eps, D,
+                               tmp, khat_out + ((int64_t)b * Hkv + g) * D);
         }
         free(tmp);
     }
@@ -372,7 +481,8 @@ void oracle_decode_append(const uint16_t *q, const uint16_t *k_new, const uint16
                 int g = hq / h_per_kv;
                 int32_t len = seqlens[b];
                 int32_t position = qpos ? qpos[b] : len;
-                norm_then_rope(q + ((int64_t)b * H + hq) * D, wqd, position, base, eps, D, tmp, qi);
+                norm_then_rope(q + ((int64_t)b * H + hq) * D, wqd, position, inv_freq, pairing, eps, D, tmp,
+                               qi);
                 for (int32_t j = 0; j <= len; ++j) {
                     double dot = 0.0;
                     if (j < len) {
@@ -405,6 +515,18 @@ void oracle_decode_append(const uint16_t *q, const uint16_t *k_new, const uint16
     }
     free(wqd);
     free(wkd);
+}
+
+void oracle_decode_append(const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
+                          const uint16_t *k_cache, const uint16_t *v_cache,
+                          const int64_t *offsets, const int32_t *seqlens, const int32_t *qpos,
+                          const float *wq, const float *wk, double base, double eps, int B,
+                          int H, int Hkv, int D, double *out, double *khat_out)
+{
+    double *f = plain_inv_freq(base, D);
+    oracle_decode_append_ex(q, k_new, v_new, k_cache, v_cache, offsets, seqlens, qpos, wq, wk, f, 0, 1.0,
+                            eps, B, H, Hkv, D, out, khat_out);
+    free(f);
 }
 
 int oracle_num_threads(void)

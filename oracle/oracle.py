@@ -55,6 +55,16 @@ def _load():
             lib.oracle_decode.argtypes = [P, P, P, P, P, P, P, Dd, Dd, I, I, I, I, P]
             lib.oracle_decode_append.argtypes = [P, P, P, P, P, P, P, P, P, P, Dd, Dd, I, I, I, I,
                                                  P, P]
+            lib.oracle_rope_inv_freq.argtypes = [Dd, I, I, Dd, I, Dd, Dd, P]
+            lib.oracle_rope_logit_mult.argtypes = [I, Dd]
+            lib.oracle_rope_logit_mult.restype = Dd
+            lib.oracle_rope_ex.argtypes = [P, Dd, P, I, I, P]
+            lib.oracle_qk_transform_ex.argtypes = [P, P, P, P, I, Dd, L, I, I, P]
+            lib.oracle_prefill_rows_ex.argtypes = [P, P, P, P, P, P, P, I, Dd, Dd, I, I, I, I, I, L,
+                                                   P, P]
+            lib.oracle_decode_ex.argtypes = [P, P, P, P, P, P, P, P, I, Dd, Dd, I, I, I, I, P]
+            lib.oracle_decode_append_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, Dd, Dd, I, I,
+                                                    I, I, P, P]
             lib.oracle_num_threads.restype = I
             _lib = lib
     return _lib
@@ -196,4 +206,109 @@ def decode_append(q_bits, k_new_bits, v_new_bits, k_cache_bits, v_cache_bits, of
     _load().oracle_decode_append(_p(q_bits), _p(k_new_bits), _p(v_new_bits), _p(k_cache_bits),
                                  _p(v_cache_bits), _p(offsets), _p(seqlens), _p(qpos_a), _p(wq),
                                  _p(wk), theta, eps, B, H, Hkv, D, _p(out), _p(khat))
+    return out, khat
+
+
+# ---- RoPE variants -------------------------------------------------------------------
+SCALINGS = {"none": 0, "linear": 1, "ntk": 2, "yarn": 3}
+PAIRINGS = {"adjacent": 0, "half": 1}
+
+
+class Rope:
+    """A RoPE variant: base theta, pairing ("adjacent" or "half"), scaling ("none",
+    "linear", "ntk", "yarn") with factor s, and YaRN's training length and ramp bounds."""
+
+    def __init__(self, theta=1.0e6, pairing="adjacent", scaling="none", factor=1.0,
+                 original_max_position=4096, beta_fast=32.0, beta_slow=1.0):
+        self.theta, self.pairing, self.scaling, self.factor = float(theta), pairing, scaling, float(factor)
+        self.original_max_position = int(original_max_position)
+        self.beta_fast, self.beta_slow = float(beta_fast), float(beta_slow)
+
+    def inv_freq(self, D: int) -> np.ndarray:
+        out = np.empty(D // 2, np.float64)
+        _load().oracle_rope_inv_freq(self.theta, D, SCALINGS[self.scaling], self.factor,
+                                     self.original_max_position, self.beta_fast, self.beta_slow,
+                                     _p(out))
+        return out
+
+    def logit_mult(self) -> float:
+        return float(_load().oracle_rope_logit_mult(SCALINGS[self.scaling], self.factor))
+
+    def pair_code(self) -> int:
+        return PAIRINGS[self.pairing]
+
+
+def rope_ex(x, pos: float, rope: Rope) -> np.ndarray:
+    x = _c(x, np.float64)
+    D = x.shape[-1]
+    f = rope.inv_freq(D)
+    out = np.empty_like(x)
+    _load().oracle_rope_ex(_p(x), float(pos), _p(f), rope.pair_code(), D, _p(out))
+    return out
+
+
+def qk_transform_ex(x_bits, pos, w, rope: Rope, eps: float) -> np.ndarray:
+    x_bits = _c(x_bits, np.uint16)
+    N, nh, D = x_bits.shape
+    pos = _c(pos, np.int32).reshape(N)
+    w = _c(w, np.float32)
+    f = rope.inv_freq(D)
+    out = np.empty((N, nh, D), np.float64)
+    _load().oracle_qk_transform_ex(_p(x_bits), _p(pos), _p(w), _p(f), rope.pair_code(), eps, N, nh, D,
+                                   _p(out))
+    return out
+
+
+def prefill_rows_ex(q_bits, k_bits, v_bits, pos, wq, wk, rope: Rope, eps: float, rows) -> np.ndarray:
+    q_bits = _c(q_bits, np.uint16)
+    k_bits = _c(k_bits, np.uint16)
+    v_bits = _c(v_bits, np.uint16)
+    B, T, H, D = q_bits.shape
+    Hkv = k_bits.shape[2]
+    pos = _c(pos, np.int32).reshape(B, T)
+    rows = _c(rows, np.int64).reshape(-1, 3)
+    assert (rows[:, 0] < B).all() and (rows[:, 1] < H).all() and (rows[:, 2] < T).all()
+    f = rope.inv_freq(D)
+    out = np.empty((rows.shape[0], D), np.float64)
+    _load().oracle_prefill_rows_ex(_p(q_bits), _p(k_bits), _p(v_bits), _p(pos), _p(_c(wq, np.float32)),
+                                   _p(_c(wk, np.float32)), _p(f), rope.pair_code(), rope.logit_mult(), eps,
+                                   B, T, H, Hkv, D, rows.shape[0], _p(rows), _p(out))
+    return out
+
+
+def decode_ex(q_bits, k_cache_bits, v_cache_bits, offsets, seqlens, qpos, wq, rope: Rope,
+              eps: float) -> np.ndarray:
+    q_bits = _c(q_bits, np.uint16)
+    k_cache_bits = _c(k_cache_bits, np.uint16)
+    v_cache_bits = _c(v_cache_bits, np.uint16)
+    B, H, D = q_bits.shape
+    Hkv = k_cache_bits.shape[1]
+    seqlens = _c(seqlens, np.int32)
+    assert (seqlens >= 1).all()
+    qpos_a = None if qpos is None else _c(qpos, np.int32)
+    f = rope.inv_freq(D)
+    out = np.empty((B, H, D), np.float64)
+    _load().oracle_decode_ex(_p(q_bits), _p(k_cache_bits), _p(v_cache_bits), _p(_c(offsets, np.int64)),
+                             _p(seqlens), _p(qpos_a), _p(_c(wq, np.float32)), _p(f), rope.pair_code(),
+                             rope.logit_mult(), eps, B, H, Hkv, D, _p(out))
+    return out
+
+
+def decode_append_ex(q_bits, k_new_bits, v_new_bits, k_cache_bits, v_cache_bits, offsets, seqlens,
+                     qpos, wq, wk, rope: Rope, eps: float):
+    q_bits = _c(q_bits, np.uint16)
+    k_new_bits = _c(k_new_bits, np.uint16)
+    v_new_bits = _c(v_new_bits, np.uint16)
+    B, H, D = q_bits.shape
+    Hkv = k_new_bits.shape[1]
+    seqlens = _c(seqlens, np.int32)
+    assert (seqlens >= 0).all()
+    qpos_a = None if qpos is None else _c(qpos, np.int32)
+    f = rope.inv_freq(D)
+    out = np.empty((B, H, D), np.float64)
+    khat = np.empty((B, Hkv, D), np.float64)
+    _load().oracle_decode_append_ex(_p(q_bits), _p(k_new_bits), _p(v_new_bits), _p(_c(k_cache_bits, np.uint16)),
+                                    _p(_c(v_cache_bits, np.uint16)), _p(_c(offsets, np.int64)), _p(seqlens),
+                                    _p(qpos_a), _p(_c(wq, np.float32)), _p(_c(wk, np.float32)), _p(f),
+                                    rope.pair_code(), rope.logit_mult(), eps, B, H, Hkv, D, _p(out), _p(khat))
     return out, khat

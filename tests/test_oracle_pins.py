@@ -483,3 +483,147 @@ def test_decode_append_ignores_rows_past_the_length():
         vc[lo:int(inp.offsets[b + 1])] = -3.0
     b_, _ = oracle.decode_append(_bits(inp.q), _bits(inp.k_new), _bits(inp.v_new), _bits(kc), _bits(vc), *args)
     np.testing.assert_array_equal(a, b_)
+
+
+# --------------------------------------------------------------------------------------
+# RoPE variants: rotate-half pairing and scaled frequencies (linear, NTK, YaRN)
+# --------------------------------------------------------------------------------------
+
+def _interleave(x, D):
+    """y[2i] = x[i], y[2i+1] = x[i + D/2] along the last axis."""
+    y = np.empty_like(x)
+    y[..., 0::2] = x[..., :D // 2]
+    y[..., 1::2] = x[..., D // 2:]
+    return y
+
+
+def _deinterleave(y, D):
+    x = np.empty_like(y)
+    x[..., :D // 2] = y[..., 0::2]
+    x[..., D // 2:] = y[..., 1::2]
+    return x
+
+
+def test_rope_defaults_equal_the_plain_rope():
+    rng = np.random.default_rng(40)
+    D = 16
+    x = rng.standard_normal(D)
+    r = oracle.Rope(theta=1e6)
+    np.testing.assert_array_equal(r.inv_freq(D), 1e6 ** (-np.arange(0, D, 2) / D))
+    for pos in (0, 3, 1000, 32767):
+        np.testing.assert_array_equal(oracle.rope_ex(x, pos, r), oracle.rope(x, pos, 1e6))
+    assert r.logit_mult() == 1.0
+    for sc in ("linear", "ntk", "yarn"):   # factor 1 is the plain RoPE for every method
+        np.testing.assert_allclose(oracle.Rope(scaling=sc, factor=1.0).inv_freq(D), r.inv_freq(D), rtol=1e-15)
+        assert oracle.Rope(scaling=sc, factor=1.0).logit_mult() == 1.0
+
+
+def test_half_pairing_is_adjacent_pairing_of_the_interleaved_vector():
+    """Rotating (x[i], x[i+D/2]) is rotating the adjacent pairs of the vector whose
+    halves are interleaved: half(x) = deinterleave(adjacent(interleave(x)))."""
+    rng = np.random.default_rng(41)
+    D = 32
+    x = rng.standard_normal(D)
+    for pos in (1, 77, 30000):
+        half = oracle.rope_ex(x, pos, oracle.Rope(pairing="half"))
+        adj = oracle.rope_ex(_interleave(x, D), pos, oracle.Rope())
+        np.testing.assert_allclose(half, _deinterleave(adj, D), rtol=0, atol=1e-15)
+        # it rotates: norm preserved, and pair 0 of (x0, x_{D/2}) turns by exactly pos radians
+        assert abs(np.linalg.norm(half) - np.linalg.norm(x)) < 1e-12
+        c, s = math.cos(pos), math.sin(pos)
+        assert abs(half[0] - (x[0] * c - x[D // 2] * s)) < 1e-12
+
+
+def test_linear_scaling_is_the_position_divided_by_the_factor():
+    rng = np.random.default_rng(42)
+    D = 16
+    x = rng.standard_normal(D)
+    for s in (2.0, 4.0, 8.0):
+        for p in (0, 5, 1000):
+            got = oracle.rope_ex(x, s * p, oracle.Rope(scaling="linear", factor=s))
+            np.testing.assert_allclose(got, oracle.rope(x, p, 1e6), rtol=0, atol=1e-12)
+
+
+def test_ntk_keeps_the_highest_frequency_and_divides_the_lowest_by_the_factor():
+    D = 128
+    base = oracle.Rope().inv_freq(D)
+    for s in (2.0, 8.0, 32.0):
+        f = oracle.Rope(scaling="ntk", factor=s).inv_freq(D)
+        assert f[0] == 1.0
+        assert abs(f[-1] / base[-1] - 1.0 / s) < 1e-12
+        ratio = f / base
+        assert (np.diff(ratio) < 0).all() and (ratio <= 1.0).all()   # interpolation grows with wavelength
+
+
+def test_yarn_by_parts_and_temperature():
+    """Pairs whose wavelength fits the training length more than beta_fast times keep their
+    frequency, pairs with fewer than beta_slow wavelengths are divided by s, the ones in
+    between blend linearly in the number of wavelengths; logits scale by (0.1 ln s + 1)^2."""
+    D, L = 128, 4096
+    base = oracle.Rope().inv_freq(D)
+    r = L * base / (2 * math.pi)           # wavelengths per training context
+    for s in (4.0, 16.0):
+        f = oracle.Rope(scaling="yarn", factor=s, original_max_position=L).inv_freq(D)
+        hi, lo = r > 32.0, r < 1.0
+        assert hi.any() and lo.any() and (~hi & ~lo).any()
+        np.testing.assert_array_equal(f[hi], base[hi])
+        np.testing.assert_allclose(f[lo], base[lo] / s, rtol=1e-15)
+        mid = ~hi & ~lo
+        gamma = (f[mid] - base[mid] / s) / (base[mid] - base[mid] / s)
+        np.testing.assert_allclose(gamma, (r[mid] - 1.0) / 31.0, rtol=1e-9)
+    assert abs(oracle.Rope(scaling="yarn", factor=math.exp(10.0)).logit_mult() - 4.0) < 1e-12
+    assert oracle.Rope(scaling="linear", factor=8.0).logit_mult() == 1.0
+
+
+def test_pipeline_defaults_equal_the_plain_pipeline():
+    B, T, H, Hkv, D = 2, 9, 4, 2, 16
+    inp = synthetic.prefill_inputs(B, T, H, Hkv, D=D, seed=43)
+    rows = np.array([(b, h, i) for b in range(B) for h in range(H) for i in range(T)], np.int64)
+    a = oracle.prefill_rows(_bits(inp.q), _bits(inp.k), _bits(inp.v), inp.pos.numpy(), inp.wq.numpy(),
+                            inp.wk.numpy(), inp.theta, inp.eps, rows)
+    b = oracle.prefill_rows_ex(_bits(inp.q), _bits(inp.k), _bits(inp.v), inp.pos.numpy(), inp.wq.numpy(),
+                               inp.wk.numpy(), oracle.Rope(theta=inp.theta), inp.eps, rows)
+    np.testing.assert_array_equal(a, b)
+    d = synthetic.decode_inputs(3, H, Hkv, D, seed=44, seqlens=[1, 4, 9])
+    args = (_bits(d.q), _bits(d.k_cache), _bits(d.v_cache), d.offsets.numpy(), d.seqlens.numpy(), None, d.wq.numpy())
+    np.testing.assert_array_equal(oracle.decode(*args, d.theta, d.eps),
+                                  oracle.decode_ex(*args, oracle.Rope(theta=d.theta), d.eps))
+
+
+def test_half_pairing_through_the_pipeline_is_adjacent_on_interleaved_heads():
+    """Scores depend on q-hat . k-hat only, which is unchanged when both vectors (and the
+    norm weights) have their head dimension interleaved the same way; V is untouched."""
+    B, T, H, Hkv, D = 1, 12, 4, 2, 16
+    inp = synthetic.prefill_inputs(B, T, H, Hkv, D=D, seed=45)
+    rows = np.array([(0, h, i) for h in range(H) for i in range(T)], np.int64)
+    il = lambda t: torch.from_numpy(_interleave(t.numpy(), D).copy())   # noqa: E731
+    got = oracle.prefill_rows_ex(_bits(inp.q), _bits(inp.k), _bits(inp.v), inp.pos.numpy(), inp.wq.numpy(),
+                                 inp.wk.numpy(), oracle.Rope(pairing="half"), inp.eps, rows)
+    ref = oracle.prefill_rows_ex(_bits(il(inp.q.float()).to(torch.bfloat16)), _bits(il(inp.k.float()).to(torch.bfloat16)),
+                                 _bits(inp.v), inp.pos.numpy(), il(inp.wq).numpy(), il(inp.wk).numpy(), oracle.Rope(),
+                                 inp.eps, rows)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_yarn_pipeline_matches_numpy_fp64():
+    """Decode with YaRN: q-hat from the (pinned) variant RoPE, logits times the temperature
+    factor, plain softmax, in numpy."""
+    B, H, Hkv, D = 2, 4, 2, 16
+    d = synthetic.decode_inputs(B, H, Hkv, D, seed=46, seqlens=[5, 11])
+    rope = oracle.Rope(scaling="yarn", factor=8.0, original_max_position=64)
+    got = oracle.decode_ex(_bits(d.q), _bits(d.k_cache), _bits(d.v_cache), d.offsets.numpy(), d.seqlens.numpy(),
+                           None, d.wq.numpy(), rope, d.eps)
+    m = rope.logit_mult()
+    assert m > 1.0
+    for b in range(B):
+        n, o0 = int(d.seqlens[b]), int(d.offsets[b])
+        for hq in range(H):
+            x = d.q[b, hq].double().numpy()
+            xn = d.wq.double().numpy() * x / np.sqrt((x * x).mean() + d.eps)
+            qh = oracle.rope_ex(xn, n, rope)
+            kc = d.k_cache[o0:o0 + n, hq // (H // Hkv)].double().numpy()
+            vc = d.v_cache[o0:o0 + n, hq // (H // Hkv)].double().numpy()
+            s = kc @ qh * m / math.sqrt(D)
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            np.testing.assert_allclose(got[b, hq], p @ vc, rtol=0, atol=1e-12)
