@@ -24,9 +24,36 @@ STATUS_NAMES = {
 EXPORTS = ("gqa_status_string", "gqa_attn_prefill_workspace_size", "gqa_attn_prefill",
            "gqa_attn_k_norm_rope", "gqa_attn_prefill_khat", "gqa_attn_decode_workspace_size",
            "gqa_attn_decode", "gqa_attn_decode_append", "gqa_attn_decode_noalloc",
-           "gqa_attn_device_status")
+           "gqa_attn_device_status", "gqa_attn_prefill_ex", "gqa_attn_k_norm_rope_ex",
+           "gqa_attn_prefill_khat_ex", "gqa_attn_decode_ex", "gqa_attn_decode_append_ex")
 # Size of the library's built-in scratch used by gqa_attn_decode_noalloc.
 NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+class RopeConfig(ctypes.Structure):
+    """gqa_rope_config: a RoPE variant (pairing "adjacent"/"half"; scaling "none",
+    "linear", "ntk" or "yarn" with factor s; YaRN's training length and ramp bounds)."""
+    _fields_ = [("theta", ctypes.c_double), ("pairing", ctypes.c_int), ("scaling", ctypes.c_int),
+                ("factor", ctypes.c_double), ("original_max_position", ctypes.c_int),
+                ("beta_fast", ctypes.c_double), ("beta_slow", ctypes.c_double)]
+
+    PAIRINGS = {"adjacent": 0, "half": 1}
+    SCALINGS = {"none": 0, "linear": 1, "ntk": 2, "yarn": 3}
+
+    @classmethod
+    def make(cls, theta: float = 1.0e6, pairing: str = "adjacent", scaling: str = "none",
+             factor: float = 1.0, original_max_position: int = 4096, beta_fast: float = 32.0,
+             beta_slow: float = 1.0) -> "RopeConfig":
+        return cls(float(theta), cls.PAIRINGS[pairing], cls.SCALINGS[scaling], float(factor),
+                   int(original_max_position), float(beta_fast), float(beta_slow))
+
+
+def _rope_call(lib, name: str, rope: Optional["RopeConfig"], theta: float):
+    """The entry point to call and the argument that goes where theta sits: the plain
+    symbol with theta, or its _ex form with a pointer to the RoPE configuration."""
+    if rope is None:
+        return getattr(lib, name), float(theta)
+    return getattr(lib, name + "_ex"), ctypes.byref(rope)
 
 
 class GqaError(RuntimeError):
@@ -67,6 +94,15 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_attn_decode_noalloc.restype = I
     lib.gqa_attn_device_status.argtypes = [P]
     lib.gqa_attn_device_status.restype = I
+    R = ctypes.POINTER(RopeConfig)
+    lib.gqa_attn_prefill_ex.argtypes = [P, P, P, P, P, P, R, F, P, I, I, I, I, I, P, Z, P]
+    lib.gqa_attn_k_norm_rope_ex.argtypes = [P, P, P, R, F, P, P, ctypes.c_int64, I, I, P]
+    lib.gqa_attn_prefill_khat_ex.argtypes = [P, P, P, P, P, P, R, F, P, I, I, I, I, I, P]
+    lib.gqa_attn_decode_ex.argtypes = [P, P, P, P, P, P, P, R, F, P, I, I, I, I, I, P, Z, P]
+    lib.gqa_attn_decode_append_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, R, F, P, I, I, I, I, I, P, Z, P]
+    for n in ("gqa_attn_prefill_ex", "gqa_attn_k_norm_rope_ex", "gqa_attn_prefill_khat_ex", "gqa_attn_decode_ex",
+              "gqa_attn_decode_append_ex"):
+        getattr(lib, n).restype = I
     _lib = lib
     return lib
 
@@ -120,9 +156,10 @@ def decode_workspace_size(B: int, H: int, Hkv: int, max_len: int, D: int = 128) 
 
 def prefill(q, k, v, pos, qnorm_w, knorm_w, theta: float = 1.0e6, eps: float = 1e-6,
             out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+            stream: Optional[torch.cuda.Stream] = None, rope: Optional[RopeConfig] = None) -> torch.Tensor:
     """Causal GQA prefill with fused q/k RMSNorm + RoPE.  q [B,T,H,D] bf16, k/v
-    [B,T,Hkv,D] bf16, pos [B,T] int32, norm weights [D] fp32 -> out [B,T,H,D] fp32."""
+    [B,T,Hkv,D] bf16, pos [B,T] int32, norm weights [D] fp32 -> out [B,T,H,D] fp32.
+    rope (a RopeConfig) selects a RoPE variant in place of theta."""
     lib = load()
     _check(q, "q", torch.bfloat16, 4)
     _check(k, "k", torch.bfloat16, 4)
@@ -142,16 +179,16 @@ def prefill(q, k, v, pos, qnorm_w, knorm_w, theta: float = 1.0e6, eps: float = 1
     need = int(lib.gqa_attn_prefill_workspace_size(B, T, H, Hkv, D))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = lib.gqa_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(qnorm_w), _ptr(knorm_w),
-                              float(theta), float(eps), _ptr(out), B, T, H, Hkv, D, _ptr(workspace),
-                              workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    fn, th = _rope_call(lib, "gqa_attn_prefill", rope, theta)
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(qnorm_w), _ptr(knorm_w), th, float(eps), _ptr(out), B, T,
+            H, Hkv, D, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _raise(st, "gqa_attn_prefill")
     return out
 
 
 def k_norm_rope(k, pos, knorm_w, theta: float = 1.0e6, eps: float = 1e-6,
                 out: Optional[torch.Tensor] = None, rope_cs: Optional[torch.Tensor] = None,
-                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+                stream: Optional[torch.cuda.Stream] = None, rope: Optional[RopeConfig] = None) -> torch.Tensor:
     """k-hat = RoPE(RMSNorm(k)) in bf16.  k [..., Hkv, D] bf16 with one position per
     token (pos has the leading shape of k) -> k_hat of k's shape (a decode cache).
     rope_cs (fp32, rope_table_numel(N) elements), when given, receives the tokens' RoPE
@@ -169,15 +206,16 @@ def k_norm_rope(k, pos, knorm_w, theta: float = 1.0e6, eps: float = 1e-6,
         raise ValueError("rope_cs must be a contiguous CUDA fp32 tensor of rope_table_numel(N) elements")
     if out is None:
         out = torch.empty_like(k)
-    st = lib.gqa_attn_k_norm_rope(_ptr(k), _ptr(pos), _ptr(knorm_w), float(theta), float(eps), _ptr(out),
-                                  _ptr(rope_cs), N, Hkv, D, _stream_handle(stream))
+    fn, th = _rope_call(lib, "gqa_attn_k_norm_rope", rope, theta)
+    st = fn(_ptr(k), _ptr(pos), _ptr(knorm_w), th, float(eps), _ptr(out), _ptr(rope_cs), N, Hkv, D,
+            _stream_handle(stream))
     _raise(st, "gqa_attn_k_norm_rope")
     return out
 
 
 def prefill_khat(q, k_hat, v, pos, qnorm_w, theta: float = 1.0e6, eps: float = 1e-6,
                  out: Optional[torch.Tensor] = None, rope_cs: Optional[torch.Tensor] = None,
-                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+                 stream: Optional[torch.cuda.Stream] = None, rope: Optional[RopeConfig] = None) -> torch.Tensor:
     """Attention stage of prefill on already normed + rotated keys (k_hat [B,T,Hkv,D]);
     rope_cs is the cos/sin table k_norm_rope wrote for the same tokens, or None."""
     lib = load()
@@ -196,8 +234,9 @@ def prefill_khat(q, k_hat, v, pos, qnorm_w, theta: float = 1.0e6, eps: float = 1
     if rope_cs is not None and (rope_cs.dtype != torch.float32 or not rope_cs.is_cuda or not rope_cs.is_contiguous()
                                 or rope_cs.numel() < rope_table_numel(B * T)):
         raise ValueError("rope_cs must be a contiguous CUDA fp32 tensor of rope_table_numel(B * T) elements")
-    st = lib.gqa_attn_prefill_khat(_ptr(q), _ptr(k_hat), _ptr(v), _ptr(pos), _ptr(rope_cs), _ptr(qnorm_w),
-                                   float(theta), float(eps), _ptr(out), B, T, H, Hkv, D, _stream_handle(stream))
+    fn, th = _rope_call(lib, "gqa_attn_prefill_khat", rope, theta)
+    st = fn(_ptr(q), _ptr(k_hat), _ptr(v), _ptr(pos), _ptr(rope_cs), _ptr(qnorm_w), th, float(eps), _ptr(out), B,
+            T, H, Hkv, D, _stream_handle(stream))
     _raise(st, "gqa_attn_prefill_khat")
     return out
 
@@ -205,7 +244,7 @@ def prefill_khat(q, k_hat, v, pos, qnorm_w, theta: float = 1.0e6, eps: float = 1
 def decode(q, k_cache, v_cache, cache_offsets, seqlens, qnorm_w, max_len: int,
            q_pos: Optional[torch.Tensor] = None, theta: float = 1.0e6, eps: float = 1e-6,
            out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+           stream: Optional[torch.cuda.Stream] = None, rope: Optional[RopeConfig] = None) -> torch.Tensor:
     """Split-KV decode.  q [B,H,D] bf16 (raw), caches [rows,Hkv,D] bf16 (normed/rotated
     K, raw V), cache_offsets [B+1] int64, seqlens [B] int32, q_pos [B] int32 or None
     (then the query sits at position seqlens[b]) -> out [B,H,D] fp32."""
@@ -230,10 +269,10 @@ def decode(q, k_cache, v_cache, cache_offsets, seqlens, qnorm_w, max_len: int,
     need = int(lib.gqa_attn_decode_workspace_size(B, H, Hkv, D, int(max_len)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = lib.gqa_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_offsets), _ptr(seqlens),
-                             _ptr(q_pos), _ptr(qnorm_w), float(theta), float(eps), _ptr(out), B, H, Hkv, D,
-                             int(max_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                             _stream_handle(stream))
+    fn, th = _rope_call(lib, "gqa_attn_decode", rope, theta)
+    st = fn(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_offsets), _ptr(seqlens), _ptr(q_pos), _ptr(qnorm_w),
+            th, float(eps), _ptr(out), B, H, Hkv, D, int(max_len), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _raise(st, "gqa_attn_decode")
     return out
 
@@ -242,7 +281,7 @@ def decode_append(q, k_new, v_new, k_cache, v_cache, cache_offsets, seqlens, qno
                   max_len: int, q_pos: Optional[torch.Tensor] = None, theta: float = 1.0e6,
                   eps: float = 1e-6, out: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None,
-                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+                  stream: Optional[torch.cuda.Stream] = None, rope: Optional[RopeConfig] = None) -> torch.Tensor:
     """Decode step that appends the new token first: k-hat of k_new [B,Hkv,D] (normed
     with knorm_w, rotated at q_pos or seqlens[b]) and v_new [B,Hkv,D] go to row seqlens[b]
     of each sequence in k_cache / v_cache (written in place), then q [B,H,D] attends to
@@ -273,11 +312,10 @@ def decode_append(q, k_new, v_new, k_cache, v_cache, cache_offsets, seqlens, qno
     need = int(lib.gqa_attn_decode_workspace_size(B, H, Hkv, D, int(max_len)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = lib.gqa_attn_decode_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
-                                    _ptr(cache_offsets), _ptr(seqlens), _ptr(q_pos), _ptr(qnorm_w),
-                                    _ptr(knorm_w), float(theta), float(eps), _ptr(out), B, H, Hkv, D,
-                                    int(max_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                    _stream_handle(stream))
+    fn, th = _rope_call(lib, "gqa_attn_decode_append", rope, theta)
+    st = fn(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(cache_offsets), _ptr(seqlens),
+            _ptr(q_pos), _ptr(qnorm_w), _ptr(knorm_w), th, float(eps), _ptr(out), B, H, Hkv, D, int(max_len),
+            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _raise(st, "gqa_attn_decode_append")
     return out
 

@@ -46,8 +46,9 @@ struct DecodeParams {
     unsigned *err;
     int B, H, Hkv, hpg, maxC, max_len;
     int len_add;              // rows attended beyond seqlens[b]: 1 after an append, else 0
+    int pairing;              // kPairAdjacent or kPairHalf
     float eps;
-    float scale_log2;         // log2(e) / sqrt(D)
+    float scale_log2;         // log2(e) / sqrt(D), times the RoPE variant's logit factor
     RopeFreqs rf;
 };
 
@@ -132,13 +133,10 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     // ---- q prologue: RMSNorm + RoPE at the query position, scaled into base-2 logits
     {
         const int ps = p.qpos ? p.qpos[b] : p.seqlens[b];
-        float cs0, sn0, cs1, sn1;
-        rope_cos_sin(ps, p.rf.inv_freq[2 * lane], cs0, sn0);
-        rope_cos_sin(ps, p.rf.inv_freq[2 * lane + 1], cs1, sn1);
         const float4 w = reinterpret_cast<const float4 *>(p.wq)[lane];
         for (int jj = warp; jj < HG; jj += 4) {
             const int j = jbase + jj;
-            float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+            float y[4] = {0.f, 0.f, 0.f, 0.f};
             if (j < p.hpg) {
                 const int hq = g * p.hpg + j;
                 const uint2 raw = *reinterpret_cast<const uint2 *>(p.q + (static_cast<size_t>(b) * p.H + hq) * kHeadDim + 4 * lane);
@@ -147,16 +145,16 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
 #pragma unroll
                 for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
                 const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + p.eps);
-                const float a0 = w.x * x0 * inv, a1 = w.y * x1 * inv, a2 = w.z * x2 * inv, a3 = w.w * x3 * inv;
-                y0 = a0 * cs0 - a1 * sn0;
-                y1 = a0 * sn0 + a1 * cs0;
-                y2 = a2 * cs1 - a3 * sn1;
-                y3 = a2 * sn1 + a3 * cs1;
+                y[0] = w.x * x0 * inv;
+                y[1] = w.y * x1 * inv;
+                y[2] = w.z * x2 * inv;
+                y[3] = w.w * x3 * inv;
             }
-            sq[jj][4 * lane + 0] = y0 * p.scale_log2;
-            sq[jj][4 * lane + 1] = y1 * p.scale_log2;
-            sq[jj][4 * lane + 2] = y2 * p.scale_log2;
-            sq[jj][4 * lane + 3] = y3 * p.scale_log2;
+            rope_warp4(y, ps, p.rf, p.pairing, lane);   // warp-uniform: j depends on the warp only
+            sq[jj][4 * lane + 0] = y[0] * p.scale_log2;
+            sq[jj][4 * lane + 1] = y[1] * p.scale_log2;
+            sq[jj][4 * lane + 2] = y[2] * p.scale_log2;
+            sq[jj][4 * lane + 3] = y[3] * p.scale_log2;
         }
     }
     __syncthreads();
@@ -354,13 +352,14 @@ struct AppendParams {
     const float *wk;          // [D]
     unsigned *err;
     int B, Hkv, max_len;
+    int pairing;              // kPairAdjacent or kPairHalf
     float eps;
     RopeFreqs rf;
 };
 
 // One warp per (sequence, KV head): RMSNorm + RoPE of the new key at the token's
 // position, rounded to bf16, written to row seqlens[b] of the sequence; the new value
-// is copied next to it.  Lane l holds elements 4l .. 4l+3 (RoPE pairs 2l and 2l+1).
+// is copied next to it.  Lane l holds elements 4l .. 4l+3.
 // A sequence whose rows cannot take the new token is flagged and left untouched.
 __global__ void __launch_bounds__(128) decode_append_kernel(const __grid_constant__ AppendParams p) {
     const int lane = threadIdx.x & 31;
@@ -386,13 +385,11 @@ __global__ void __launch_bounds__(128) decode_append_kernel(const __grid_constan
     for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + p.eps);
     const float4 w = reinterpret_cast<const float4 *>(p.wk)[lane];
-    const float a0 = w.x * x0 * inv, a1 = w.y * x1 * inv, a2 = w.z * x2 * inv, a3 = w.w * x3 * inv;
-    float cs0, sn0, cs1, sn1;
-    rope_cos_sin(ps, p.rf.inv_freq[2 * lane], cs0, sn0);
-    rope_cos_sin(ps, p.rf.inv_freq[2 * lane + 1], cs1, sn1);
+    float y[4] = {w.x * x0 * inv, w.y * x1 * inv, w.z * x2 * inv, w.w * x3 * inv};
+    rope_warp4(y, ps, p.rf, p.pairing, lane);
     uint2 o;
-    o.x = pack_bf16x2(a0 * cs0 - a1 * sn0, a0 * sn0 + a1 * cs0);
-    o.y = pack_bf16x2(a2 * cs1 - a3 * sn1, a2 * sn1 + a3 * cs1);
+    o.x = pack_bf16x2(y[0], y[1]);
+    o.y = pack_bf16x2(y[2], y[3]);
     *reinterpret_cast<uint2 *>(p.kc + dst) = o;
     *reinterpret_cast<uint2 *>(p.vc + dst) = vraw;
 }

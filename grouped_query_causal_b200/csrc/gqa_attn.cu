@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -82,6 +83,55 @@ RopeFreqs rope_freqs(double theta) {
     return rf;
 }
 
+// The kernels' form of a RoPE variant, or false for an invalid configuration.
+//   linear: theta_i / s;  ntk: (b s^(D/(D-2)))^(-2i/D);  yarn: with r_i = L theta_i / (2 pi)
+//   and gamma_i = clamp((r_i - beta_slow) / (beta_fast - beta_slow), 0, 1),
+//   theta_i ((1 - gamma_i) / s + gamma_i), and the logits times (0.1 ln s + 1)^2.
+bool rope_spec(const gqa_rope_config *c, RopeSpec &out) {
+    if (!c) return false;
+    if (!(c->theta > 0.0) || !std::isfinite(c->theta)) return false;
+    if (c->pairing != GQA_ROPE_PAIR_ADJACENT && c->pairing != GQA_ROPE_PAIR_HALF) return false;
+    if (c->scaling < GQA_ROPE_SCALE_NONE || c->scaling > GQA_ROPE_SCALE_YARN) return false;
+    const bool scaled = c->scaling != GQA_ROPE_SCALE_NONE;
+    if (scaled && (!(c->factor >= 1.0) || !std::isfinite(c->factor))) return false;
+    if (c->scaling == GQA_ROPE_SCALE_YARN &&
+        (c->original_max_position < 1 || !std::isfinite(c->beta_fast) || !std::isfinite(c->beta_slow) ||
+         !(c->beta_fast > c->beta_slow)))
+        return false;
+    const double s = scaled ? c->factor : 1.0;
+    const double two_pi = 6.283185307179586476925286766559;
+    const double ntk_base = c->theta * std::pow(s, static_cast<double>(kHeadDim) / (kHeadDim - 2));
+    for (int i = 0; i < kPairs; ++i) {
+        const double e = -2.0 * i / kHeadDim;
+        double th = std::pow(c->theta, e);
+        switch (c->scaling) {
+            case GQA_ROPE_SCALE_LINEAR: th /= s; break;
+            case GQA_ROPE_SCALE_NTK: th = std::pow(ntk_base, e); break;
+            case GQA_ROPE_SCALE_YARN: {
+                const double r = c->original_max_position * th / two_pi;
+                const double gamma = std::min(1.0, std::max(0.0, (r - c->beta_slow) / (c->beta_fast - c->beta_slow)));
+                th = (1.0 - gamma) * th / s + gamma * th;
+                break;
+            }
+            default: break;
+        }
+        out.rf.inv_freq[i] = th;
+    }
+    out.pairing = c->pairing == GQA_ROPE_PAIR_HALF ? kPairHalf : kPairAdjacent;
+    const double m = c->scaling == GQA_ROPE_SCALE_YARN ? 0.1 * std::log(s) + 1.0 : 1.0;
+    out.logit_mult = static_cast<float>(m * m);
+    return true;
+}
+
+// The plain RoPE of base theta (adjacent pairs, no scaling).
+RopeSpec plain_rope(float theta) {
+    RopeSpec r;
+    r.rf = rope_freqs(static_cast<double>(theta));
+    r.pairing = kPairAdjacent;
+    r.logit_mult = 1.0f;
+    return r;
+}
+
 int attn_sm_count() {
     static std::atomic<int> cache[kMaxDevices];
     const int dev = current_device();
@@ -98,7 +148,9 @@ bool attn_smem_attr_set() {
     const int dev = current_device();
     if (dev < 0) return false;
     if (done[dev].load()) return true;
-    if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_fwd_kernel<kPairAdjacent>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<kPairHalf>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess)
         return false;
     done[dev].store(1);
@@ -155,8 +207,10 @@ bool params_ok(float theta, float eps) {
     return theta > 0.f && std::isfinite(theta) && eps >= 0.f && std::isfinite(eps);
 }
 
+bool eps_ok(float eps) { return eps >= 0.f && std::isfinite(eps); }
+
 // Enqueue the k-hat prologue (arguments already validated).
-gqa_status launch_k_norm_rope(const void *k, const int32_t *pos, const float *knorm_w, const RopeFreqs &rf,
+gqa_status launch_k_norm_rope(const void *k, const int32_t *pos, const float *knorm_w, const RopeSpec &rs,
                               float eps, void *k_hat, float *rope_cs, long long ntok, int Hkv, cudaStream_t st) {
     KPrologueParams kp;
     kp.k = static_cast<const uint16_t *>(k);
@@ -167,17 +221,20 @@ gqa_status launch_k_norm_rope(const void *k, const int32_t *pos, const float *kn
     kp.ntok = ntok;
     kp.Hkv = Hkv;
     kp.eps = eps;
-    kp.rf = rf;
+    kp.rf = rs.rf;
     long long blocks = (ntok + 7) / 8;   // one warp per token, 8 warps per block
     const long long cap = static_cast<long long>(attn_sm_count()) * 8;
     if (blocks > cap) blocks = cap;
-    k_prologue_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(kp);
+    if (rs.pairing == kPairHalf)
+        k_prologue_kernel<kPairHalf><<<static_cast<unsigned>(blocks), 256, 0, st>>>(kp);
+    else
+        k_prologue_kernel<kPairAdjacent><<<static_cast<unsigned>(blocks), 256, 0, st>>>(kp);
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
 // Enqueue the attention kernel (arguments already validated).
 gqa_status launch_attention(const void *q, const void *k_hat, const void *v, const int32_t *pos,
-                            const float *rope_cs, const float *qnorm_w, const RopeFreqs &rf, float eps, float *out,
+                            const float *rope_cs, const float *qnorm_w, const RopeSpec &rs, float eps, float *out,
                             int B, int T, int H, int Hkv, cudaStream_t st) {
     unsigned *err = device_error_word();
     if (!err) return GQA_ERR_CUDA;
@@ -200,22 +257,26 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
     ap.nqb = (T + kBM - 1) / kBM;
     ap.npairs = (ap.hpg + 1) / 2;
     ap.eps = eps;
-    ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim)));
-    ap.rf = rf;
+    ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim))) * rs.logit_mult;
+    ap.rf = rs.rf;
     const long long jobs = static_cast<long long>(ap.nqb) * B * Hkv * ap.npairs;
     if (jobs <= 0 || jobs > 0x7fffffffLL) return GQA_ERR_INVALID_ARG;
-    attn_fwd_kernel<<<static_cast<unsigned>(jobs), kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
+    if (rs.pairing == kPairHalf)
+        attn_fwd_kernel<kPairHalf><<<static_cast<unsigned>(jobs), kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
+    else
+        attn_fwd_kernel<kPairAdjacent><<<static_cast<unsigned>(jobs), kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v,
+                                                                                                   ap);
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
 }  // namespace
 
-extern "C" gqa_status gqa_attn_k_norm_rope(const void *k, const int32_t *pos, const float *knorm_w, float theta,
-                                           float eps, void *k_hat, float *rope_cs, int64_t N, int Hkv, int D,
-                                           void *stream) {
+namespace {
+
+gqa_status k_norm_rope_impl(const void *k, const int32_t *pos, const float *knorm_w, const RopeSpec &rs, float eps,
+                            void *k_hat, float *rope_cs, int64_t N, int Hkv, int D, void *stream) {
     if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
     if (N < 0 || Hkv <= 0 || N > (1LL << 31)) return GQA_ERR_INVALID_ARG;
-    if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
     if (N == 0) return GQA_OK;
     if (!k || !pos || !knorm_w || !k_hat) return GQA_ERR_INVALID_ARG;
     if (!aligned(k, 16) || !aligned(k_hat, 16) || !aligned(knorm_w, 16) || !aligned(pos, 4) ||
@@ -229,32 +290,28 @@ extern "C" gqa_status gqa_attn_k_norm_rope(const void *k, const int32_t *pos, co
         const size_t tb = round_up(static_cast<size_t>(N), 128) * kHeadDim * sizeof(float);
         if ((c < b + bytes && b < c + tb) || (c < a + bytes && a < c + tb)) return GQA_ERR_INVALID_ARG;
     }
-    return launch_k_norm_rope(k, pos, knorm_w, rope_freqs(static_cast<double>(theta)), eps, k_hat, rope_cs, N, Hkv,
-                              static_cast<cudaStream_t>(stream));
+    return launch_k_norm_rope(k, pos, knorm_w, rs, eps, k_hat, rope_cs, N, Hkv, static_cast<cudaStream_t>(stream));
 }
 
-extern "C" gqa_status gqa_attn_prefill_khat(const void *q, const void *k_hat, const void *v, const int32_t *pos,
-                                            const float *rope_cs, const float *qnorm_w, float theta, float eps,
-                                            float *out, int B, int T, int H, int Hkv, int D, void *stream) {
+gqa_status prefill_khat_impl(const void *q, const void *k_hat, const void *v, const int32_t *pos,
+                             const float *rope_cs, const float *qnorm_w, const RopeSpec &rs, float eps, float *out,
+                             int B, int T, int H, int Hkv, int D, void *stream) {
     if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
     if (!prefill_shape_ok(B, T, H, Hkv)) return GQA_ERR_INVALID_ARG;
-    if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
     if (B == 0 || T == 0) return GQA_OK;
     if (!q || !k_hat || !v || !pos || !qnorm_w || !out) return GQA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k_hat, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(qnorm_w, 16) ||
         !aligned(pos, 4) || (rope_cs && !aligned(rope_cs, 16)))
         return GQA_ERR_INVALID_ARG;
-    return launch_attention(q, k_hat, v, pos, rope_cs, qnorm_w, rope_freqs(static_cast<double>(theta)), eps, out, B,
-                            T, H, Hkv, static_cast<cudaStream_t>(stream));
+    return launch_attention(q, k_hat, v, pos, rope_cs, qnorm_w, rs, eps, out, B, T, H, Hkv,
+                            static_cast<cudaStream_t>(stream));
 }
 
-extern "C" gqa_status gqa_attn_prefill(const void *q, const void *k, const void *v, const int32_t *pos,
-                                       const float *qnorm_w, const float *knorm_w, float theta, float eps,
-                                       float *out, int B, int T, int H, int Hkv, int D, void *workspace,
-                                       size_t workspace_bytes, void *stream) {
+gqa_status prefill_impl(const void *q, const void *k, const void *v, const int32_t *pos, const float *qnorm_w,
+                        const float *knorm_w, const RopeSpec &rs, float eps, float *out, int B, int T, int H,
+                        int Hkv, int D, void *workspace, size_t workspace_bytes, void *stream) {
     if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
     if (!prefill_shape_ok(B, T, H, Hkv)) return GQA_ERR_INVALID_ARG;
-    if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
     if (B == 0 || T == 0) return GQA_OK;
     if (!q || !k || !v || !pos || !qnorm_w || !knorm_w || !out) return GQA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(qnorm_w, 16) ||
@@ -264,12 +321,64 @@ extern "C" gqa_status gqa_attn_prefill(const void *q, const void *k, const void 
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const RopeFreqs rf = rope_freqs(static_cast<double>(theta));
     float *table = reinterpret_cast<float *>(static_cast<char *>(workspace) + khat_bytes(B, T, Hkv));
     gqa_status s =
-        launch_k_norm_rope(k, pos, knorm_w, rf, eps, workspace, table, static_cast<long long>(B) * T, Hkv, st);
+        launch_k_norm_rope(k, pos, knorm_w, rs, eps, workspace, table, static_cast<long long>(B) * T, Hkv, st);
     if (s != GQA_OK) return s;
-    return launch_attention(q, workspace, v, pos, table, qnorm_w, rf, eps, out, B, T, H, Hkv, st);
+    return launch_attention(q, workspace, v, pos, table, qnorm_w, rs, eps, out, B, T, H, Hkv, st);
+}
+
+}  // namespace
+
+extern "C" gqa_status gqa_attn_k_norm_rope(const void *k, const int32_t *pos, const float *knorm_w, float theta,
+                                           float eps, void *k_hat, float *rope_cs, int64_t N, int Hkv, int D,
+                                           void *stream) {
+    if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
+    return k_norm_rope_impl(k, pos, knorm_w, plain_rope(theta), eps, k_hat, rope_cs, N, Hkv, D, stream);
+}
+
+extern "C" gqa_status gqa_attn_k_norm_rope_ex(const void *k, const int32_t *pos, const float *knorm_w,
+                                              const gqa_rope_config *rope, float eps, void *k_hat, float *rope_cs,
+                                              int64_t N, int Hkv, int D, void *stream) {
+    RopeSpec rs;
+    if (!rope_spec(rope, rs) || !eps_ok(eps)) return GQA_ERR_INVALID_ARG;
+    return k_norm_rope_impl(k, pos, knorm_w, rs, eps, k_hat, rope_cs, N, Hkv, D, stream);
+}
+
+extern "C" gqa_status gqa_attn_prefill_khat(const void *q, const void *k_hat, const void *v, const int32_t *pos,
+                                            const float *rope_cs, const float *qnorm_w, float theta, float eps,
+                                            float *out, int B, int T, int H, int Hkv, int D, void *stream) {
+    if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
+    return prefill_khat_impl(q, k_hat, v, pos, rope_cs, qnorm_w, plain_rope(theta), eps, out, B, T, H, Hkv, D,
+                             stream);
+}
+
+extern "C" gqa_status gqa_attn_prefill_khat_ex(const void *q, const void *k_hat, const void *v, const int32_t *pos,
+                                               const float *rope_cs, const float *qnorm_w,
+                                               const gqa_rope_config *rope, float eps, float *out, int B, int T,
+                                               int H, int Hkv, int D, void *stream) {
+    RopeSpec rs;
+    if (!rope_spec(rope, rs) || !eps_ok(eps)) return GQA_ERR_INVALID_ARG;
+    return prefill_khat_impl(q, k_hat, v, pos, rope_cs, qnorm_w, rs, eps, out, B, T, H, Hkv, D, stream);
+}
+
+extern "C" gqa_status gqa_attn_prefill(const void *q, const void *k, const void *v, const int32_t *pos,
+                                       const float *qnorm_w, const float *knorm_w, float theta, float eps,
+                                       float *out, int B, int T, int H, int Hkv, int D, void *workspace,
+                                       size_t workspace_bytes, void *stream) {
+    if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
+    return prefill_impl(q, k, v, pos, qnorm_w, knorm_w, plain_rope(theta), eps, out, B, T, H, Hkv, D, workspace,
+                        workspace_bytes, stream);
+}
+
+extern "C" gqa_status gqa_attn_prefill_ex(const void *q, const void *k, const void *v, const int32_t *pos,
+                                          const float *qnorm_w, const float *knorm_w, const gqa_rope_config *rope,
+                                          float eps, float *out, int B, int T, int H, int Hkv, int D,
+                                          void *workspace, size_t workspace_bytes, void *stream) {
+    RopeSpec rs;
+    if (!rope_spec(rope, rs) || !eps_ok(eps)) return GQA_ERR_INVALID_ARG;
+    return prefill_impl(q, k, v, pos, qnorm_w, knorm_w, rs, eps, out, B, T, H, Hkv, D, workspace, workspace_bytes,
+                        stream);
 }
 
 extern "C" size_t gqa_attn_decode_workspace_size(int B, int H, int Hkv, int D, int max_len) {
@@ -297,12 +406,12 @@ namespace {
 // more than seqlens[b].
 gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
                        const int64_t *cache_offsets, const int32_t *seqlens, const int32_t *q_pos,
-                       const float *qnorm_w, const float *knorm_w, float theta, float eps, float *out, int B,
+                       const float *qnorm_w, const float *knorm_w, const RopeSpec &rs, float eps, float *out, int B,
                        int H, int Hkv, int D, int max_len, void *workspace, size_t workspace_bytes, void *stream) {
     const bool append = k_new != nullptr || v_new != nullptr || knorm_w != nullptr;
     if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
     if (B < 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0) return GQA_ERR_INVALID_ARG;
-    if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
+    if (!eps_ok(eps)) return GQA_ERR_INVALID_ARG;
     if (B == 0) return GQA_OK;
     if (max_len <= 0) return GQA_ERR_INVALID_ARG;
     if ((static_cast<long long>(max_len) + kChunk - 1) / kChunk > 65535) return GQA_ERR_INVALID_ARG;
@@ -320,7 +429,6 @@ gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void
     if (!err) return GQA_ERR_CUDA;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const RopeFreqs rf = rope_freqs(static_cast<double>(theta));
     if (append) {
         AppendParams ap;
         ap.k_new = static_cast<const uint16_t *>(k_new);
@@ -335,8 +443,9 @@ gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void
         ap.B = B;
         ap.Hkv = Hkv;
         ap.max_len = max_len;
+        ap.pairing = rs.pairing;
         ap.eps = eps;
-        ap.rf = rf;
+        ap.rf = rs.rf;
         const long long warps = static_cast<long long>(B) * Hkv;
         decode_append_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, st>>>(ap);
         if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
@@ -362,9 +471,10 @@ gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void
     p.maxC = static_cast<int>((static_cast<long long>(max_len) + kChunk - 1) / kChunk);
     p.max_len = max_len;
     p.len_add = append ? 1 : 0;
+    p.pairing = rs.pairing;
     p.eps = eps;
-    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim)));
-    p.rf = rf;
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim))) * rs.logit_mult;
+    p.rf = rs.rf;
 
     const int h = p.hpg;
     if (h == 1) return launch_decode<1>(p, 1, st);
@@ -380,8 +490,21 @@ extern "C" gqa_status gqa_attn_decode(const void *q, const void *k_cache, const 
                                       const float *qnorm_w, float theta, float eps, float *out, int B, int H,
                                       int Hkv, int D, int max_len, void *workspace, size_t workspace_bytes,
                                       void *stream) {
+    if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
     return decode_impl(q, nullptr, nullptr, const_cast<void *>(k_cache), const_cast<void *>(v_cache), cache_offsets,
-                       seqlens, q_pos, qnorm_w, nullptr, theta, eps, out, B, H, Hkv, D, max_len, workspace,
+                       seqlens, q_pos, qnorm_w, nullptr, plain_rope(theta), eps, out, B, H, Hkv, D, max_len,
+                       workspace, workspace_bytes, stream);
+}
+
+extern "C" gqa_status gqa_attn_decode_ex(const void *q, const void *k_cache, const void *v_cache,
+                                         const int64_t *cache_offsets, const int32_t *seqlens, const int32_t *q_pos,
+                                         const float *qnorm_w, const gqa_rope_config *rope, float eps, float *out,
+                                         int B, int H, int Hkv, int D, int max_len, void *workspace,
+                                         size_t workspace_bytes, void *stream) {
+    RopeSpec rs;
+    if (!rope_spec(rope, rs)) return GQA_ERR_INVALID_ARG;
+    return decode_impl(q, nullptr, nullptr, const_cast<void *>(k_cache), const_cast<void *>(v_cache), cache_offsets,
+                       seqlens, q_pos, qnorm_w, nullptr, rs, eps, out, B, H, Hkv, D, max_len, workspace,
                        workspace_bytes, stream);
 }
 
@@ -391,8 +514,22 @@ extern "C" gqa_status gqa_attn_decode_append(const void *q, const void *k_new, c
                                              float theta, float eps, float *out, int B, int H, int Hkv, int D,
                                              int max_len, void *workspace, size_t workspace_bytes, void *stream) {
     if (!k_new || !v_new || !knorm_w) return GQA_ERR_INVALID_ARG;
-    return decode_impl(q, k_new, v_new, k_cache, v_cache, cache_offsets, seqlens, q_pos, qnorm_w, knorm_w, theta,
-                       eps, out, B, H, Hkv, D, max_len, workspace, workspace_bytes, stream);
+    if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
+    return decode_impl(q, k_new, v_new, k_cache, v_cache, cache_offsets, seqlens, q_pos, qnorm_w, knorm_w,
+                       plain_rope(theta), eps, out, B, H, Hkv, D, max_len, workspace, workspace_bytes, stream);
+}
+
+extern "C" gqa_status gqa_attn_decode_append_ex(const void *q, const void *k_new, const void *v_new, void *k_cache,
+                                                void *v_cache, const int64_t *cache_offsets, const int32_t *seqlens,
+                                                const int32_t *q_pos, const float *qnorm_w, const float *knorm_w,
+                                                const gqa_rope_config *rope, float eps, float *out, int B, int H,
+                                                int Hkv, int D, int max_len, void *workspace, size_t workspace_bytes,
+                                                void *stream) {
+    if (!k_new || !v_new || !knorm_w) return GQA_ERR_INVALID_ARG;
+    RopeSpec rs;
+    if (!rope_spec(rope, rs)) return GQA_ERR_INVALID_ARG;
+    return decode_impl(q, k_new, v_new, k_cache, v_cache, cache_offsets, seqlens, q_pos, qnorm_w, knorm_w, rs, eps,
+                       out, B, H, Hkv, D, max_len, workspace, workspace_bytes, stream);
 }
 
 namespace {

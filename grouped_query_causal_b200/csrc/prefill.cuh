@@ -50,9 +50,13 @@ struct KPrologueParams {
 };
 
 // One warp per token at a time; each half-warp transforms one head vector, each lane
-// eight consecutive elements (four RoPE pairs).  cos/sin are evaluated once per token,
-// reused for all of its KV heads, and optionally stored so the query side (same
-// positions) can read them instead of evaluating them again.
+// eight consecutive elements.  Adjacent pairing: the lane's elements are four RoPE pairs.
+// Rotate-half pairing: lane j < 8 holds elements 8j .. 8j+7, whose partners 64 + 8j ..
+// sit in lane j + 8; both rotate by the frequencies 8j .. 8j+7.  Each lane evaluates the
+// cos/sin of four frequencies once per token (reused for all of the token's KV heads,
+// exchanged with the partner lane for rotate-half) and optionally stores them so the
+// query side (same positions) can read them instead of evaluating them again.
+template <int PAIRING>
 __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__ KPrologueParams p) {
     const int lane = threadIdx.x & 31;
     const int half = lane >> 4;
@@ -64,15 +68,43 @@ __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__
     const float4 wb = reinterpret_cast<const float4 *>(p.wk)[2 * sub + 1];
     const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 
+    constexpr bool half_pairs = PAIRING == kPairHalf;
+    // frequencies this lane evaluates: 4 sub .. 4 sub + 3 (adjacent), or 8 (sub & 7) +
+    // 4 (sub >> 3) + 0..3 (rotate-half: the partner lane evaluates the other four)
+    const int f0 = half_pairs ? 8 * (sub & 7) + 4 * (sub >> 3) : 4 * sub;
+
     for (; tok < p.ntok; tok += nwarps) {
         const int ps = p.pos[tok];
-        float cs[4], sn[4];
+        float cs[8], sn[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) rope_cos_sin(ps, p.rf.inv_freq[4 * sub + i], cs[i], sn[i]);
+        for (int i = 0; i < 4; ++i) rope_cos_sin(ps, p.rf.inv_freq[f0 + i], cs[i], sn[i]);
         if (p.rope_cs != nullptr && half == 0) {
             float4 *tab = reinterpret_cast<float4 *>(p.rope_cs);
-            tab[rope_table_index(tok, 2 * sub)] = make_float4(cs[0], sn[0], cs[1], sn[1]);
-            tab[rope_table_index(tok, 2 * sub + 1)] = make_float4(cs[2], sn[2], cs[3], sn[3]);
+            tab[rope_table_index(tok, f0 / 2)] = make_float4(cs[0], sn[0], cs[1], sn[1]);
+            tab[rope_table_index(tok, f0 / 2 + 1)] = make_float4(cs[2], sn[2], cs[3], sn[3]);
+        }
+        if constexpr (half_pairs) {   // cos/sin of frequencies 8 (sub & 7) + 0..7, in that order
+            float pc[4], ps4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                pc[i] = __shfl_xor_sync(0xffffffffu, cs[i], 8);
+                ps4[i] = __shfl_xor_sync(0xffffffffu, sn[i], 8);
+            }
+            if (sub >= 8) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    cs[4 + i] = cs[i];
+                    sn[4 + i] = sn[i];
+                    cs[i] = pc[i];
+                    sn[i] = ps4[i];
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    cs[4 + i] = pc[i];
+                    sn[4 + i] = ps4[i];
+                }
+            }
         }
         // up to 8 head pairs per batch: all loads first, so they are in flight together
         for (int h0 = 0; h0 < p.Hkv; h0 += 16) {
@@ -103,11 +135,24 @@ __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__
                 for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
                 const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + p.eps);
                 uint32_t outw[4];
+                if constexpr (!half_pairs) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float a = w[2 * i] * x[2 * i] * inv;
-                    const float b = w[2 * i + 1] * x[2 * i + 1] * inv;
-                    outw[i] = pack_bf16x2(a * cs[i] - b * sn[i], a * sn[i] + b * cs[i]);
+                    for (int i = 0; i < 4; ++i) {
+                        const float a = w[2 * i] * x[2 * i] * inv;
+                        const float b = w[2 * i + 1] * x[2 * i + 1] * inv;
+                        outw[i] = pack_bf16x2(a * cs[i] - b * sn[i], a * sn[i] + b * cs[i]);
+                    }
+                } else {
+                    const float sign = sub < 8 ? -1.0f : 1.0f;   // first half: a c - b s; second: a c + b s
+                    float y[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float a = w[e] * x[e] * inv;
+                        const float b = __shfl_xor_sync(0xffffffffu, a, 8);
+                        y[e] = fmaf(sign * b, sn[e], a * cs[e]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) outw[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
                 }
                 if (hh < p.Hkv)
                     *reinterpret_cast<uint4 *>(p.khat + (static_cast<size_t>(tok) * p.Hkv + hh) * kHeadDim + 8 * sub) =
@@ -153,7 +198,7 @@ struct AttnParams {
     unsigned *err;
     int B, T, H, Hkv, hpg, nqb, npairs;
     float eps;
-    float scale_log2;      // log2(e) / sqrt(D): softmax runs in base 2
+    float scale_log2;      // log2(e) / sqrt(D) times the RoPE variant's logit factor: softmax runs in base 2
     RopeFreqs rf;
 };
 
@@ -189,9 +234,11 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
 }
 
 // RMSNorm (w_q, eps) and RoPE of query row r (flattened token n) of a raw Q tile, in
-// place.  The rotation uses the K prologue's cos/sin table when given (coalesced across
-// the warp: consecutive rows are consecutive tokens), fetched in two batches of 16
-// loads, else evaluates cos/sin from the position ps.
+// place, with adjacent or rotate-half pairing.  The rotation uses the K prologue's
+// cos/sin table when given (coalesced across the warp: consecutive rows are consecutive
+// tokens), fetched in batches of 16 (adjacent) or 8 (rotate-half) loads, else evaluates
+// cos/sin from the position ps.
+template <int PAIRING>
 __device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, const float *table, long long n,
                                                 const float *wq, float eps, const RopeFreqs &rf) {
     float ss = 0.f;
@@ -207,6 +254,51 @@ __device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, cons
         }
     }
     const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + eps);
+    if constexpr (PAIRING == kPairHalf) {
+        // rotate-half: chunk c (elements 8c .. 8c+7, c < 8) meets chunk c + 8, at the
+        // frequencies 8c .. 8c+7; four batches of 16 frequencies (8 table entries)
+#pragma unroll 1
+        for (int qt = 0; qt < 4; ++qt) {
+            float4 tb[8];   // (cos, sin) of frequencies 16 qt .. 16 qt + 15, two per float4
+            if (table != nullptr) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    tb[i] = __ldg(reinterpret_cast<const float4 *>(table) + rope_table_index(n, 8 * qt + i));
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int f = 16 * qt + 2 * i;
+                    rope_cos_sin(ps, rf.inv_freq[f], tb[i].x, tb[i].y);
+                    rope_cos_sin(ps, rf.inv_freq[f + 1], tb[i].z, tb[i].w);
+                }
+            }
+#pragma unroll
+            for (int c8 = 0; c8 < 2; ++c8) {
+                const int c = 2 * qt + c8;
+                const uint32_t addr1 = tile_chunk_addr(sq, r, c), addr2 = tile_chunk_addr(sq, r, c + 8);
+                const uint4 v1 = ld_shared_v4(addr1), v2 = ld_shared_v4(addr2);
+                const uint32_t u1[4] = {v1.x, v1.y, v1.z, v1.w}, u2[4] = {v2.x, v2.y, v2.z, v2.w};
+                const float4 w1a = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c);
+                const float4 w1b = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c + 1);
+                const float4 w2a = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c + 16);
+                const float4 w2b = __ldg(reinterpret_cast<const float4 *>(wq) + 2 * c + 17);
+                const float w1[8] = {w1a.x, w1a.y, w1a.z, w1a.w, w1b.x, w1b.y, w1b.z, w1b.w};
+                const float w2[8] = {w2a.x, w2a.y, w2a.z, w2a.w, w2b.x, w2b.y, w2b.z, w2b.w};
+                uint32_t o1[4], o2[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 t = tb[4 * c8 + i];   // frequencies 8c + 2i, 8c + 2i + 1
+                    const float a0 = w1[2 * i] * bf16lo(u1[i]) * inv, a1 = w1[2 * i + 1] * bf16hi(u1[i]) * inv;
+                    const float b0 = w2[2 * i] * bf16lo(u2[i]) * inv, b1 = w2[2 * i + 1] * bf16hi(u2[i]) * inv;
+                    o1[i] = pack_bf16x2(a0 * t.x - b0 * t.y, a1 * t.z - b1 * t.w);
+                    o2[i] = pack_bf16x2(b0 * t.x + a0 * t.y, b1 * t.z + a1 * t.w);
+                }
+                st_shared_v4(addr1, make_uint4(o1[0], o1[1], o1[2], o1[3]));
+                st_shared_v4(addr2, make_uint4(o2[0], o2[1], o2[2], o2[3]));
+            }
+        }
+        return;
+    }
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         float4 tb[16];   // (cos, sin) of pairs 32*half .. 32*half+31, two pairs per float4
@@ -258,6 +350,7 @@ __device__ __forceinline__ void exp_pack64(const float *x, float scale, float ne
     }
 }
 
+template <int PAIRING>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
@@ -427,7 +520,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (ok) {
                 const long long tok = static_cast<long long>(b) * p.T + t;
                 const int ps = valid ? p.pos[tok] : 0;
-                transform_q_row(sQ0 + s * kTileBytes, r, ps, valid ? p.rope_cs : nullptr, tok, p.wq, p.eps, p.rf);
+                transform_q_row<PAIRING>(sQ0 + s * kTileBytes, r, ps, valid ? p.rope_cs : nullptr, tok, p.wq, p.eps,
+                                         p.rf);
                 fence_proxy_async_smem();
                 mbar_arrive(BAR(BAR_Q_READY + s));
             }

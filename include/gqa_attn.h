@@ -222,6 +222,90 @@ gqa_status gqa_attn_decode_noalloc(const void *q, const void *k_cache, const voi
                                    float eps, float *out, int B, int H, int Hkv, int D,
                                    int max_len, void *stream);
 
+/* ----------------------------------------------------------------- RoPE variants
+ *
+ * The entry points above rotate adjacent pairs (x[2i], x[2i+1]) by pos * theta_i with
+ * theta_i = theta^(-2i/D) ("Qwen3系列1" D2-2; "深入剖析Qwen3模型架构" 3.1.2, 3.4.1).
+ * The _ex forms below take a gqa_rope_config instead of theta, for the variants a
+ * long-context deployment uses:
+ *
+ *   pairing  GQA_ROPE_PAIR_ADJACENT: (x[2i], x[2i+1]), as above
+ *            GQA_ROPE_PAIR_HALF:     (x[i], x[i + D/2]) (the rotate-half layout)
+ *   scaling  GQA_ROPE_SCALE_NONE:    theta_i
+ *            GQA_ROPE_SCALE_LINEAR:  theta_i / factor, i.e. the position divided by the
+ *                                    extension factor ("Qwen3 技术报告深度解读" 4.2, linear
+ *                                    interpolation)
+ *            GQA_ROPE_SCALE_NTK:     (theta * factor^(D/(D-2)))^(-2i/D), the NTK-aware base
+ *                                    change (the page's 4.2 formula is garbled; this is the
+ *                                    published form)
+ *            GQA_ROPE_SCALE_YARN:    YaRN's "NTK-by-parts" (Peng et al. 2023; the page's
+ *                                    3.4.2 formula is garbled): with r_i = L theta_i / (2 pi),
+ *                                    L = original_max_position, and gamma_i =
+ *                                    clamp((r_i - beta_slow) / (beta_fast - beta_slow), 0, 1),
+ *                                    theta_i ((1 - gamma_i) / factor + gamma_i); the attention
+ *                                    logits are multiplied by (0.1 ln(factor) + 1)^2, YaRN's
+ *                                    temperature.  The stored k-hat is not scaled by it.
+ *
+ * factor must be finite and >= 1 for a scaled variant (1 gives the plain frequencies);
+ * YaRN also needs original_max_position >= 1 and finite beta_fast > beta_slow (the YaRN
+ * paper uses 32 and 1).  theta must be finite and > 0.  An invalid configuration or a
+ * NULL pointer is GQA_ERR_INVALID_ARG.  k-hat written and RoPE tables filled with one
+ * configuration must be read with the same one.
+ */
+typedef enum { GQA_ROPE_PAIR_ADJACENT = 0, GQA_ROPE_PAIR_HALF = 1 } gqa_rope_pairing;
+typedef enum {
+    GQA_ROPE_SCALE_NONE = 0,
+    GQA_ROPE_SCALE_LINEAR = 1,
+    GQA_ROPE_SCALE_NTK = 2,
+    GQA_ROPE_SCALE_YARN = 3
+} gqa_rope_scaling;
+
+typedef struct {
+    double theta;               /* frequency base */
+    int pairing;                /* gqa_rope_pairing */
+    int scaling;                /* gqa_rope_scaling */
+    double factor;              /* context extension factor s (scaled variants) */
+    int original_max_position;  /* YaRN: training context length L */
+    double beta_fast;           /* YaRN: ramp end (pairs with more wavelengths keep theta_i) */
+    double beta_slow;           /* YaRN: ramp start (pairs with fewer get theta_i / s) */
+} gqa_rope_config;
+
+/* gqa_attn_prefill with a RoPE variant (the same variant for q and k). */
+gqa_status gqa_attn_prefill_ex(const void *q, const void *k, const void *v, const int32_t *pos,
+                               const float *qnorm_w, const float *knorm_w,
+                               const gqa_rope_config *rope, float eps, float *out, int B, int T,
+                               int H, int Hkv, int D, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/* gqa_attn_k_norm_rope with a RoPE variant; the table it fills holds that variant's
+ * cos/sin. */
+gqa_status gqa_attn_k_norm_rope_ex(const void *k, const int32_t *pos, const float *knorm_w,
+                                   const gqa_rope_config *rope, float eps, void *k_hat,
+                                   float *rope_cs, int64_t N, int Hkv, int D, void *stream);
+
+/* gqa_attn_prefill_khat with a RoPE variant (the one k_hat and rope_cs were made with). */
+gqa_status gqa_attn_prefill_khat_ex(const void *q, const void *k_hat, const void *v,
+                                    const int32_t *pos, const float *rope_cs,
+                                    const float *qnorm_w, const gqa_rope_config *rope, float eps,
+                                    float *out, int B, int T, int H, int Hkv, int D, void *stream);
+
+/* gqa_attn_decode with a RoPE variant (the one the cached keys were rotated with). */
+gqa_status gqa_attn_decode_ex(const void *q, const void *k_cache, const void *v_cache,
+                              const int64_t *cache_offsets, const int32_t *seqlens,
+                              const int32_t *q_pos, const float *qnorm_w,
+                              const gqa_rope_config *rope, float eps, float *out, int B, int H,
+                              int Hkv, int D, int max_len, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+/* gqa_attn_decode_append with a RoPE variant (for the appended key and the query). */
+gqa_status gqa_attn_decode_append_ex(const void *q, const void *k_new, const void *v_new,
+                                     void *k_cache, void *v_cache, const int64_t *cache_offsets,
+                                     const int32_t *seqlens, const int32_t *q_pos,
+                                     const float *qnorm_w, const float *knorm_w,
+                                     const gqa_rope_config *rope, float eps, float *out, int B,
+                                     int H, int Hkv, int D, int max_len, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
 /*
  * Device status: waits for `stream` (a cudaStream_t as void*, NULL = legacy default
  * stream), then reads and clears the library's device error word on the current

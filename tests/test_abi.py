@@ -131,6 +131,34 @@ def test_decode_append_argument_errors_are_caught_on_the_host(lib):
     assert _decode_append(lib, B=0) == 0
 
 
+def _rope(**kw):
+    return binding.RopeConfig.make(**kw)
+
+
+def test_rope_config_errors_are_caught_on_the_host(lib):
+    def pre(rope):
+        return lib.gqa_attn_prefill_ex(16, 16, 16, 16, 16, 16, rope, 1e-6, 16, 1, 8, 4, 2, 128, 256, 1 << 20, None)
+    assert pre(None) == -1
+    bad = [_rope(theta=0.0), _rope(theta=float("inf")), _rope(scaling="linear", factor=0.5),
+           _rope(scaling="ntk", factor=float("nan")), _rope(scaling="yarn", factor=4.0, original_max_position=0),
+           _rope(scaling="yarn", factor=4.0, beta_fast=1.0, beta_slow=1.0)]
+    c = _rope()
+    c.pairing = 2
+    bad.append(c)
+    c = _rope()
+    c.scaling = 7
+    bad.append(c)
+    for r in bad:
+        assert pre(ctypes.byref(r)) == -1
+        assert lib.gqa_attn_decode_ex(16, 16, 16, 16, 16, None, 16, ctypes.byref(r), 1e-6, 16, 2, 8, 2, 128, 100, 256,
+                                      1 << 20, None) == -1
+    ok = _rope(pairing="half", scaling="yarn", factor=8.0)
+    assert lib.gqa_attn_prefill_ex(16, 16, 16, 16, 16, 16, ctypes.byref(ok), 1e-6, 16, 0, 8, 4, 2, 128, 256, 1 << 20,
+                                   None) == 0          # B = 0: valid configuration, nothing to do
+    assert lib.gqa_attn_k_norm_rope_ex(16, 16, 16, ctypes.byref(ok), 1e-6, 16, None, 0, 2, 128, None) == 0
+    assert lib.gqa_attn_k_norm_rope_ex(16, 16, 16, ctypes.byref(ok), -1.0, 16, None, 0, 2, 128, None) == -1
+
+
 def test_binding_fails_loudly_without_the_library(tmp_path):
     saved = binding._lib
     binding._lib = None
