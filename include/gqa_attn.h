@@ -233,8 +233,9 @@ gqa_status gqa_attn_decode_noalloc(const void *q, const void *k_cache, const voi
  *            GQA_ROPE_PAIR_HALF:     (x[i], x[i + D/2]) (the rotate-half layout)
  *   scaling  GQA_ROPE_SCALE_NONE:    theta_i
  *            GQA_ROPE_SCALE_LINEAR:  theta_i / factor, i.e. the position divided by the
- *                                    extension factor ("Qwen3 技术报告深度解读" 4.2, linear
- *                                    interpolation)
+ *                                    extension factor (linear interpolation, 4.2
+ *                                    "序列长度扩展的技术方案" of the zizhi168.cn summary of
+ *                                    the Qwen3 report)
  *            GQA_ROPE_SCALE_NTK:     (theta * factor^(D/(D-2)))^(-2i/D), the NTK-aware base
  *                                    change (the page's 4.2 formula is garbled; this is the
  *                                    published form)

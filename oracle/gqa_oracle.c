@@ -27,6 +27,8 @@
  *      (order: q/k RMSNorm, then rotary embedding, then attention).
  *  [D] "Qwen3学习日志" (2048ai.net), section 一 (GQA: H query heads in G groups
  *      of h = H/G sharing one K/V head; G = H is MHA, G = 1 is MQA).
+ *  [E] the zizhi168.cn summary of the Qwen3 report (no title), 4.2 "序列长度扩展的技术方案"
+ *      (linear position interpolation; an NTK-aware variant).
  *
  * Readings where the pages are silent or disagree (each also listed in the
  * design notes): adjacent-pair RoPE; weight multiplies the normalised vector
@@ -86,13 +88,13 @@ void oracle_rope(const double *x, double pos, double base, int D, double *out)
  *
  * Frequencies theta_i, i = 0 .. D/2-1, for a base b and an extension factor s >= 1:
  *   none    b^(-2i/D)                                   ([B] 3.4.1)
- *   linear  b^(-2i/D) / s: the position divided by s     (the linear interpolation of
- *           "Qwen3 技术报告深度解读" 4.2, i.e. Position Interpolation, Chen et al. 2023)
+ *   linear  b^(-2i/D) / s: the position divided by s (the linear interpolation of [E] 4.2,
+ *           i.e. Position Interpolation, Chen et al. 2023)
  *   ntk     (b * s^(D/(D-2)))^(-2i/D): the base raised so that the lowest frequency is
- *           divided by s and the highest is kept ("NTK-aware" scaling; the page's own
- *           formula in 4.2 is garbled, so the published form is used)
+ *           divided by s and the highest is kept ("NTK-aware" scaling; [E] 4.2 prints a
+ *           garbled formula, so the published form is used)
  *   yarn    "NTK-by-parts" of YaRN (Peng, Quesnelle, Fan, Shippole 2023, sec. 3.2-3.4;
- *           the page's 3.4.2 snippet is garbled): with wavelength lambda_i = 2 pi / theta_i
+ *           [B] 3.4.2 prints a garbled formula): with wavelength lambda_i = 2 pi / theta_i
  *           and r_i = L / lambda_i (L the training context length),
  *           gamma_i = clamp((r_i - beta_slow) / (beta_fast - beta_slow), 0, 1) and
  *           theta'_i = (1 - gamma_i) theta_i / s + gamma_i theta_i;
