@@ -18,6 +18,7 @@ fp64 CPU oracle on bounded samples of the same workloads on the host cores.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import math
@@ -259,6 +260,8 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- the decode step that appends the new token first (its own timed region)
     app = run_decode_append(gqa, dev, stream, world, K, args.warmup)
+    # ---- the batched decode on a paged copy of the same cache (its own timed region)
+    paged = run_decode_paged(gqa, dec, dq, kc, vc, sl, dwq, dev, stream, world, K, args.warmup)
 
     if rank != 0:
         return None
@@ -313,6 +316,9 @@ def run_ours(args, rank, world, local_rank):
         "decode_append": dict(app, roofline=dict(app["roofline"], peak=hbm,
                                                  frac=round(app["roofline"]["achieved"] / hbm, 4),
                                                  peak_source=f"hbm_gbs of {pk_kind}")),
+        "decode_paged": dict(paged, roofline=dict(paged["roofline"], peak=hbm,
+                                                  frac=round(paged["roofline"]["achieved"] / hbm, 4),
+                                                  peak_source=f"hbm_gbs of {pk_kind}")),
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
@@ -367,6 +373,71 @@ def run_decode_append(gqa, dev, stream, world, K, W):
             "bytes_per_call": nbytes, "gpu_launches": 3 * K,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s", "traffic": None,
                          "kernel": "decode_append_kernel + decode_split_kernel + decode_merge_kernel (one call)"}}
+
+
+def run_decode_paged(gqa, dec, dq, kc, vc, sl, dwq, dev, stream, world, K, W, page_size=64):
+    """gqa_attn_decode_paged on the batched decode workload, its cache copied on the
+    device into pages of page_size rows handed out in a seeded random order; CUDA events
+    around K calls after W warm-up calls."""
+    lib = gqa.load()
+    sh = stream.cuda_stream
+    B, H, D = dec.q.shape
+    Hkv = dec.k_cache.shape[1]
+    lens = dec.seqlens.tolist()
+    offs = dec.offsets.tolist()
+    need = [(n + page_size - 1) // page_size for n in lens]
+    num_pages = sum(need)
+    perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(30))
+    table = torch.full((B, max(need)), -1, dtype=torch.int32)
+    src = torch.full((num_pages * page_size,), -1, dtype=torch.int64)
+    start = 0
+    for b in range(B):
+        pids = perm[start:start + need[b]]
+        start += need[b]
+        table[b, :need[b]] = pids.to(torch.int32)
+        rows = torch.arange(lens[b], dtype=torch.int64)
+        src[pids.repeat_interleave(page_size)[:lens[b]] * page_size + rows % page_size] = offs[b] + rows
+    src = src.to(dev)
+    ok = (src >= 0).view(-1, 1, 1)
+    kp = torch.where(ok, kc[src.clamp(min=0)], 0).view(num_pages, page_size, Hkv, D)
+    vp = torch.where(ok, vc[src.clamp(min=0)], 0).view(num_pages, page_size, Hkv, D)
+    del src, ok
+    tab = table.to(dev)
+    out = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(gqa.decode_workspace_size(B, H, Hkv, dec.max_len, D), dtype=torch.uint8, device=dev)
+    rope = gqa.RopeConfig.make(theta=dec.theta)
+
+    def call():
+        st = lib.gqa_attn_decode_paged(dq.data_ptr(), kp.data_ptr(), vp.data_ptr(), tab.data_ptr(), num_pages,
+                                       page_size, tab.shape[1], sl.data_ptr(), None, dwq.data_ptr(),
+                                       ctypes.byref(rope), dec.eps, out.data_ptr(), B, H, Hkv, D, dec.max_len,
+                                       ws.data_ptr(), ws.numel(), sh)
+        if st != 0:
+            raise RuntimeError(f"gqa_attn_decode_paged failed with status {st}")
+
+    for _ in range(W):
+        call()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if gqa.device_status() != 0:
+        raise RuntimeError("device status error in the paged-decode timing")
+    sec = max_over_ranks([e0.elapsed_time(e1)], dev, world)[0] / 1e3
+    nbytes = decode_bytes(lens, H, Hkv, D)
+    gbs = nbytes * K / sec / 1e9
+    del kp, vp, tab, out, ws
+    return {"value": round(whole_job_rate(nbytes * K, world, sec) / 1e9, 1), "unit": "GB/s",
+            "ms": round(1e3 * sec / K, 4), "page_size": page_size, "num_pages": num_pages,
+            "workload": "the batched decode (64 seqs, cache len U[1024,32768], H32 Hkv8 D128) in shuffled pages",
+            "bytes_per_call": nbytes, "gpu_launches": 2 * K,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s", "traffic": None,
+                         "kernel": "decode_split_kernel (paged) + decode_merge_kernel (one call)"}}
 
 
 def run_e2e(gqa, pin, dec, dev, stream, rank, world, steps):

@@ -25,7 +25,8 @@ EXPORTS = ("gqa_status_string", "gqa_attn_prefill_workspace_size", "gqa_attn_pre
            "gqa_attn_k_norm_rope", "gqa_attn_prefill_khat", "gqa_attn_decode_workspace_size",
            "gqa_attn_decode", "gqa_attn_decode_append", "gqa_attn_decode_noalloc",
            "gqa_attn_device_status", "gqa_attn_prefill_ex", "gqa_attn_k_norm_rope_ex",
-           "gqa_attn_prefill_khat_ex", "gqa_attn_decode_ex", "gqa_attn_decode_append_ex")
+           "gqa_attn_prefill_khat_ex", "gqa_attn_decode_ex", "gqa_attn_decode_append_ex",
+           "gqa_attn_decode_paged", "gqa_attn_decode_append_paged")
 # Size of the library's built-in scratch used by gqa_attn_decode_noalloc.
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -100,8 +101,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_attn_prefill_khat_ex.argtypes = [P, P, P, P, P, P, R, F, P, I, I, I, I, I, P]
     lib.gqa_attn_decode_ex.argtypes = [P, P, P, P, P, P, P, R, F, P, I, I, I, I, I, P, Z, P]
     lib.gqa_attn_decode_append_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, R, F, P, I, I, I, I, I, P, Z, P]
+    lib.gqa_attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, P, P, R, F, P, I, I, I, I, I, P, Z, P]
+    lib.gqa_attn_decode_append_paged.argtypes = [P, P, P, P, P, P, I, I, I, P, P, P, P, R, F, P, I, I, I, I, I, P, Z,
+                                                 P]
     for n in ("gqa_attn_prefill_ex", "gqa_attn_k_norm_rope_ex", "gqa_attn_prefill_khat_ex", "gqa_attn_decode_ex",
-              "gqa_attn_decode_append_ex"):
+              "gqa_attn_decode_append_ex", "gqa_attn_decode_paged", "gqa_attn_decode_append_paged"):
         getattr(lib, n).restype = I
     _lib = lib
     return lib
@@ -317,6 +321,83 @@ def decode_append(q, k_new, v_new, k_cache, v_cache, cache_offsets, seqlens, qno
             _ptr(q_pos), _ptr(qnorm_w), _ptr(knorm_w), th, float(eps), _ptr(out), B, H, Hkv, D, int(max_len),
             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _raise(st, "gqa_attn_decode_append")
+    return out
+
+
+def _check_pages(k_pages, v_pages, page_table, B):
+    _check(k_pages, "k_pages", torch.bfloat16, 4)
+    _check(v_pages, "v_pages", torch.bfloat16, 4)
+    _check(page_table, "page_table", torch.int32, 2)
+    if v_pages.shape != k_pages.shape:
+        raise ValueError("k_pages and v_pages must have one shape [num_pages, page_size, Hkv, D]")
+    if page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, max_pages_per_seq]")
+    return k_pages.shape[0], k_pages.shape[1], k_pages.shape[2], page_table.shape[1]
+
+
+def decode_paged(q, k_pages, v_pages, page_table, seqlens, qnorm_w, max_len: int,
+                 q_pos: Optional[torch.Tensor] = None, rope: Optional[RopeConfig] = None, eps: float = 1e-6,
+                 out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Decode on a paged cache: k_pages / v_pages [num_pages, page_size, Hkv, D] bf16,
+    page_table [B, max_pages] int32 (row r of sequence b: row r % page_size of page
+    page_table[b, r // page_size]).  rope defaults to the plain RoPE of base 1e6."""
+    lib = load()
+    _check(q, "q", torch.bfloat16, 3)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    _check(qnorm_w, "qnorm_w", torch.float32, 1)
+    if q_pos is not None:
+        _check(q_pos, "q_pos", torch.int32, 1)
+    B, H, D = q.shape
+    num_pages, page_size, Hkv, _ = _check_pages(k_pages, v_pages, page_table, B)
+    rope = rope if rope is not None else RopeConfig.make()
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 3)
+    need = int(lib.gqa_attn_decode_workspace_size(B, H, Hkv, D, int(max_len)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib.gqa_attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), num_pages, page_size,
+                                   page_table.shape[1], _ptr(seqlens), _ptr(q_pos), _ptr(qnorm_w), ctypes.byref(rope),
+                                   float(eps), _ptr(out), B, H, Hkv, D, int(max_len), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _raise(st, "gqa_attn_decode_paged")
+    return out
+
+
+def decode_append_paged(q, k_new, v_new, k_pages, v_pages, page_table, seqlens, qnorm_w, knorm_w,
+                        max_len: int, q_pos: Optional[torch.Tensor] = None, rope: Optional[RopeConfig] = None,
+                        eps: float = 1e-6, out: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """decode_append on a paged cache: the new token's k-hat and v go to row seqlens[b]
+    (in its page), then the query attends to rows 0..seqlens[b]."""
+    lib = load()
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_new, "k_new", torch.bfloat16, 3)
+    _check(v_new, "v_new", torch.bfloat16, 3)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    _check(qnorm_w, "qnorm_w", torch.float32, 1)
+    _check(knorm_w, "knorm_w", torch.float32, 1)
+    if q_pos is not None:
+        _check(q_pos, "q_pos", torch.int32, 1)
+    B, H, D = q.shape
+    num_pages, page_size, Hkv, _ = _check_pages(k_pages, v_pages, page_table, B)
+    if k_new.shape != (B, Hkv, D) or v_new.shape != (B, Hkv, D):
+        raise ValueError("k_new and v_new must be [B, Hkv, D]")
+    rope = rope if rope is not None else RopeConfig.make()
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 3)
+    need = int(lib.gqa_attn_decode_workspace_size(B, H, Hkv, D, int(max_len)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib.gqa_attn_decode_append_paged(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pages), _ptr(v_pages),
+                                          _ptr(page_table), num_pages, page_size, page_table.shape[1], _ptr(seqlens),
+                                          _ptr(q_pos), _ptr(qnorm_w), _ptr(knorm_w), ctypes.byref(rope), float(eps),
+                                          _ptr(out), B, H, Hkv, D, int(max_len), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _raise(st, "gqa_attn_decode_append_paged")
     return out
 
 

@@ -47,6 +47,10 @@ struct DecodeParams {
     int B, H, Hkv, hpg, maxC, max_len;
     int len_add;              // rows attended beyond seqlens[b]: 1 after an append, else 0
     int pairing;              // kPairAdjacent or kPairHalf
+    // Paged cache (pages != nullptr): row r of sequence b is row r % page_size of page
+    // pages[b * max_pages + r / page_size]; kc / vc are [num_pages, page_size, Hkv, D].
+    const int32_t *pages;
+    int page_size, max_pages, num_pages;
     float eps;
     float scale_log2;         // log2(e) / sqrt(D), times the RoPE variant's logit factor
     RopeFreqs rf;
@@ -56,6 +60,11 @@ struct DecodeParams {
 // 1 <= len <= max_len and len fits its rows.
 __device__ __forceinline__ bool decode_seq_ok(const DecodeParams &p, int b, int &len, long long &off) {
     len = p.seqlens[b] + p.len_add;
+    if (p.pages != nullptr) {   // paged: the rows of a sequence are its table's pages
+        off = 0;
+        const long long cap = static_cast<long long>(p.max_pages) * p.page_size;
+        return len >= 1 && len <= p.max_len && static_cast<long long>(len) <= cap;
+    }
     off = p.offsets[b];
     const long long cap = p.offsets[b + 1] - off;
     return len >= 1 && len <= p.max_len && static_cast<long long>(len) <= cap && off >= 0;
@@ -107,7 +116,7 @@ __device__ __forceinline__ int decode_head_of_lane(int lane) {
     return h;
 }
 
-template <int HG>
+template <int HG, bool PAGED>
 __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int LG = HeadsLog2<HG>::value;
     __shared__ __align__(16) float sq[HG][kHeadDim];
@@ -129,6 +138,35 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     const int k1 = min(len, k0 + kChunk);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int32_t *ptab = PAGED ? p.pages + static_cast<size_t>(b) * p.max_pages : nullptr;
+    if constexpr (PAGED) {
+        // every page this chunk reads must exist; otherwise the chunk reads nothing and
+        // poisons its partial sums so that the merged output of the sequence is NaN
+        bool bad = false;
+        for (int pg = k0 / p.page_size + tid; pg <= (k1 - 1) / p.page_size; pg += 128) {
+            const int id = ptab[pg];
+            bad |= id < 0 || id >= p.num_pages;
+        }
+        if (__syncthreads_or(bad)) {
+            const size_t slot0 = (static_cast<size_t>(b) * p.maxC + c) * p.H + static_cast<size_t>(g) * p.hpg;
+            if (tid < HG && jbase + tid < p.hpg) {
+                p.part_ml[2 * (slot0 + jbase + tid)] = 0.f;
+                p.part_ml[2 * (slot0 + jbase + tid) + 1] = __int_as_float(0x7fc00000);
+            }
+            if (tid == 0) atomicOr(p.err, kErrInput);
+            return;
+        }
+    }
+    // Physical row of the 16-row batch that starts at logical row `base` (16-aligned: a
+    // batch never crosses a page, whose size is a multiple of 16).
+    auto batch_row = [&](int base) -> long long {
+        if constexpr (PAGED) {
+            const int pg = base / p.page_size;
+            return static_cast<long long>(ptab[pg]) * p.page_size + (base - pg * p.page_size);
+        } else {
+            return base;
+        }
+    };
 
     // ---- q prologue: RMSNorm + RoPE at the query position, scaled into base-2 logits
     {
@@ -178,21 +216,35 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     const int my_head = decode_head_of_lane<HG>(lane);
 
     // ---- K sweep: base-2 logits of the HG heads for each key of this warp
-    uint4 kn[kRowPairs];
+    // Loads of the 16-row batch that starts at logical row `base` (rows past kw1 read
+    // as zero).  Contiguous caches index rows directly; paged ones look the page up once
+    // per batch.
+    auto load_batch = [&](const uint16_t *rbase, int base, uint4 (&dst)[kRowPairs]) {
+        if constexpr (PAGED) {
+            if (base >= kw1) return;
+            const long long pr = batch_row(base);
 #pragma unroll
-    for (int u = 0; u < kRowPairs; ++u) {
-        const int row = kw0 + 2 * u + rsel;
-        kn[u] = row < kw1 ? ldg_stream_v4(kbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
-    }
+            for (int u = 0; u < kRowPairs; ++u) {
+                const int row = base + 2 * u + rsel;
+                dst[u] = row < kw1 ? ldg_stream_v4(rbase + static_cast<size_t>(pr + 2 * u + rsel) * row_stride)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < kRowPairs; ++u) {
+                const int row = base + 2 * u + rsel;
+                dst[u] = row < kw1 ? ldg_stream_v4(rbase + static_cast<size_t>(row) * row_stride)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    };
+    uint4 kn[kRowPairs];
+    load_batch(kbase, kw0, kn);
     for (int base = kw0; base < kw1; base += 2 * kRowPairs) {
         uint4 kv[kRowPairs];
 #pragma unroll
         for (int u = 0; u < kRowPairs; ++u) kv[u] = kn[u];
-#pragma unroll
-        for (int u = 0; u < kRowPairs; ++u) {
-            const int row = base + 2 * kRowPairs + 2 * u + rsel;
-            kn[u] = row < kw1 ? ldg_stream_v4(kbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
-        }
+        load_batch(kbase, base + 2 * kRowPairs, kn);
 #pragma unroll
         for (int u = 0; u < kRowPairs; ++u) {
             const uint32_t rw[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
@@ -213,11 +265,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
         }
     }
     uint4 vn[kRowPairs];
-#pragma unroll
-    for (int u = 0; u < kRowPairs; ++u) {
-        const int row = kw0 + 2 * u + rsel;
-        vn[u] = row < kw1 ? ldg_stream_v4(vbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
-    }
+    load_batch(vbase, kw0, vn);
     __syncwarp();
 
     // ---- per-warp softmax statistics; lane handles head lane % HG
@@ -246,11 +294,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
         uint4 vv[kRowPairs];
 #pragma unroll
         for (int u = 0; u < kRowPairs; ++u) vv[u] = vn[u];
-#pragma unroll
-        for (int u = 0; u < kRowPairs; ++u) {
-            const int row = base + 2 * kRowPairs + 2 * u + rsel;
-            vn[u] = row < kw1 ? ldg_stream_v4(vbase + static_cast<size_t>(row) * row_stride) : make_uint4(0u, 0u, 0u, 0u);
-        }
+        load_batch(vbase, base + 2 * kRowPairs, vn);
 #pragma unroll
         for (int u = 0; u < kRowPairs; ++u) {
             const int row = base + 2 * u + rsel;
@@ -353,13 +397,15 @@ struct AppendParams {
     unsigned *err;
     int B, Hkv, max_len;
     int pairing;              // kPairAdjacent or kPairHalf
+    const int32_t *pages;     // paged cache (as DecodeParams), or nullptr
+    int page_size, max_pages, num_pages;
     float eps;
     RopeFreqs rf;
 };
 
 // One warp per (sequence, KV head): RMSNorm + RoPE of the new key at the token's
-// position, rounded to bf16, written to row seqlens[b] of the sequence; the new value
-// is copied next to it.  Lane l holds elements 4l .. 4l+3.
+// position, rounded to bf16, written to row seqlens[b] of the sequence (in its page, for
+// a paged cache); the new value is copied next to it.  Lane l holds elements 4l .. 4l+3.
 // A sequence whose rows cannot take the new token is flagged and left untouched.
 __global__ void __launch_bounds__(128) decode_append_kernel(const __grid_constant__ AppendParams p) {
     const int lane = threadIdx.x & 31;
@@ -368,15 +414,29 @@ __global__ void __launch_bounds__(128) decode_append_kernel(const __grid_constan
     const int b = static_cast<int>(pair / p.Hkv);
     const int g = static_cast<int>(pair % p.Hkv);
     const int len = p.seqlens[b];
-    const long long off = p.offsets[b];
-    const long long cap = p.offsets[b + 1] - off;
-    if (!(len >= 0 && len + 1 <= p.max_len && static_cast<long long>(len) + 1 <= cap && off >= 0)) {
-        if (g == 0 && lane == 0) atomicOr(p.err, kErrInput);
-        return;
+    long long row;   // physical cache row that receives the new token
+    if (p.pages != nullptr) {
+        const long long cap = static_cast<long long>(p.max_pages) * p.page_size;
+        const int id = (len >= 0 && static_cast<long long>(len) < cap) ? p.pages[static_cast<size_t>(b) * p.max_pages +
+                                                                                  len / p.page_size]
+                                                                       : -1;
+        if (!(len >= 0 && len + 1 <= p.max_len && id >= 0 && id < p.num_pages)) {
+            if (g == 0 && lane == 0) atomicOr(p.err, kErrInput);
+            return;
+        }
+        row = static_cast<long long>(id) * p.page_size + len % p.page_size;
+    } else {
+        const long long off = p.offsets[b];
+        const long long cap = p.offsets[b + 1] - off;
+        if (!(len >= 0 && len + 1 <= p.max_len && static_cast<long long>(len) + 1 <= cap && off >= 0)) {
+            if (g == 0 && lane == 0) atomicOr(p.err, kErrInput);
+            return;
+        }
+        row = off + len;
     }
     const int ps = p.qpos ? p.qpos[b] : len;
     const size_t src = (static_cast<size_t>(b) * p.Hkv + g) * kHeadDim + 4 * lane;
-    const size_t dst = ((static_cast<size_t>(off) + len) * p.Hkv + g) * kHeadDim + 4 * lane;
+    const size_t dst = (static_cast<size_t>(row) * p.Hkv + g) * kHeadDim + 4 * lane;
     const uint2 raw = *reinterpret_cast<const uint2 *>(p.k_new + src);
     const uint2 vraw = *reinterpret_cast<const uint2 *>(p.v_new + src);
     const float x0 = bf16lo(raw.x), x1 = bf16hi(raw.x), x2 = bf16lo(raw.y), x3 = bf16hi(raw.y);

@@ -391,7 +391,10 @@ namespace {
 template <int HG>
 gqa_status launch_decode(const DecodeParams &p, int npass, cudaStream_t st) {
     const dim3 grid(static_cast<unsigned>(p.B * p.Hkv), static_cast<unsigned>(p.maxC), static_cast<unsigned>(npass));
-    decode_split_kernel<HG><<<grid, 128, 0, st>>>(p);
+    if (p.pages != nullptr)
+        decode_split_kernel<HG, true><<<grid, 128, 0, st>>>(p);
+    else
+        decode_split_kernel<HG, false><<<grid, 128, 0, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
     decode_merge_kernel<<<static_cast<unsigned>(p.B * p.H), 128, 0, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
@@ -404,8 +407,15 @@ namespace {
 // Shared body of the decode entry points.  With k_new != nullptr the new token is first
 // appended to the cache (decode_append_kernel) and the split kernel attends to one row
 // more than seqlens[b].
+// A paged cache: page table [B, max_pages] of page ids < num_pages, page_size rows a page.
+struct PagedCache {
+    const int32_t *pages;
+    int num_pages, page_size, max_pages;
+};
+
 gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
-                       const int64_t *cache_offsets, const int32_t *seqlens, const int32_t *q_pos,
+                       const int64_t *cache_offsets, const PagedCache *paged, const int32_t *seqlens,
+                       const int32_t *q_pos,
                        const float *qnorm_w, const float *knorm_w, const RopeSpec &rs, float eps, float *out, int B,
                        int H, int Hkv, int D, int max_len, void *workspace, size_t workspace_bytes, void *stream) {
     const bool append = k_new != nullptr || v_new != nullptr || knorm_w != nullptr;
@@ -417,9 +427,17 @@ gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void
     if ((static_cast<long long>(max_len) + kChunk - 1) / kChunk > 65535) return GQA_ERR_INVALID_ARG;
     if (static_cast<long long>(B) * Hkv > 0x7fffffffLL || static_cast<long long>(B) * H > 0x7fffffffLL)
         return GQA_ERR_INVALID_ARG;
-    if (!q || !k_cache || !v_cache || !cache_offsets || !seqlens || !qnorm_w || !out) return GQA_ERR_INVALID_ARG;
+    if (!q || !k_cache || !v_cache || !seqlens || !qnorm_w || !out) return GQA_ERR_INVALID_ARG;
+    if (paged) {
+        if (!paged->pages || !aligned(paged->pages, 4) || paged->num_pages < 1 || paged->max_pages < 1 ||
+            paged->page_size < 16 || paged->page_size % 16 != 0 ||
+            static_cast<long long>(B) * paged->max_pages > 0x7fffffffLL)
+            return GQA_ERR_INVALID_ARG;
+    } else if (!cache_offsets || !aligned(cache_offsets, 8)) {
+        return GQA_ERR_INVALID_ARG;
+    }
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(qnorm_w, 16) ||
-        !aligned(out, 4) || !aligned(cache_offsets, 8) || !aligned(seqlens, 4) || (q_pos && !aligned(q_pos, 4)))
+        !aligned(out, 4) || !aligned(seqlens, 4) || (q_pos && !aligned(q_pos, 4)))
         return GQA_ERR_INVALID_ARG;
     if (append && (!k_new || !v_new || !knorm_w || !aligned(k_new, 8) || !aligned(v_new, 8) || !aligned(knorm_w, 16)))
         return GQA_ERR_INVALID_ARG;
@@ -444,6 +462,10 @@ gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void
         ap.Hkv = Hkv;
         ap.max_len = max_len;
         ap.pairing = rs.pairing;
+        ap.pages = paged ? paged->pages : nullptr;
+        ap.page_size = paged ? paged->page_size : 0;
+        ap.max_pages = paged ? paged->max_pages : 0;
+        ap.num_pages = paged ? paged->num_pages : 0;
         ap.eps = eps;
         ap.rf = rs.rf;
         const long long warps = static_cast<long long>(B) * Hkv;
@@ -472,6 +494,10 @@ gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void
     p.max_len = max_len;
     p.len_add = append ? 1 : 0;
     p.pairing = rs.pairing;
+    p.pages = paged ? paged->pages : nullptr;
+    p.page_size = paged ? paged->page_size : 0;
+    p.max_pages = paged ? paged->max_pages : 0;
+    p.num_pages = paged ? paged->num_pages : 0;
     p.eps = eps;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim))) * rs.logit_mult;
     p.rf = rs.rf;
@@ -492,7 +518,7 @@ extern "C" gqa_status gqa_attn_decode(const void *q, const void *k_cache, const 
                                       void *stream) {
     if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
     return decode_impl(q, nullptr, nullptr, const_cast<void *>(k_cache), const_cast<void *>(v_cache), cache_offsets,
-                       seqlens, q_pos, qnorm_w, nullptr, plain_rope(theta), eps, out, B, H, Hkv, D, max_len,
+                       nullptr, seqlens, q_pos, qnorm_w, nullptr, plain_rope(theta), eps, out, B, H, Hkv, D, max_len,
                        workspace, workspace_bytes, stream);
 }
 
@@ -504,7 +530,7 @@ extern "C" gqa_status gqa_attn_decode_ex(const void *q, const void *k_cache, con
     RopeSpec rs;
     if (!rope_spec(rope, rs)) return GQA_ERR_INVALID_ARG;
     return decode_impl(q, nullptr, nullptr, const_cast<void *>(k_cache), const_cast<void *>(v_cache), cache_offsets,
-                       seqlens, q_pos, qnorm_w, nullptr, rs, eps, out, B, H, Hkv, D, max_len, workspace,
+                       nullptr, seqlens, q_pos, qnorm_w, nullptr, rs, eps, out, B, H, Hkv, D, max_len, workspace,
                        workspace_bytes, stream);
 }
 
@@ -515,7 +541,7 @@ extern "C" gqa_status gqa_attn_decode_append(const void *q, const void *k_new, c
                                              int max_len, void *workspace, size_t workspace_bytes, void *stream) {
     if (!k_new || !v_new || !knorm_w) return GQA_ERR_INVALID_ARG;
     if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
-    return decode_impl(q, k_new, v_new, k_cache, v_cache, cache_offsets, seqlens, q_pos, qnorm_w, knorm_w,
+    return decode_impl(q, k_new, v_new, k_cache, v_cache, cache_offsets, nullptr, seqlens, q_pos, qnorm_w, knorm_w,
                        plain_rope(theta), eps, out, B, H, Hkv, D, max_len, workspace, workspace_bytes, stream);
 }
 
@@ -528,8 +554,37 @@ extern "C" gqa_status gqa_attn_decode_append_ex(const void *q, const void *k_new
     if (!k_new || !v_new || !knorm_w) return GQA_ERR_INVALID_ARG;
     RopeSpec rs;
     if (!rope_spec(rope, rs)) return GQA_ERR_INVALID_ARG;
-    return decode_impl(q, k_new, v_new, k_cache, v_cache, cache_offsets, seqlens, q_pos, qnorm_w, knorm_w, rs, eps,
-                       out, B, H, Hkv, D, max_len, workspace, workspace_bytes, stream);
+    return decode_impl(q, k_new, v_new, k_cache, v_cache, cache_offsets, nullptr, seqlens, q_pos, qnorm_w, knorm_w, rs,
+                       eps, out, B, H, Hkv, D, max_len, workspace, workspace_bytes, stream);
+}
+
+extern "C" gqa_status gqa_attn_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                                            const int32_t *page_table, int num_pages, int page_size,
+                                            int max_pages_per_seq, const int32_t *seqlens, const int32_t *q_pos,
+                                            const float *qnorm_w, const gqa_rope_config *rope, float eps, float *out,
+                                            int B, int H, int Hkv, int D, int max_len, void *workspace,
+                                            size_t workspace_bytes, void *stream) {
+    RopeSpec rs;
+    if (!rope_spec(rope, rs)) return GQA_ERR_INVALID_ARG;
+    const PagedCache pc{page_table, num_pages, page_size, max_pages_per_seq};
+    return decode_impl(q, nullptr, nullptr, const_cast<void *>(k_pages), const_cast<void *>(v_pages), nullptr, &pc,
+                       seqlens, q_pos, qnorm_w, nullptr, rs, eps, out, B, H, Hkv, D, max_len, workspace,
+                       workspace_bytes, stream);
+}
+
+extern "C" gqa_status gqa_attn_decode_append_paged(const void *q, const void *k_new, const void *v_new, void *k_pages,
+                                                   void *v_pages, const int32_t *page_table, int num_pages,
+                                                   int page_size, int max_pages_per_seq, const int32_t *seqlens,
+                                                   const int32_t *q_pos, const float *qnorm_w, const float *knorm_w,
+                                                   const gqa_rope_config *rope, float eps, float *out, int B, int H,
+                                                   int Hkv, int D, int max_len, void *workspace,
+                                                   size_t workspace_bytes, void *stream) {
+    if (!k_new || !v_new || !knorm_w) return GQA_ERR_INVALID_ARG;
+    RopeSpec rs;
+    if (!rope_spec(rope, rs)) return GQA_ERR_INVALID_ARG;
+    const PagedCache pc{page_table, num_pages, page_size, max_pages_per_seq};
+    return decode_impl(q, k_new, v_new, k_pages, v_pages, nullptr, &pc, seqlens, q_pos, qnorm_w, knorm_w, rs, eps, out,
+                       B, H, Hkv, D, max_len, workspace, workspace_bytes, stream);
 }
 
 namespace {

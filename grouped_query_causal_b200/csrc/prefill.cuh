@@ -297,8 +297,7 @@ __device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, cons
                 st_shared_v4(addr2, make_uint4(o2[0], o2[1], o2[2], o2[3]));
             }
         }
-        return;
-    }
+    } else {
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         float4 tb[16];   // (cos, sin) of pairs 32*half .. 32*half+31, two pairs per float4
@@ -334,6 +333,7 @@ __device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, cons
             }
             st_shared_v4(addr, make_uint4(o[0], o[1], o[2], o[3]));
         }
+    }
     }
 }
 

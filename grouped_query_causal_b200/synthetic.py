@@ -151,6 +151,42 @@ def decode_append_inputs(B: int = 64, H: int = 32, Hkv: int = 8, D: int = HEAD_D
     return DecodeAppendInputs(q, k_new, v_new, k_cache, v_cache, offsets, seqlens.to(torch.int32), wq, wk)
 
 
+@dataclass
+class PagedCache:
+    k_pages: torch.Tensor     # bf16 [num_pages, page_size, Hkv, D]
+    v_pages: torch.Tensor     # bf16 [num_pages, page_size, Hkv, D]
+    page_table: torch.Tensor  # int32 [B, max_pages]; unused entries -1
+    page_size: int
+
+
+def page_cache(k_rows: torch.Tensor, v_rows: torch.Tensor, offsets, capacities, page_size: int, seed: int = 0,
+               spare_pages: int = 3) -> PagedCache:
+    """Scatter per-sequence rows (sequence b: rows offsets[b] .. + capacities[b]) into
+    pages of page_size rows, pages handed out in a seeded random order with a few unused
+    ones; the tail of a sequence's last page is zero."""
+    B = len(capacities)
+    Hkv, D = k_rows.shape[1], k_rows.shape[2]
+    need = [(int(c) + page_size - 1) // page_size for c in capacities]
+    max_pages = max(1, max(need))
+    num_pages = sum(need) + spare_pages
+    order = torch.randperm(num_pages, generator=_gen(seed + 20)).tolist()
+    kp = torch.zeros(num_pages, page_size, Hkv, D, dtype=k_rows.dtype)
+    vp = torch.zeros_like(kp)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    nxt = 0
+    for b in range(B):
+        o = int(offsets[b])
+        for j in range(need[b]):
+            pid = order[nxt]
+            nxt += 1
+            table[b, j] = pid
+            lo = j * page_size
+            n = min(page_size, int(capacities[b]) - lo)
+            kp[pid, :n] = k_rows[o + lo:o + lo + n]
+            vp[pid, :n] = v_rows[o + lo:o + lo + n]
+    return PagedCache(kp, vp, table, page_size)
+
+
 # The documented workloads, by name.
 WORKLOADS = {
     "prefill_correctness": dict(kind="prefill", B=1, T=128, H=16, Hkv=8),

@@ -307,6 +307,39 @@ gqa_status gqa_attn_decode_append_ex(const void *q, const void *k_new, const voi
                                      int H, int Hkv, int D, int max_len, void *workspace,
                                      size_t workspace_bytes, void *stream);
 
+/* ----------------------------------------------------------------- paged KV cache
+ *
+ * The decode cache may also live in fixed-size pages (the layout of paged-attention
+ * servers): k_pages and v_pages are bf16 [num_pages, page_size, Hkv, D], and row r of
+ * sequence b is row r % page_size of page page_table[b * max_pages_per_seq +
+ * r / page_size].  page_table is int32 [B, max_pages_per_seq] on the device; page_size
+ * is a multiple of 16 (>= 16).  A sequence may use at most max_pages_per_seq *
+ * page_size rows.  The calls otherwise behave as gqa_attn_decode_ex /
+ * gqa_attn_decode_append_ex (the append writes the new row into its page).  Page ids are
+ * checked on the device: a sequence with an id outside [0, num_pages) among the pages it
+ * reads gets NaN output, reads no page memory through that id, and sets
+ * GQA_ERR_DEVICE_INPUT.  The workspace is gqa_attn_decode_workspace_size(B, H, Hkv, D,
+ * max_len).  rope must not be NULL.  This layout is not on the pages; it follows the
+ * paged KV cache that serving engines use, so that a cache managed that way needs no
+ * copy into one contiguous block per sequence.
+ */
+gqa_status gqa_attn_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                                 const int32_t *page_table, int num_pages, int page_size,
+                                 int max_pages_per_seq, const int32_t *seqlens,
+                                 const int32_t *q_pos, const float *qnorm_w,
+                                 const gqa_rope_config *rope, float eps, float *out, int B, int H,
+                                 int Hkv, int D, int max_len, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
+gqa_status gqa_attn_decode_append_paged(const void *q, const void *k_new, const void *v_new,
+                                        void *k_pages, void *v_pages, const int32_t *page_table,
+                                        int num_pages, int page_size, int max_pages_per_seq,
+                                        const int32_t *seqlens, const int32_t *q_pos,
+                                        const float *qnorm_w, const float *knorm_w,
+                                        const gqa_rope_config *rope, float eps, float *out, int B,
+                                        int H, int Hkv, int D, int max_len, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
 /*
  * Device status: waits for `stream` (a cudaStream_t as void*, NULL = legacy default
  * stream), then reads and clears the library's device error word on the current

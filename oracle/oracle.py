@@ -312,3 +312,41 @@ def decode_append_ex(q_bits, k_new_bits, v_new_bits, k_cache_bits, v_cache_bits,
                                     _p(qpos_a), _p(_c(wq, np.float32)), _p(_c(wk, np.float32)), _p(f),
                                     rope.pair_code(), rope.logit_mult(), eps, B, H, Hkv, D, _p(out), _p(khat))
     return out, khat
+
+
+# ---- paged KV cache: the same attention on rows gathered through a page table --------
+def _gather_pages(pages_bits, table, page_size, nrows):
+    """Rows 0..nrows-1 of one sequence from [num_pages, page_size, Hkv, D] pages."""
+    idx = np.arange(nrows)
+    return pages_bits[table[idx // page_size], idx % page_size]
+
+
+def decode_paged_ex(q_bits, k_pages_bits, v_pages_bits, page_table, page_size, seqlens, qpos, wq,
+                    rope: Rope, eps: float) -> np.ndarray:
+    """Decode on a paged cache: row r of sequence b is row r % page_size of page
+    page_table[b, r // page_size]; the attention is decode_ex on the gathered rows."""
+    k_pages_bits = _c(k_pages_bits, np.uint16)
+    v_pages_bits = _c(v_pages_bits, np.uint16)
+    table = np.asarray(page_table)
+    sl = np.asarray(seqlens, np.int64)
+    kc = np.concatenate([_gather_pages(k_pages_bits, table[b], page_size, sl[b]) for b in range(len(sl))])
+    vc = np.concatenate([_gather_pages(v_pages_bits, table[b], page_size, sl[b]) for b in range(len(sl))])
+    offsets = np.concatenate([[0], np.cumsum(sl)]).astype(np.int64)
+    return decode_ex(q_bits, kc, vc, offsets, sl.astype(np.int32), qpos, wq, rope, eps)
+
+
+def decode_append_paged_ex(q_bits, k_new_bits, v_new_bits, k_pages_bits, v_pages_bits, page_table, page_size,
+                           seqlens, qpos, wq, wk, rope: Rope, eps: float):
+    """decode_append_ex on a paged cache (the cached rows gathered through the table)."""
+    k_pages_bits = _c(k_pages_bits, np.uint16)
+    v_pages_bits = _c(v_pages_bits, np.uint16)
+    table = np.asarray(page_table)
+    sl = np.asarray(seqlens, np.int64)
+    Hkv, D = k_pages_bits.shape[2], k_pages_bits.shape[3]
+    ks, vs = [], []
+    for b in range(len(sl)):   # the cached rows, then one free row for the appended token
+        ks += [_gather_pages(k_pages_bits, table[b], page_size, sl[b]), np.zeros((1, Hkv, D), np.uint16)]
+        vs += [_gather_pages(v_pages_bits, table[b], page_size, sl[b]), np.zeros((1, Hkv, D), np.uint16)]
+    offsets = np.concatenate([[0], np.cumsum(sl + 1)]).astype(np.int64)
+    return decode_append_ex(q_bits, k_new_bits, v_new_bits, np.concatenate(ks), np.concatenate(vs), offsets,
+                            sl.astype(np.int32), qpos, wq, wk, rope, eps)

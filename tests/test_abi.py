@@ -159,6 +159,29 @@ def test_rope_config_errors_are_caught_on_the_host(lib):
     assert lib.gqa_attn_k_norm_rope_ex(16, 16, 16, ctypes.byref(ok), -1.0, 16, None, 0, 2, 128, None) == -1
 
 
+def test_paged_decode_argument_errors_are_caught_on_the_host(lib):
+    r = ctypes.byref(_rope())
+
+    def dec(**kw):
+        a = dict(q=16, kp=16, vp=16, tab=16, npages=10, ps=16, maxp=4, sl=16, qpos=None, wq=16, rope=r, eps=1e-6,
+                 out=16, B=2, H=8, Hkv=2, D=128, max_len=64, ws=256, wsb=1 << 20)
+        a.update(kw)
+        return lib.gqa_attn_decode_paged(a["q"], a["kp"], a["vp"], a["tab"], a["npages"], a["ps"], a["maxp"], a["sl"],
+                                         a["qpos"], a["wq"], a["rope"], a["eps"], a["out"], a["B"], a["H"], a["Hkv"],
+                                         a["D"], a["max_len"], a["ws"], a["wsb"], None)
+    assert dec(ps=8) == -1          # page size must be a multiple of 16
+    assert dec(ps=24) == -1
+    assert dec(npages=0) == -1
+    assert dec(maxp=0) == -1
+    assert dec(tab=None) == -1
+    assert dec(tab=18) == -1        # int32 table must be 4-byte aligned
+    assert dec(rope=None) == -1
+    assert dec(D=64) == -2
+    assert dec(B=0) == 0
+    assert lib.gqa_attn_decode_append_paged(16, None, 16, 16, 16, 16, 10, 16, 4, 16, None, 16, 16, r, 1e-6, 16, 2, 8,
+                                            2, 128, 64, 256, 1 << 20, None) == -1
+
+
 def test_binding_fails_loudly_without_the_library(tmp_path):
     saved = binding._lib
     binding._lib = None

@@ -627,3 +627,37 @@ def test_yarn_pipeline_matches_numpy_fp64():
             p = np.exp(s - s.max())
             p /= p.sum()
             np.testing.assert_allclose(got[b, hq], p @ vc, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------------------
+# Paged KV cache: a storage layout, so the attention must not change
+# --------------------------------------------------------------------------------------
+
+def test_paged_decode_equals_contiguous_decode():
+    B, H, Hkv, D = 3, 4, 2, 16
+    seqlens = [5, 33, 16]
+    d = synthetic.decode_inputs(B, H, Hkv, D, seed=60, seqlens=seqlens)
+    ref = oracle.decode(_bits(d.q), _bits(d.k_cache), _bits(d.v_cache), d.offsets.numpy(), d.seqlens.numpy(), None,
+                        d.wq.numpy(), d.theta, d.eps)
+    for ps in (16, 32):
+        pc = synthetic.page_cache(d.k_cache, d.v_cache, d.offsets, seqlens, ps, seed=61)
+        # pages handed out in a shuffled order: the table is not the identity
+        assert not np.array_equal(pc.page_table.numpy()[0, :2], [0, 1])
+        got = oracle.decode_paged_ex(_bits(d.q), _bits(pc.k_pages), _bits(pc.v_pages), pc.page_table.numpy(), ps,
+                                     d.seqlens.numpy(), None, d.wq.numpy(), oracle.Rope(theta=d.theta), d.eps)
+        np.testing.assert_array_equal(got, ref)
+
+
+def test_paged_append_equals_contiguous_append():
+    B, H, Hkv, D = 3, 4, 2, 16
+    seqlens = [0, 15, 40]
+    a = synthetic.decode_append_inputs(B, H, Hkv, D, seed=62, seqlens=seqlens, spare=1)
+    ref, kref = oracle.decode_append(_bits(a.q), _bits(a.k_new), _bits(a.v_new), _bits(a.k_cache), _bits(a.v_cache),
+                                     a.offsets.numpy(), a.seqlens.numpy(), None, a.wq.numpy(), a.wk.numpy(), a.theta,
+                                     a.eps)
+    pc = synthetic.page_cache(a.k_cache, a.v_cache, a.offsets, [s + 1 for s in seqlens], 16, seed=63)
+    got, kh = oracle.decode_append_paged_ex(_bits(a.q), _bits(a.k_new), _bits(a.v_new), _bits(pc.k_pages),
+                                            _bits(pc.v_pages), pc.page_table.numpy(), 16, a.seqlens.numpy(), None,
+                                            a.wq.numpy(), a.wk.numpy(), oracle.Rope(theta=a.theta), a.eps)
+    np.testing.assert_array_equal(got, ref)
+    np.testing.assert_array_equal(kh, kref)
