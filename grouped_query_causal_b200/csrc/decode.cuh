@@ -157,12 +157,21 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
             return;
         }
     }
+    // Page ids of this warp's rows (at most 17 pages of >= 16 rows cover its 256 rows),
+    // one per lane, so a batch finds its page with a shuffle rather than a dependent load.
+    const int wpg0 = PAGED ? (k0 + warp * kWarpKeys) / p.page_size : 0;
+    int my_page = 0;
+    if constexpr (PAGED) {
+        const int last = (min(k1, k0 + (warp + 1) * kWarpKeys) - 1) / p.page_size;
+        if (wpg0 + lane <= last) my_page = ptab[wpg0 + lane];
+    }
     // Physical row of the 16-row batch that starts at logical row `base` (16-aligned: a
-    // batch never crosses a page, whose size is a multiple of 16).
+    // batch never crosses a page, whose size is a multiple of 16).  Warp-uniform.
     auto batch_row = [&](int base) -> long long {
         if constexpr (PAGED) {
             const int pg = base / p.page_size;
-            return static_cast<long long>(ptab[pg]) * p.page_size + (base - pg * p.page_size);
+            const int id = __shfl_sync(0xffffffffu, my_page, pg - wpg0);
+            return static_cast<long long>(id) * p.page_size + (base - pg * p.page_size);
         } else {
             return base;
         }

@@ -174,13 +174,14 @@ constexpr uint32_t kOffBar = kOffKV + kStages * kTileBytes;
 enum {
     BAR_Q_FULL = 0,    // [2] TMA -> softmax WG: raw Q tile landed
     BAR_Q_READY = 2,   // [2] softmax WG -> MMA: Q tile normed + rotated in place (128 arrivals)
-    BAR_KV_FULL = 4,   // [kStages] TMA -> MMA
+    BAR_KV_FULL = 4,   // [kStages] TMA -> MMA (only K_0, in slot 0, uses it)
     BAR_KV_EMPTY = 4 + kStages,      // [kStages] MMA (commit) -> TMA
     BAR_S_FULL = 4 + 2 * kStages,    // [2] MMA (commit) -> softmax WG: S of the next tile is in TMEM
     BAR_P_FULL = 6 + 2 * kStages,    // [2] softmax WG -> MMA: P written over S in TMEM, O rescaled (128 arrivals)
     BAR_O_FULL = 8 + 2 * kStages,    // [2] MMA (commit) -> softmax WG: last P V finished
     BAR_DRAIN = 10 + 2 * kStages,    // MMA drains its own work before TMEM is released
-    NUM_BARS = 11 + 2 * kStages
+    BAR_STEP_FULL = 11 + 2 * kStages,  // [3] TMA -> MMA: V_j and K_{j+1} landed (one wait per tile)
+    NUM_BARS = 14 + 2 * kStages
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + NUM_BARS * 8;
 constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align the base to 1024
@@ -394,6 +395,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(BAR(BAR_KV_FULL + i), 1);
             mbar_init(BAR(BAR_KV_EMPTY + i), 1);
         }
+        for (int i = 0; i < 3; ++i) {
+            mbar_init(BAR(BAR_STEP_FULL + i), 1);
+        }
         mbar_init(BAR(BAR_DRAIN), 1);
         fence_mbarrier_init();
     }
@@ -437,16 +441,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const CUtensorMap *m = (it & 1) ? &tm_v : &tm_k;
                 const uint32_t dst = sKV0 + buf * kTileBytes;
                 const int row0 = (it >> 1) * kBN;
-                mbar_arrive_expect_tx(BAR(BAR_KV_FULL + buf), kTileBytes);
-                tma_load_4d(dst, m, 0, g, row0, b, BAR(BAR_KV_FULL + buf));
-                tma_load_4d(dst + kBoxBytes, m, 64, g, row0, b, BAR(BAR_KV_FULL + buf));
+                // K_0 signals its slot; V_j and K_{j+1} both signal step barrier j % 3,
+                // armed once for both when V_j is issued
+                const int jstep = (it - 1) >> 1;
+                const uint32_t bar = it == 0 ? BAR(BAR_KV_FULL + 0) : BAR(BAR_STEP_FULL + jstep % 3);
+                if (it == 0)
+                    mbar_arrive_expect_tx(bar, kTileBytes);
+                else if (it & 1)
+                    mbar_arrive_expect_tx(bar, jstep + 1 < n_kv ? 2 * kTileBytes : kTileBytes);
+                tma_load_4d(dst, m, 0, g, row0, b, bar);
+                tma_load_4d(dst + kBoxBytes, m, 64, g, row0, b, bar);
                 issued = it + 1;
             }
             if (!ok) {
                 // Failure path: let every copy still in flight land before the CTA exits.
                 for (int s = 0; s < nslots; ++s) mbar_wait(BAR(BAR_Q_FULL + s), 0, p.err);
-                for (int it = max(0, issued - kStages); it < issued; ++it)
-                    mbar_wait(BAR(BAR_KV_FULL + it % kStages), (it / kStages) & 1, p.err);
+                if (issued > 0) mbar_wait(BAR(BAR_KV_FULL + 0), 0, p.err);
+                for (int j = max(0, (issued - kStages - 1) >> 1); 2 * j + 1 < issued; ++j)
+                    mbar_wait(BAR(BAR_STEP_FULL + j % 3), (j / 3) & 1, p.err);
             }
         }
         __syncwarp();
@@ -458,8 +470,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         //   (which overwrites P_j: tcgen05.mma operations of one thread run in issue
         //   order).  While head 0's softmax works on S_{j+1}, the tensor core runs head
         //   1's P V and Q K^T, and vice versa.
-        // The issuing thread is on the critical path, so its waits carry a short suspend
-        // hint: a default try_wait can wake up ~900 cycles after the phase completes.
+        // The issuing thread is on the critical path: its queue of MMAs is shallow, so
+        // every wait it makes idles the tensor core.  Its waits carry a short suspend hint
+        // (a default try_wait can wake up ~900 cycles after the phase completes), and V_j
+        // and K_{j+1} share one barrier so that each tile costs one wait for data.
 #define MMA_WAIT(b_, par_, e_) mbar_wait_hint((b_), (par_), 20u, (e_))
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16_f32(kBM, kBN, false);
@@ -478,16 +492,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int j = 0; j < n_kv && ok; ++j) {
                 const int iv = 2 * j + 1, ik = 2 * j + 2;   // ring items of V_j and K_{j+1}
                 const bool more = j + 1 < n_kv;
-                if (!MMA_WAIT(BAR(BAR_KV_FULL + iv % kStages), (iv / kStages) & 1, p.err)) { ok = false; break; }
+                if (!MMA_WAIT(BAR(BAR_STEP_FULL + j % 3), (j / 3) & 1, p.err)) { ok = false; break; }
                 for (int s = 0; s < nslots; ++s) {
                     if (!MMA_WAIT(BAR(BAR_P_FULL + s), j & 1, p.err)) { ok = false; break; }
                     tc_fence_after();
                     issue_pv(tmem + 256 + s * 128, tmem + s * 128, sKV0 + (iv % kStages) * kTileBytes, id_pv, j > 0);
                     if (more) {
-                        if (s == 0 && !MMA_WAIT(BAR(BAR_KV_FULL + ik % kStages), (ik / kStages) & 1, p.err)) {
-                            ok = false;
-                            break;
-                        }
                         issue_qk(tmem + s * 128, sQ0 + s * kTileBytes, sKV0 + (ik % kStages) * kTileBytes, id_qk);
                         umma_commit(BAR(BAR_S_FULL + s));
                     } else {
