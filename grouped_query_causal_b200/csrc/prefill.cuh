@@ -13,6 +13,8 @@
 //      runs in two warpgroups (one per head of the pair, ping-ponging with the tensor
 //      core) with one query row per thread; causal tiles above the diagonal are never
 //      loaded.
+//  Both kernels take the RoPE pairing (adjacent or rotate-half) as a template
+//  parameter; the frequencies (plain or scaled) arrive precomputed from the host.
 //
 // Sources, by page title and section: "Qwen3系列1-理论基础&真实结构" D1-2 (stable
 // softmax), D1-4 (softmax(QK^T/sqrt(d)+M)V), D1-5 (causal mask), D2-1 (RMSNorm), D2-2
