@@ -65,3 +65,11 @@ def test_whole_job_rate_counts_every_rank():
     # two replicas, each 4e12 FLOP in at most 2 s: 4 TFLOP/s for the job
     assert bench.whole_job_rate(4e12, 2, 2.0) == pytest.approx(4e12)
     assert bench.max_over_ranks([1.5, 2.5], torch.device("cpu"), 1) == [1.5, 2.5]
+
+
+def test_traffic_staleness_ignores_comments_only():
+    sys.path.insert(0, ROOT)
+    import bench
+    src = "int a = 1;  // one\n/* block\n comment */\nint b = 2;\n"
+    assert bench._code_only(src) == bench._code_only("int a = 1;\n// other words\nint b = 2;  /* x */\n")
+    assert bench._code_only(src) != bench._code_only("int a = 2;\nint b = 2;\n")
