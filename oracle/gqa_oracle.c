@@ -531,6 +531,94 @@ void oracle_decode_append(const uint16_t *q, const uint16_t *k_new, const uint16
     free(f);
 }
 
+/* Chunked prefill against a cache prefix ([A] D2-3: a sequence's earlier tokens already
+ * sit in the KV cache; [A] D1-5: the causal mask on the token index).  Sequence b holds
+ * P_b = prefix_len[b] cached rows (k-hat and v) from row offsets[b] on, and brings a
+ * chunk of C new tokens: raw q [B, C, H, D], k and v [B, C, Hkv, D] (bf16 bits), at
+ * positions pos [B, C].  Chunk row i of query head hq attends to the P_b cached rows of
+ * KV head hq / (H/Hkv) and to the chunk's rows 0 .. i (token indices up to P_b + i).
+ * The chunk's k-hat goes to khat_out [B, C, Hkv, D] (what a caller appends to the
+ * cache); out is [B, C, H, D]. */
+void oracle_prefill_chunk_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                             const uint16_t *k_cache, const uint16_t *v_cache,
+                             const int64_t *offsets, const int32_t *prefix_len, const int32_t *pos,
+                             const float *wq, const float *wk, const double *inv_freq, int pairing,
+                             double logit_mult, double eps, int B, int C, int H, int Hkv, int D,
+                             double *out, double *khat_out)
+{
+    int h_per_kv = H / Hkv;
+    double inv_sqrt_d = logit_mult / sqrt((double)D);
+    int32_t maxkeys = 1;
+    for (int b = 0; b < B; ++b)
+        if (prefix_len[b] + C > maxkeys)
+            maxkeys = prefix_len[b] + C;
+    double *wqd = (double *)malloc(sizeof(double) * D);
+    double *wkd = (double *)malloc(sizeof(double) * D);
+    for (int d = 0; d < D; ++d) {
+        wqd[d] = (double)wq[d];
+        wkd[d] = (double)wk[d];
+    }
+    /* k-hat of the chunk's keys */
+    {
+        double *tmp = (double *)malloc(sizeof(double) * D);
+        for (int64_t n = 0; n < (int64_t)B * C; ++n)
+            for (int g = 0; g < Hkv; ++g)
+                norm_then_rope(k + (n * Hkv + g) * D, wkd, pos[n], inv_freq, pairing, eps, D, tmp,
+                               khat_out + (n * Hkv + g) * D);
+        free(tmp);
+    }
+#pragma omp parallel
+    {
+        double *tmp = (double *)malloc(sizeof(double) * D);
+        double *qi = (double *)malloc(sizeof(double) * D);
+        double *s = (double *)malloc(sizeof(double) * maxkeys);
+        double *p = (double *)malloc(sizeof(double) * maxkeys);
+        double *vbuf = (double *)malloc(sizeof(double) * (size_t)maxkeys * D);
+        const double **vr = (const double **)malloc(sizeof(double *) * maxkeys);
+#pragma omp for collapse(3) schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b)
+            for (int hq = 0; hq < H; ++hq)
+                for (int i = 0; i < C; ++i) {
+                    int g = hq / h_per_kv;
+                    int32_t P = prefix_len[b];
+                    int64_t n = (int64_t)b * C + i;
+                    norm_then_rope(q + (n * H + hq) * D, wqd, pos[n], inv_freq, pairing, eps, D, tmp, qi);
+                    int nkeys = P + i + 1;
+                    for (int j = 0; j < nkeys; ++j) {
+                        double dot = 0.0;
+                        if (j < P) {
+                            int64_t row = offsets[b] + j;
+                            const uint16_t *kj = k_cache + (row * Hkv + g) * D;
+                            const uint16_t *vj = v_cache + (row * Hkv + g) * D;
+                            for (int d = 0; d < D; ++d) {
+                                dot += qi[d] * bf16_bits_to_double(kj[d]);
+                                vbuf[(int64_t)j * D + d] = bf16_bits_to_double(vj[d]);
+                            }
+                        } else {
+                            int64_t m = (int64_t)b * C + (j - P);
+                            const double *kj = khat_out + (m * Hkv + g) * D;
+                            const uint16_t *vj = v + (m * Hkv + g) * D;
+                            for (int d = 0; d < D; ++d) {
+                                dot += qi[d] * kj[d];
+                                vbuf[(int64_t)j * D + d] = bf16_bits_to_double(vj[d]);
+                            }
+                        }
+                        s[j] = dot * inv_sqrt_d;
+                        vr[j] = vbuf + (int64_t)j * D;
+                    }
+                    softmax_weighted_sum(s, nkeys, vr, D, p, out + (n * H + hq) * D);
+                }
+        free(tmp);
+        free(qi);
+        free(s);
+        free(p);
+        free(vbuf);
+        free(vr);
+    }
+    free(wqd);
+    free(wkd);
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

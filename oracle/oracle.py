@@ -65,6 +65,8 @@ def _load():
             lib.oracle_decode_ex.argtypes = [P, P, P, P, P, P, P, P, I, Dd, Dd, I, I, I, I, P]
             lib.oracle_decode_append_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, Dd, Dd, I, I,
                                                     I, I, P, P]
+            lib.oracle_prefill_chunk_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, Dd, Dd, I, I, I,
+                                                    I, I, P, P]
             lib.oracle_num_threads.restype = I
             _lib = lib
     return _lib
@@ -350,3 +352,28 @@ def decode_append_paged_ex(q_bits, k_new_bits, v_new_bits, k_pages_bits, v_pages
     offsets = np.concatenate([[0], np.cumsum(sl + 1)]).astype(np.int64)
     return decode_append_ex(q_bits, k_new_bits, v_new_bits, np.concatenate(ks), np.concatenate(vs), offsets,
                             sl.astype(np.int32), qpos, wq, wk, rope, eps)
+
+
+def prefill_chunk_ex(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, offsets, prefix_len, pos, wq, wk,
+                     rope: Rope, eps: float):
+    """Chunked prefill against a cache prefix: q [B,C,H,D], k/v [B,C,Hkv,D] raw bf16 bits of
+    the chunk at positions pos [B,C]; the cache [rows,Hkv,D] holds prefix_len[b] rows of
+    sequence b from offsets[b] on (k-hat, v).  Returns (out [B,C,H,D], chunk k-hat
+    [B,C,Hkv,D]), both fp64."""
+    q_bits = _c(q_bits, np.uint16)
+    k_bits = _c(k_bits, np.uint16)
+    v_bits = _c(v_bits, np.uint16)
+    B, C, H, D = q_bits.shape
+    Hkv = k_bits.shape[2]
+    assert k_bits.shape == (B, C, Hkv, D) and v_bits.shape == k_bits.shape
+    pl = _c(prefix_len, np.int32)
+    assert (pl >= 0).all()
+    f = rope.inv_freq(D)
+    out = np.empty((B, C, H, D), np.float64)
+    khat = np.empty((B, C, Hkv, D), np.float64)
+    _load().oracle_prefill_chunk_ex(_p(q_bits), _p(k_bits), _p(v_bits), _p(_c(k_cache_bits, np.uint16)),
+                                    _p(_c(v_cache_bits, np.uint16)), _p(_c(offsets, np.int64)), _p(pl),
+                                    _p(_c(pos, np.int32).reshape(B, C)), _p(_c(wq, np.float32)),
+                                    _p(_c(wk, np.float32)), _p(f), rope.pair_code(), rope.logit_mult(), eps, B, C,
+                                    H, Hkv, D, _p(out), _p(khat))
+    return out, khat

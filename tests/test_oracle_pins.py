@@ -661,3 +661,65 @@ def test_paged_append_equals_contiguous_append():
                                             a.wq.numpy(), a.wk.numpy(), oracle.Rope(theta=a.theta), a.eps)
     np.testing.assert_array_equal(got, ref)
     np.testing.assert_array_equal(kh, kref)
+
+
+# --------------------------------------------------------------------------------------
+# Chunked prefill against a cache prefix
+# --------------------------------------------------------------------------------------
+
+def _chunk_setup(B, P, C, H, Hkv, D, seed):
+    """Prefill inputs for P + C tokens; the cache holds the bf16 k-hat / v of the first P."""
+    inp = synthetic.prefill_inputs(B, P + C, H, Hkv, D=D, seed=seed)
+    ntok = B * (P + C)
+    pos = inp.pos.numpy().reshape(ntok)
+    kh = oracle.qk_transform(_bits(inp.k).reshape(ntok, Hkv, D), pos, inp.wk.numpy(), inp.theta, inp.eps)
+    kh = kh.reshape(B, P + C, Hkv, D)
+    kc = torch.from_numpy(kh[:, :P].copy()).to(torch.bfloat16).reshape(B * P, Hkv, D)
+    vc = inp.v[:, :P].reshape(B * P, Hkv, D)
+    offsets = np.arange(B + 1, dtype=np.int64) * P
+    return inp, kh, kc, vc, offsets
+
+
+def test_chunk_after_a_prefix_equals_the_tail_of_prefill():
+    """The last C rows of causal attention over P + C tokens, with the prefix keys as the
+    cache stores them (bf16 k-hat), are the chunked prefill of those C tokens."""
+    B, P, C, H, Hkv, D = 2, 13, 7, 4, 2, 16
+    inp, kh, kc, vc, offsets = _chunk_setup(B, P, C, H, Hkv, D, seed=80)
+    ntok = B * (P + C)
+    qh = oracle.qk_transform(_bits(inp.q).reshape(ntok, H, D), inp.pos.numpy().reshape(ntok), inp.wq.numpy(),
+                             inp.theta, inp.eps).reshape(B, P + C, H, D)
+    k_ref = np.concatenate([kc.double().numpy().reshape(B, P, Hkv, D), kh[:, P:]], axis=1)
+    ref = oracle.sdpa_gqa(qh, k_ref, inp.v.double().numpy())[:, P:]
+    got, khat = oracle.prefill_chunk_ex(_bits(inp.q)[:, P:], _bits(inp.k)[:, P:], _bits(inp.v)[:, P:], _bits(kc),
+                                        _bits(vc), offsets, np.full(B, P, np.int32), inp.pos.numpy()[:, P:],
+                                        inp.wq.numpy(), inp.wk.numpy(), oracle.Rope(theta=inp.theta), inp.eps)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(khat, kh[:, P:])
+
+
+def test_chunk_without_prefix_is_plain_prefill():
+    B, C, H, Hkv, D = 2, 9, 4, 2, 16
+    inp = synthetic.prefill_inputs(B, C, H, Hkv, D=D, seed=81)
+    empty = np.zeros((0, Hkv, D), np.uint16)
+    got, _ = oracle.prefill_chunk_ex(_bits(inp.q), _bits(inp.k), _bits(inp.v), empty, empty,
+                                     np.zeros(B + 1, np.int64), np.zeros(B, np.int32), inp.pos.numpy(), inp.wq.numpy(),
+                                     inp.wk.numpy(), oracle.Rope(theta=inp.theta), inp.eps)
+    ref = oracle.prefill(_bits(inp.q), _bits(inp.k), _bits(inp.v), inp.pos.numpy(), inp.wq.numpy(), inp.wk.numpy(),
+                         inp.theta, inp.eps)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_chunk_of_one_token_is_the_append_step():
+    B, H, Hkv, D = 3, 4, 2, 16
+    seqlens = [0, 6, 11]
+    a = synthetic.decode_append_inputs(B, H, Hkv, D, seed=82, seqlens=seqlens, spare=1)
+    rope = oracle.Rope(theta=a.theta, scaling="yarn", factor=4.0, original_max_position=8)
+    qpos = np.array([3, 40, 7], np.int32)
+    ref, kref = oracle.decode_append_ex(_bits(a.q), _bits(a.k_new), _bits(a.v_new), _bits(a.k_cache),
+                                        _bits(a.v_cache), a.offsets.numpy(), a.seqlens.numpy(), qpos, a.wq.numpy(),
+                                        a.wk.numpy(), rope, a.eps)
+    got, khat = oracle.prefill_chunk_ex(_bits(a.q)[:, None], _bits(a.k_new)[:, None], _bits(a.v_new)[:, None],
+                                        _bits(a.k_cache), _bits(a.v_cache), a.offsets.numpy(), a.seqlens.numpy(),
+                                        qpos[:, None], a.wq.numpy(), a.wk.numpy(), rope, a.eps)
+    np.testing.assert_array_equal(got[:, 0], ref)
+    np.testing.assert_array_equal(khat[:, 0], kref)
