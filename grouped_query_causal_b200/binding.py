@@ -26,7 +26,7 @@ EXPORTS = ("gqa_status_string", "gqa_attn_prefill_workspace_size", "gqa_attn_pre
            "gqa_attn_decode", "gqa_attn_decode_append", "gqa_attn_decode_noalloc",
            "gqa_attn_device_status", "gqa_attn_prefill_ex", "gqa_attn_k_norm_rope_ex",
            "gqa_attn_prefill_khat_ex", "gqa_attn_decode_ex", "gqa_attn_decode_append_ex",
-           "gqa_attn_decode_paged", "gqa_attn_decode_append_paged", "gqa_attn_prefill_chunk")
+           "gqa_attn_decode_paged", "gqa_attn_decode_append_paged")
 # Size of the library's built-in scratch used by gqa_attn_decode_noalloc.
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -102,12 +102,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_attn_decode_ex.argtypes = [P, P, P, P, P, P, P, R, F, P, I, I, I, I, I, P, Z, P]
     lib.gqa_attn_decode_append_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, R, F, P, I, I, I, I, I, P, Z, P]
     lib.gqa_attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, P, P, R, F, P, I, I, I, I, I, P, Z, P]
-    lib.gqa_attn_prefill_chunk.argtypes = [P, P, P, P, P, P, R, F, P, I, I, I, I, I, I, P]
     lib.gqa_attn_decode_append_paged.argtypes = [P, P, P, P, P, P, I, I, I, P, P, P, P, R, F, P, I, I, I, I, I, P, Z,
                                                  P]
     for n in ("gqa_attn_prefill_ex", "gqa_attn_k_norm_rope_ex", "gqa_attn_prefill_khat_ex", "gqa_attn_decode_ex",
-              "gqa_attn_decode_append_ex", "gqa_attn_decode_paged", "gqa_attn_decode_append_paged",
-              "gqa_attn_prefill_chunk"):
+              "gqa_attn_decode_append_ex", "gqa_attn_decode_paged", "gqa_attn_decode_append_paged"):
         getattr(lib, n).restype = I
     _lib = lib
     return lib
@@ -244,34 +242,6 @@ def prefill_khat(q, k_hat, v, pos, qnorm_w, theta: float = 1.0e6, eps: float = 1
     st = fn(_ptr(q), _ptr(k_hat), _ptr(v), _ptr(pos), _ptr(rope_cs), _ptr(qnorm_w), th, float(eps), _ptr(out), B,
             T, H, Hkv, D, _stream_handle(stream))
     _raise(st, "gqa_attn_prefill_khat")
-    return out
-
-
-def prefill_chunk(q, k_hat, v, pos, qnorm_w, eps: float = 1e-6, rope: Optional[RopeConfig] = None,
-                  out: Optional[torch.Tensor] = None, rope_cs: Optional[torch.Tensor] = None,
-                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """Chunked prefill after a cached prefix: q [B,C,H,D] raw queries of the chunk;
-    k_hat / v [B,P+C,Hkv,D] (prefix rows, then the chunk's); pos [B,C].  Chunk row i sees
-    keys 0..P+i.  rope defaults to the plain RoPE of base 1e6."""
-    lib = load()
-    _check(q, "q", torch.bfloat16, 4)
-    _check(k_hat, "k_hat", torch.bfloat16, 4)
-    _check(v, "v", torch.bfloat16, 4)
-    _check(pos, "pos", torch.int32, 2)
-    _check(qnorm_w, "qnorm_w", torch.float32, 1)
-    B, C, H, D = q.shape
-    Tk, Hkv = k_hat.shape[1], k_hat.shape[2]
-    P = Tk - C
-    if P < 0 or k_hat.shape != (B, Tk, Hkv, D) or v.shape != k_hat.shape or pos.shape != (B, C):
-        raise ValueError("shape mismatch between q, k_hat, v, pos")
-    rope = rope if rope is not None else RopeConfig.make()
-    if out is None:
-        out = torch.empty((B, C, H, D), dtype=torch.float32, device=q.device)
-    _check(out, "out", torch.float32, 4)
-    st = lib.gqa_attn_prefill_chunk(_ptr(q), _ptr(k_hat), _ptr(v), _ptr(pos), _ptr(rope_cs), _ptr(qnorm_w),
-                                    ctypes.byref(rope), float(eps), _ptr(out), B, C, P, H, Hkv, D,
-                                    _stream_handle(stream))
-    _raise(st, "gqa_attn_prefill_chunk")
     return out
 
 

@@ -232,17 +232,15 @@ gqa_status launch_k_norm_rope(const void *k, const int32_t *pos, const float *kn
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
-// Enqueue the attention kernel (arguments already validated).  The T queries of each
-// sequence are tokens P .. P+T-1 and see keys 0 .. P+T-1 (P = 0: plain prefill).
+// Enqueue the attention kernel (arguments already validated).
 gqa_status launch_attention(const void *q, const void *k_hat, const void *v, const int32_t *pos,
                             const float *rope_cs, const float *qnorm_w, const RopeSpec &rs, float eps, float *out,
-                            int B, int T, int H, int Hkv, cudaStream_t st, int P = 0) {
+                            int B, int T, int H, int Hkv, cudaStream_t st) {
     unsigned *err = device_error_word();
     if (!err) return GQA_ERR_CUDA;
-    const int Tk = P + T;
     CUtensorMap tm_q, tm_k, tm_v;
-    if (!make_bf16_map(&tm_q, q, kHeadDim, H, T, B) || !make_bf16_map(&tm_k, k_hat, kHeadDim, Hkv, Tk, B) ||
-        !make_bf16_map(&tm_v, v, kHeadDim, Hkv, Tk, B))
+    if (!make_bf16_map(&tm_q, q, kHeadDim, H, T, B) || !make_bf16_map(&tm_k, k_hat, kHeadDim, Hkv, T, B) ||
+        !make_bf16_map(&tm_v, v, kHeadDim, Hkv, T, B))
         return GQA_ERR_CUDA;
     if (!attn_smem_attr_set()) return GQA_ERR_CUDA;
     AttnParams ap;
@@ -258,8 +256,6 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
     ap.hpg = H / Hkv;
     ap.nqb = (T + kBM - 1) / kBM;
     ap.npairs = (ap.hpg + 1) / 2;
-    ap.Tk = Tk;
-    ap.q_off = P;
     ap.eps = eps;
     ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim))) * rs.logit_mult;
     ap.rf = rs.rf;
@@ -364,25 +360,6 @@ extern "C" gqa_status gqa_attn_prefill_khat_ex(const void *q, const void *k_hat,
     RopeSpec rs;
     if (!rope_spec(rope, rs) || !eps_ok(eps)) return GQA_ERR_INVALID_ARG;
     return prefill_khat_impl(q, k_hat, v, pos, rope_cs, qnorm_w, rs, eps, out, B, T, H, Hkv, D, stream);
-}
-
-extern "C" gqa_status gqa_attn_prefill_chunk(const void *q, const void *k_hat, const void *v, const int32_t *pos,
-                                             const float *rope_cs, const float *qnorm_w, const gqa_rope_config *rope,
-                                             float eps, float *out, int B, int C, int P, int H, int Hkv, int D,
-                                             void *stream) {
-    RopeSpec rs;
-    if (!rope_spec(rope, rs) || !eps_ok(eps)) return GQA_ERR_INVALID_ARG;
-    if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
-    if (P < 0 || !prefill_shape_ok(B, C, H, Hkv) || static_cast<long long>(P) + C > 0x7fffffffLL ||
-        !prefill_shape_ok(B, P + C, H, Hkv))
-        return GQA_ERR_INVALID_ARG;
-    if (B == 0 || C == 0) return GQA_OK;
-    if (!q || !k_hat || !v || !pos || !qnorm_w || !out) return GQA_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(k_hat, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(qnorm_w, 16) ||
-        !aligned(pos, 4) || (rope_cs && !aligned(rope_cs, 16)))
-        return GQA_ERR_INVALID_ARG;
-    return launch_attention(q, k_hat, v, pos, rope_cs, qnorm_w, rs, eps, out, B, C, H, Hkv,
-                            static_cast<cudaStream_t>(stream), P);
 }
 
 extern "C" gqa_status gqa_attn_prefill(const void *q, const void *k, const void *v, const int32_t *pos,

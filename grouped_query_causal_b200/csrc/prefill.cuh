@@ -200,8 +200,6 @@ struct AttnParams {
     float *out;            // fp32 [B, T, H, D]
     unsigned *err;
     int B, T, H, Hkv, hpg, nqb, npairs;
-    int Tk;                // keys per sequence (T, or P + T for a chunk after a P-row prefix)
-    int q_off;             // token index of query row 0 (0, or P for a chunk)
     float eps;
     float scale_log2;      // log2(e) / sqrt(D) times the RoPE variant's logit factor: softmax runs in base 2
     RopeFreqs rf;
@@ -381,8 +379,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int j0 = 2 * pair;
     const int nslots = min(2, p.hpg - j0);
     const int hq0 = g * p.hpg + j0;
-    // causal: K/V tiles 0 .. the one holding the last key the block's last valid row sees
-    const int n_kv = min((p.q_off + min(p.T, (qb + 1) * kBM) - 1) / kBN + 1, (p.Tk + kBN - 1) / kBN);
+    const int n_kv = qb + 1;  // causal: K/V tiles 0 .. qb
 
     const uint32_t sQ0 = sbase + kOffQ, sKV0 = sbase + kOffKV;
     const uint32_t bar0 = sbase + kOffBar;
@@ -554,13 +551,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tmem_ld32(tS + 64, x + 64);
                 tmem_ld32(tS + 96, x + 96);
                 tmem_wait_ld();
-                // causal mask: key j*128 + c is visible to row r iff it is at most the row's
-                // token index q_off + qb*128 + r (only tiles on the diagonal band need it)
-                const int lim = p.q_off + qb * kBM + r - j * kBN;
-                if (lim < kBN - 1) {
+                if (j == qb) {   // diagonal tile: key c is visible to row r iff c <= r
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
-                        if (c > lim) x[c] = -INFINITY;
+                        if (c > r) x[c] = -INFINITY;
                 }
                 // row max with eight independent partial maxima (short dependency chains)
                 float mp[8];

@@ -307,29 +307,6 @@ gqa_status gqa_attn_decode_append_ex(const void *q, const void *k_new, const voi
                                      int H, int Hkv, int D, int max_len, void *workspace,
                                      size_t workspace_bytes, void *stream);
 
-/*
- * Chunked prefill against a cache prefix: the attention stage for a chunk of C new tokens
- * of each sequence whose first P tokens are already cached ("Qwen3系列1" D2-3: earlier
- * tokens' K/V sit in the cache; D1-5: the causal mask on the token index).  Chunk row i
- * (token P + i) attends to keys 0 .. P + i.
- *
- *   q        bf16 [B, C, H, D]       raw queries of the chunk (normed and rotated here)
- *   k_hat    bf16 [B, P + C, Hkv, D] rows 0 .. P-1: the cached prefix k-hat; rows P ..: the
- *                                    chunk's k-hat (e.g. from gqa_attn_k_norm_rope_ex)
- *   v        bf16 [B, P + C, Hkv, D] values, prefix then chunk
- *   pos      int32 [B, C]            positions of the chunk's tokens (RoPE of q)
- *   rope_cs  the table gqa_attn_k_norm_rope_ex wrote for the B*C chunk tokens, or NULL
- *   out      fp32 [B, C, H, D]
- *   rope     the RoPE variant the keys were rotated with (not NULL)
- *
- * P is the same for every sequence of the batch (P = 0 is gqa_attn_prefill_khat_ex).
- * Errors as for gqa_attn_prefill_khat.  Needs no workspace.
- */
-gqa_status gqa_attn_prefill_chunk(const void *q, const void *k_hat, const void *v,
-                                  const int32_t *pos, const float *rope_cs, const float *qnorm_w,
-                                  const gqa_rope_config *rope, float eps, float *out, int B, int C,
-                                  int P, int H, int Hkv, int D, void *stream);
-
 /* ----------------------------------------------------------------- paged KV cache
  *
  * The decode cache may also live in fixed-size pages (the layout of paged-attention
