@@ -619,6 +619,66 @@ void oracle_prefill_chunk_ex(const uint16_t *q, const uint16_t *k, const uint16_
     free(wkd);
 }
 
+/* Variable-length packed prefill: B sequences laid end to end, sequence b owning tokens
+ * cu_seqlens[b] .. cu_seqlens[b+1]-1 of q [N, H, D], k and v [N, Hkv, D] (bf16 bits), with
+ * positions pos [N].  Each token attends causally within its own sequence only ([A]
+ * D1-5 per sequence); out is [N, H, D]. */
+void oracle_prefill_varlen_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                              const int64_t *cu_seqlens, const int32_t *pos, const float *wq,
+                              const float *wk, const double *inv_freq, int pairing,
+                              double logit_mult, double eps, int B, int H, int Hkv, int D,
+                              double *out)
+{
+    int h_per_kv = H / Hkv;
+    double inv_sqrt_d = logit_mult / sqrt((double)D);
+    int64_t N = cu_seqlens[B];
+    int64_t maxlen = 1;
+    for (int b = 0; b < B; ++b)
+        if (cu_seqlens[b + 1] - cu_seqlens[b] > maxlen)
+            maxlen = cu_seqlens[b + 1] - cu_seqlens[b];
+    double *qh = (double *)malloc(sizeof(double) * (size_t)(N * H * D + 1));
+    double *kh = (double *)malloc(sizeof(double) * (size_t)(N * Hkv * D + 1));
+    oracle_qk_transform_ex(q, pos, wq, inv_freq, pairing, eps, N, H, D, qh);
+    oracle_qk_transform_ex(k, pos, wk, inv_freq, pairing, eps, N, Hkv, D, kh);
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * maxlen);
+        double *p = (double *)malloc(sizeof(double) * maxlen);
+        double *vbuf = (double *)malloc(sizeof(double) * (size_t)maxlen * D);
+        const double **vr = (const double **)malloc(sizeof(double *) * maxlen);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t n = 0; n < N; ++n) {
+            int b = 0;
+            while (cu_seqlens[b + 1] <= n)
+                ++b;
+            int64_t t0 = cu_seqlens[b];
+            for (int hq = 0; hq < H; ++hq) {
+                int g = hq / h_per_kv;
+                const double *qi = qh + (n * H + hq) * D;
+                int nkeys = (int)(n - t0 + 1);
+                for (int j = 0; j < nkeys; ++j) {
+                    const double *kj = kh + ((t0 + j) * Hkv + g) * D;
+                    const uint16_t *vj = v + ((t0 + j) * Hkv + g) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) {
+                        dot += qi[d] * kj[d];
+                        vbuf[(int64_t)j * D + d] = bf16_bits_to_double(vj[d]);
+                    }
+                    s[j] = dot * inv_sqrt_d;
+                    vr[j] = vbuf + (int64_t)j * D;
+                }
+                softmax_weighted_sum(s, nkeys, vr, D, p, out + (n * H + hq) * D);
+            }
+        }
+        free(s);
+        free(p);
+        free(vbuf);
+        free(vr);
+    }
+    free(qh);
+    free(kh);
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -67,6 +67,7 @@ def _load():
                                                     I, I, P, P]
             lib.oracle_prefill_chunk_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, Dd, Dd, I, I, I,
                                                     I, I, P, P]
+            lib.oracle_prefill_varlen_ex.argtypes = [P, P, P, P, P, P, P, P, I, Dd, Dd, I, I, I, I, P]
             lib.oracle_num_threads.restype = I
             _lib = lib
     return _lib
@@ -377,3 +378,23 @@ def prefill_chunk_ex(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, offsets
                                     _p(_c(wk, np.float32)), _p(f), rope.pair_code(), rope.logit_mult(), eps, B, C,
                                     H, Hkv, D, _p(out), _p(khat))
     return out, khat
+
+
+def prefill_varlen_ex(q_bits, k_bits, v_bits, cu_seqlens, pos, wq, wk, rope: Rope, eps: float) -> np.ndarray:
+    """Packed variable-length prefill: q [N,H,D], k/v [N,Hkv,D] bf16 bits, sequence b on
+    tokens cu_seqlens[b] .. cu_seqlens[b+1]-1, positions pos [N]; causal within each
+    sequence.  Returns out [N,H,D] fp64."""
+    q_bits = _c(q_bits, np.uint16)
+    k_bits = _c(k_bits, np.uint16)
+    v_bits = _c(v_bits, np.uint16)
+    N, H, D = q_bits.shape
+    Hkv = k_bits.shape[1]
+    cu = _c(cu_seqlens, np.int64)
+    B = cu.shape[0] - 1
+    assert cu[0] == 0 and cu[-1] == N and (np.diff(cu) >= 0).all()
+    f = rope.inv_freq(D)
+    out = np.empty((N, H, D), np.float64)
+    _load().oracle_prefill_varlen_ex(_p(q_bits), _p(k_bits), _p(v_bits), _p(cu), _p(_c(pos, np.int32).reshape(N)),
+                                     _p(_c(wq, np.float32)), _p(_c(wk, np.float32)), _p(f), rope.pair_code(),
+                                     rope.logit_mult(), eps, B, H, Hkv, D, _p(out))
+    return out

@@ -723,3 +723,32 @@ def test_chunk_of_one_token_is_the_append_step():
                                         qpos[:, None], a.wq.numpy(), a.wk.numpy(), rope, a.eps)
     np.testing.assert_array_equal(got[:, 0], ref)
     np.testing.assert_array_equal(khat[:, 0], kref)
+
+
+# --------------------------------------------------------------------------------------
+# Variable-length packed prefill
+# --------------------------------------------------------------------------------------
+
+def test_varlen_prefill_is_each_sequence_on_its_own():
+    """Packing sequences end to end changes nothing: each token attends causally within
+    its own sequence, so every sequence's rows equal its own prefill, and no key of a
+    neighbouring sequence leaks in."""
+    H, Hkv, D = 4, 2, 16
+    lens = [5, 1, 12, 0, 7]
+    seqs = [synthetic.prefill_inputs(1, n, H, Hkv, D=D, seed=100 + i) for i, n in enumerate(lens) if n > 0]
+    q = torch.cat([s.q[0] for s in seqs])
+    k = torch.cat([s.k[0] for s in seqs])
+    v = torch.cat([s.v[0] for s in seqs])
+    pos = torch.cat([s.pos[0] + 1000 * i for i, s in enumerate(seqs)])
+    wq, wk = seqs[0].wq, seqs[0].wk
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    got = oracle.prefill_varlen_ex(_bits(q), _bits(k), _bits(v), cu, pos.numpy(), wq.numpy(), wk.numpy(),
+                                   oracle.Rope(), 1e-6)
+    o = 0
+    for i, s in enumerate(seqs):
+        n = s.q.shape[1]
+        ref = oracle.prefill(_bits(s.q), _bits(s.k), _bits(s.v), (s.pos + 1000 * i).numpy(), wq.numpy(), wk.numpy(),
+                             1e6, 1e-6)[0]
+        np.testing.assert_allclose(got[o:o + n], ref, rtol=0, atol=1e-12)
+        o += n
+    assert o == q.shape[0]
