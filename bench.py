@@ -384,6 +384,26 @@ def run_decode_append(gqa, dev, stream, world, K, W):
                          "kernel": "decode_append_kernel + decode_split_kernel + decode_merge_kernel (one call)"}}
 
 
+def paged_layout(lens, offs, page_size, seed=30):
+    """Page table [B, max pages] (int32, -1 unused) and, for every row of every page, the
+    contiguous cache row it holds (-1: past the end of its sequence), with the pages of all
+    sequences handed out in a seeded random order."""
+    B = len(lens)
+    need = [(int(n) + page_size - 1) // page_size for n in lens]
+    num_pages = sum(need)
+    perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(seed))
+    table = torch.full((B, max(1, max(need))), -1, dtype=torch.int32)
+    src = torch.full((num_pages * page_size,), -1, dtype=torch.int64)
+    start = 0
+    for b in range(B):
+        pids = perm[start:start + need[b]]
+        start += need[b]
+        table[b, :need[b]] = pids.to(torch.int32)
+        rows = torch.arange(int(lens[b]), dtype=torch.int64)
+        src[pids.repeat_interleave(page_size)[:int(lens[b])] * page_size + rows % page_size] = int(offs[b]) + rows
+    return table, src
+
+
 def run_decode_paged(gqa, dec, dq, kc, vc, sl, dwq, dev, stream, world, K, W, page_size=64):
     """gqa_attn_decode_paged on the batched decode workload, its cache copied on the
     device into pages of page_size rows handed out in a seeded random order; CUDA events
@@ -393,19 +413,8 @@ def run_decode_paged(gqa, dec, dq, kc, vc, sl, dwq, dev, stream, world, K, W, pa
     B, H, D = dec.q.shape
     Hkv = dec.k_cache.shape[1]
     lens = dec.seqlens.tolist()
-    offs = dec.offsets.tolist()
-    need = [(n + page_size - 1) // page_size for n in lens]
-    num_pages = sum(need)
-    perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(30))
-    table = torch.full((B, max(need)), -1, dtype=torch.int32)
-    src = torch.full((num_pages * page_size,), -1, dtype=torch.int64)
-    start = 0
-    for b in range(B):
-        pids = perm[start:start + need[b]]
-        start += need[b]
-        table[b, :need[b]] = pids.to(torch.int32)
-        rows = torch.arange(lens[b], dtype=torch.int64)
-        src[pids.repeat_interleave(page_size)[:lens[b]] * page_size + rows % page_size] = offs[b] + rows
+    table, src = paged_layout(lens, dec.offsets.tolist(), page_size)
+    num_pages = src.numel() // page_size
     src = src.to(dev)
     ok = (src >= 0).view(-1, 1, 1)
     kp = torch.where(ok, kc[src.clamp(min=0)], 0).view(num_pages, page_size, Hkv, D)

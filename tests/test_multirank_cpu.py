@@ -73,3 +73,21 @@ def test_traffic_staleness_ignores_comments_only():
     src = "int a = 1;  // one\n/* block\n comment */\nint b = 2;\n"
     assert bench._code_only(src) == bench._code_only("int a = 1;\n// other words\nint b = 2;  /* x */\n")
     assert bench._code_only(src) != bench._code_only("int a = 2;\nint b = 2;\n")
+
+
+def test_paged_layout_maps_every_row_once():
+    """The bench's paged copy: row r of sequence b sits at row r % P of page table[b][r // P],
+    every cache row appears exactly once, and the rest of each last page is empty."""
+    sys.path.insert(0, ROOT)
+    import bench
+    lens, P = [5, 64, 65, 1, 130], 16
+    offs = [0]
+    for n in lens:
+        offs.append(offs[-1] + n)
+    table, src = bench.paged_layout(lens, offs, P)
+    for b, n in enumerate(lens):
+        for r in range(n):
+            assert int(src[int(table[b, r // P]) * P + r % P]) == offs[b] + r
+    used = src[src >= 0]
+    assert sorted(used.tolist()) == list(range(offs[-1]))
+    assert (table[0, :1] >= 0).all() and int(table[0, 1]) == -1
