@@ -679,6 +679,32 @@ void oracle_prefill_varlen_ex(const uint16_t *q, const uint16_t *k, const uint16
     free(kh);
 }
 
+/* Linear projection without bias ([A] D1-2: a linear layer is Y = XW + b, and Qwen3's
+ * projections carry no b; [B] 3.1.2: Qwen3 removed the QKV bias; [C] forward steps 1
+ * and 7: the fused qkv_proj before the attention and o_proj after it, nn.Linear
+ * semantics y = x W^T): y[m][n] = sum_k x[m][k] w[n][k].  x [M, K] and w [N, K] are bf16
+ * bits, y [M, N] fp64, summed in the order k = 0 .. K-1. */
+void oracle_linear(const uint16_t *x, const uint16_t *w, int64_t M, int64_t N, int64_t K, double *y)
+{
+#pragma omp parallel
+    {
+        double *xr = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t m = 0; m < M; ++m) {
+            for (int64_t k = 0; k < K; ++k)
+                xr[k] = bf16_bits_to_double(x[m * K + k]);
+            for (int64_t n = 0; n < N; ++n) {
+                const uint16_t *wr = w + n * K;
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k)
+                    acc += xr[k] * bf16_bits_to_double(wr[k]);
+                y[m * N + n] = acc;
+            }
+        }
+        free(xr);
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -68,6 +68,7 @@ def _load():
             lib.oracle_prefill_chunk_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, Dd, Dd, I, I, I,
                                                     I, I, P, P]
             lib.oracle_prefill_varlen_ex.argtypes = [P, P, P, P, P, P, P, P, I, Dd, Dd, I, I, I, I, P]
+            lib.oracle_linear.argtypes = [P, P, L, L, L, P]
             lib.oracle_num_threads.restype = I
             _lib = lib
     return _lib
@@ -398,3 +399,38 @@ def prefill_varlen_ex(q_bits, k_bits, v_bits, cu_seqlens, pos, wq, wk, rope: Rop
                                      _p(_c(wq, np.float32)), _p(_c(wk, np.float32)), _p(f), rope.pair_code(),
                                      rope.logit_mult(), eps, B, H, Hkv, D, _p(out))
     return out
+
+
+def linear(x_bits, w_bits) -> np.ndarray:
+    """Projection without bias: y = x W^T over the last axis of x (nn.Linear; the pages
+    give Qwen3's projections no bias).  x [..., K] and w [N, K] bf16 bits -> y [..., N]
+    fp64."""
+    x_bits = _c(x_bits, np.uint16)
+    w_bits = _c(w_bits, np.uint16)
+    K = x_bits.shape[-1]
+    N = w_bits.shape[0]
+    assert w_bits.shape == (N, K)
+    M = x_bits.size // K if K else 0
+    y = np.empty(x_bits.shape[:-1] + (N,), np.float64)
+    _load().oracle_linear(_p(x_bits), _p(w_bits), M, N, K, _p(y))
+    return y
+
+
+def qkv_proj(x_bits, w_qkv_bits, H: int, Hkv: int, D: int):
+    """Fused QKV projection, then the split and the per-head view of the "Qwen3"
+    walkthrough's forward steps 1-3: qkv = x W_qkv^T with W_qkv = [W_q; W_k; W_v]
+    ((H + 2 Hkv) D rows), split into H D, Hkv D, Hkv D columns and viewed as
+    q [N, H, D], k [N, Hkv, D], v [N, Hkv, D] (fp64)."""
+    y = linear(x_bits, w_qkv_bits)
+    N = y.size // ((H + 2 * Hkv) * D)
+    y = y.reshape(N, H + 2 * Hkv, D)
+    return y[:, :H], y[:, H:H + Hkv], y[:, H + Hkv:]
+
+
+def o_proj(o_bits, w_o_bits) -> np.ndarray:
+    """Output projection of the "Qwen3" walkthrough's forward step 7: the heads of the
+    attention output o [N, H, D] (bf16 bits) flattened to [N, H D], times W_o^T
+    (W_o [hidden, H D]) -> [N, hidden] fp64."""
+    o_bits = _c(o_bits, np.uint16)
+    N = o_bits.shape[0]
+    return linear(o_bits.reshape(N, -1), w_o_bits)

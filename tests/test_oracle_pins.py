@@ -752,3 +752,76 @@ def test_varlen_prefill_is_each_sequence_on_its_own():
         np.testing.assert_allclose(got[o:o + n], ref, rtol=0, atol=1e-12)
         o += n
     assert o == q.shape[0]
+
+
+# ----------------------------------------------------------------------------- projections
+# "Qwen3系列1" D1-2 (a linear layer is Y = XW + b; Qwen3's projections have no b), D1-4
+# Q4/Q5 (heads concatenated, then W_O); "深入剖析Qwen3模型架构" 3.1.2 (no QKV bias); the
+# "Qwen3" walkthrough's forward steps 1-3 (qkv_proj, split, per-head view) and 7 (o_proj).
+
+def _bf(a):
+    return synthetic.bf16_bits(torch.as_tensor(np.asarray(a, np.float32)).to(torch.bfloat16))
+
+
+def test_linear_worked_example():
+    """y = x W^T by hand: x = [[1,2,3],[4,5,6]], W = [[1,0,-1],[2,1,0]] gives
+    [[1-3, 2+2], [4-6, 8+5]] = [[-2, 4], [-2, 13]].  A transposed W (3x2) or x W
+    instead of x W^T cannot produce this shape and these values."""
+    y = oracle.linear(_bf([[1, 2, 3], [4, 5, 6]]), _bf([[1, 0, -1], [2, 1, 0]]))
+    np.testing.assert_array_equal(y, [[-2.0, 4.0], [-2.0, 13.0]])
+
+
+def test_linear_identity_scaling_and_permutation():
+    g = torch.Generator().manual_seed(200)
+    x = torch.randn(5, 64, generator=g).to(torch.bfloat16)
+    xb = synthetic.bf16_bits(x)
+    # identity weights return the input exactly (every bf16 value is a double)
+    np.testing.assert_array_equal(oracle.linear(xb, _bf(np.eye(64))), x.double().numpy())
+    w = torch.randn(48, 64, generator=g).to(torch.bfloat16)
+    y = oracle.linear(xb, synthetic.bf16_bits(w))
+    # doubling the weights doubles the output exactly
+    np.testing.assert_array_equal(oracle.linear(xb, synthetic.bf16_bits(w * 2)), 2 * y)
+    # permuting the output rows of W permutes the output columns
+    perm = torch.randperm(48, generator=g)
+    np.testing.assert_array_equal(oracle.linear(xb, synthetic.bf16_bits(w[perm])), y[:, perm.numpy()])
+    # linear in x: inputs with disjoint supports add
+    mask = torch.arange(64) % 3 == 0
+    x1, x2 = torch.where(mask, x, 0), torch.where(mask, 0, x)
+    y12 = oracle.linear(synthetic.bf16_bits(x1), synthetic.bf16_bits(w)) + \
+        oracle.linear(synthetic.bf16_bits(x2), synthetic.bf16_bits(w))
+    np.testing.assert_allclose(y12, y, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_matches_torch_fp64_matmul():
+    g = torch.Generator().manual_seed(201)
+    x = torch.randn(7, 3, 96, generator=g).to(torch.bfloat16)
+    w = torch.randn(40, 96, generator=g).to(torch.bfloat16)
+    ref = (x.double() @ w.double().T).numpy()
+    got = oracle.linear(synthetic.bf16_bits(x), synthetic.bf16_bits(w))
+    assert got.shape == (7, 3, 40)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-11)
+
+
+def test_qkv_proj_splits_into_the_three_projections():
+    """The fused projection's q, k and v sections are the separate q/k/v projections
+    (W_qkv = [W_q; W_k; W_v]) viewed per head, bit for bit."""
+    H, Hkv, D, hidden = 4, 2, 16, 32
+    g = torch.Generator().manual_seed(202)
+    x = synthetic.bf16_bits(torch.randn(6, hidden, generator=g).to(torch.bfloat16))
+    wq, wk, wv = (torch.randn(n * D, hidden, generator=g).to(torch.bfloat16) for n in (H, Hkv, Hkv))
+    q, k, v = oracle.qkv_proj(x, synthetic.bf16_bits(torch.cat([wq, wk, wv])), H, Hkv, D)
+    np.testing.assert_array_equal(q, oracle.linear(x, synthetic.bf16_bits(wq)).reshape(6, H, D))
+    np.testing.assert_array_equal(k, oracle.linear(x, synthetic.bf16_bits(wk)).reshape(6, Hkv, D))
+    np.testing.assert_array_equal(v, oracle.linear(x, synthetic.bf16_bits(wv)).reshape(6, Hkv, D))
+
+
+def test_o_proj_is_concat_then_w_o():
+    """Concatenating the heads and applying W_O equals summing each head's share of W_O:
+    o_proj(o) = sum_h o[:, h] W_O[:, h D:(h+1) D]^T."""
+    H, D, hidden = 3, 8, 20
+    g = torch.Generator().manual_seed(203)
+    o = torch.randn(5, H, D, generator=g).to(torch.bfloat16)
+    w = torch.randn(hidden, H * D, generator=g).to(torch.bfloat16)
+    got = oracle.o_proj(synthetic.bf16_bits(o), synthetic.bf16_bits(w))
+    ref = sum(o[:, h].double() @ w[:, h * D:(h + 1) * D].double().T for h in range(H)).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-11)
