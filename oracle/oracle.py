@@ -434,3 +434,38 @@ def o_proj(o_bits, w_o_bits) -> np.ndarray:
     o_bits = _c(o_bits, np.uint16)
     N = o_bits.shape[0]
     return linear(o_bits.reshape(N, -1), w_o_bits)
+
+
+def round_bf16_bits(a) -> np.ndarray:
+    """fp64 values rounded to the nearest bfloat16 (ties to even), returned as bf16 bit
+    patterns: the dtype boundary where a bf16 model stores a tensor.  Written from the
+    format (8 significant bits, 8 exponent bits) for finite normal-range values."""
+    a = np.asarray(a, np.float64)
+    m, e = np.frexp(a)                     # a = m 2^e, 0.5 <= |m| < 1
+    r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)   # 8 significant bits, ties to even
+    return (r.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def attn_block_prefill(x_bits, w_qkv_bits, w_o_bits, pos, wq, wk, rope: Rope, eps: float, H: int, Hkv: int,
+                       D: int, rows=None) -> np.ndarray:
+    """The attention sub-block of a prefill in the order of the "Qwen3" walkthrough's
+    forward steps: qkv projection (steps 1-3), q/k RMSNorm (4), RoPE (5), causal GQA
+    attention (6), output projection over the concatenated heads (7).  x [B, T, hidden]
+    bf16 bits; q, k, v and the attention output are stored as bf16 between the steps
+    (the tensors' dtype in a bf16 model), every step computed in fp64.  Returns y
+    [B, T, hidden] fp64, or, with rows (an array of (b, t)), only those rows (the
+    attention rows of every head of those tokens are evaluated one by one)."""
+    x_bits = _c(x_bits, np.uint16)
+    B, T, hidden = x_bits.shape
+    q, k, v = qkv_proj(x_bits.reshape(B * T, hidden), w_qkv_bits, H, Hkv, D)
+    qb = round_bf16_bits(q).reshape(B, T, H, D)
+    kb = round_bf16_bits(k).reshape(B, T, Hkv, D)
+    vb = round_bf16_bits(v).reshape(B, T, Hkv, D)
+    if rows is None:
+        rs = np.array([(b, h, t) for b in range(B) for t in range(T) for h in range(H)], np.int64)
+    else:
+        rs = np.array([(b, h, t) for b, t in rows for h in range(H)], np.int64)
+    o = prefill_rows_ex(qb, kb, vb, pos, wq, wk, rope, eps, rs)
+    ob = round_bf16_bits(o).reshape(-1, H, D)
+    y = o_proj(ob, w_o_bits)
+    return y.reshape(B, T, hidden) if rows is None else y

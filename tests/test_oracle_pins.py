@@ -825,3 +825,54 @@ def test_o_proj_is_concat_then_w_o():
     got = oracle.o_proj(synthetic.bf16_bits(o), synthetic.bf16_bits(w))
     ref = sum(o[:, h].double() @ w[:, h * D:(h + 1) * D].double().T for h in range(H)).numpy()
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-11)
+
+
+def test_round_bf16_ties_to_even_and_matches_torch():
+    # 1 + 2^-8 lies halfway between 1 and 1 + 2^-7: the even neighbour is 1;
+    # 1 + 3 * 2^-8 lies halfway between 1 + 2^-7 and 1 + 2^-6: the even one is 1 + 2^-6
+    got = oracle.round_bf16_bits([1.0, 1 + 2 ** -8, 1 + 3 * 2 ** -8, -2.5, 0.0, 3.0e-3])
+    assert got[0] == 0x3F80 and got[1] == 0x3F80 and got[2] == 0x3F82
+    assert got[3] == 0xC020 and got[4] == 0
+    g = torch.Generator().manual_seed(204)
+    x = torch.randn(10000, generator=g) * 10.0 ** torch.randint(-3, 4, (10000,), generator=g)
+    ref = synthetic.bf16_bits(x.to(torch.bfloat16))
+    np.testing.assert_array_equal(oracle.round_bf16_bits(x.double().numpy()), ref)
+
+
+def test_attention_block_with_identity_projections_is_the_prefill():
+    """With W_qkv = [I; I_kv; I_kv] (hidden = H D, k and v the first Hkv D features) and
+    W_o = I, the sub-block reduces to the prefill on q = x, k = v = x[:, :Hkv D], rounded
+    to bf16 at the end: steps in the pages' order, split at the right boundaries."""
+    B, T, H, Hkv, D = 1, 40, 4, 2, 16
+    hidden = H * D
+    inp = synthetic.prefill_inputs(B, T, H, Hkv, D=D, seed=205)
+    x = inp.q.reshape(B, T, hidden)
+    eye = torch.eye(hidden)
+    w_qkv = torch.cat([eye, eye[:Hkv * D], eye[:Hkv * D]]).to(torch.bfloat16)
+    w_o = eye.to(torch.bfloat16)
+    rope = oracle.Rope(theta=inp.theta)
+    y = oracle.attn_block_prefill(synthetic.bf16_bits(x), synthetic.bf16_bits(w_qkv), synthetic.bf16_bits(w_o),
+                                  inp.pos.numpy(), inp.wq.numpy(), inp.wk.numpy(), rope, inp.eps, H, Hkv, D)
+    xk = x.reshape(B, T, H, D)[:, :, :Hkv].contiguous()
+    o = oracle.prefill(synthetic.bf16_bits(inp.q), synthetic.bf16_bits(xk), synthetic.bf16_bits(xk),
+                       inp.pos.numpy(), inp.wq.numpy(), inp.wk.numpy(), inp.theta, inp.eps)
+    ref = oracle.round_bf16_bits(o).view(np.uint16)
+    ref = torch.from_numpy(ref.astype(np.int16)).view(torch.bfloat16).double().numpy().reshape(B, T, hidden)
+    np.testing.assert_array_equal(y, ref)
+
+
+def test_attention_block_rows_equal_the_full_block():
+    B, T, H, Hkv, D, hidden = 2, 24, 4, 2, 16, 48
+    g = torch.Generator().manual_seed(206)
+    x = torch.randn(B, T, hidden, generator=g).to(torch.bfloat16)
+    w_qkv = (torch.randn((H + 2 * Hkv) * D, hidden, generator=g) / hidden ** 0.5).to(torch.bfloat16)
+    w_o = (torch.randn(hidden, H * D, generator=g) / (H * D) ** 0.5).to(torch.bfloat16)
+    pos = torch.arange(T, dtype=torch.int32).repeat(B, 1).numpy()
+    wq = np.linspace(0.5, 1.5, D).astype(np.float32)
+    wk = wq[::-1].copy()
+    args = (synthetic.bf16_bits(x), synthetic.bf16_bits(w_qkv), synthetic.bf16_bits(w_o), pos, wq, wk,
+            oracle.Rope(theta=1e6), 1e-6, H, Hkv, D)
+    full = oracle.attn_block_prefill(*args)
+    rows = [(1, 0), (0, 23), (1, 17)]
+    part = oracle.attn_block_prefill(*args, rows=rows)
+    np.testing.assert_array_equal(part, np.stack([full[b, t] for b, t in rows]))
