@@ -2,11 +2,14 @@
 KV-read GB/s, each against its roofline.
 
 One step = one pass of the whole hot path over one batch of synthetic inputs:
-  * prefill, large workload (B=4, T=4096, H=32, Hkv=8, D=128, inputs x0.5):
-    k-hat prologue (RMSNorm + RoPE of K) then the fused q-prologue + causal GQA
-    attention kernel;
+  * prefill, the long-context workload (B=1, T=32768, H=64, Hkv=8, D=128), the
+    largest single-GPU prefill: k-hat prologue (RMSNorm + RoPE of K) then the fused
+    q-prologue + causal GQA attention kernel;
   * decode, batched workload (64 sequences, cache lengths U[1024, 32768], H=32,
     Hkv=8, D=128): split-KV kernel then the log-sum-exp merge.
+The large prefill (B=4, T=4096, H=32, Hkv=8, inputs x0.5), the decode step with cache
+append and the paged-cache decode are timed in regions of their own and reported as
+extra keys.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -39,13 +42,21 @@ sys.path.insert(0, ROOT)
 from grouped_query_causal_b200 import synthetic  # noqa: E402
 
 METRIC = "prefill attn TFLOPS and decode KV-read GB/s on 1 B200, % of roofline"
-PREFILL = "large_prefill"
+PREFILL = "long_context_prefill"
+PREFILL_EXTRA = "large_prefill"
 DECODE = "batched_decode"
+WORKLOAD_TEXT = {
+    "long_context_prefill": "long-context prefill (B1 T32768 H64 Hkv8 D128, causal)",
+    "large_prefill": "large prefill (B4 T4096 H32 Hkv8 D128, inputs x0.5, causal)",
+    "batched_decode": "batched decode (64 seqs, cache len U[1024,32768], H32 Hkv8 D128)",
+}
+L2_FLUSH_BYTES = 256 << 20   # written between timed calls whose inputs may still sit in L2 (126 MB)
 DECODE_APPEND = "batched_decode_append"
-# The sources each kernel is compiled from; its ncu traffic figure is stale once they change.
+# The sources each kernel is compiled from; its ncu traffic figures are stale once they change.
 KERNEL_SOURCES = {
     "attn_fwd_kernel": ["prefill.cuh", "ptx.cuh", "rope.cuh", "gqa_attn.cu"],
     "decode_split_kernel": ["decode.cuh", "ptx.cuh", "rope.cuh", "gqa_attn.cu"],
+    "decode_split_kernel<paged>": ["decode.cuh", "ptx.cuh", "rope.cuh", "gqa_attn.cu"],
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -112,9 +123,10 @@ def kernel_source_hash(kernel):
     return h.hexdigest()[:16]
 
 
-def traffic_from_profiles(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
-    kernel sources changed since the counters were taken."""
+def traffic_from_profiles(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary
+    (profiles/traffic.json), or None when there is none or the kernel's sources changed
+    since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -124,7 +136,8 @@ def traffic_from_profiles(kernel):
     e = t.get(kernel)
     if not e or kernel not in KERNEL_SOURCES or e.get("source_hash") != kernel_source_hash(kernel):
         return None
-    return e.get("dram_bytes_per_launch")
+    w = e.get("workloads", {}).get(workload)
+    return None if w is None else w.get("dram_bytes_per_launch")
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -267,6 +280,13 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the public API with host buffers (pinned), copies timed
     e2e = run_e2e(gqa, pin, dec, dev, stream, rank, world, max(3, min(K, 10)))
 
+    # ---- the large prefill (its own timed region)
+    extra = run_prefill_leg(gqa, PREFILL_EXTRA, dev, stream, world, K, args.warmup)
+    # ---- packed variable-length and chunked prefill, the projections (own timed regions)
+    varlen = run_packed_leg(gqa, "varlen_prefill", dev, stream, world, K, args.warmup)
+    chunked = run_packed_leg(gqa, "chunked_prefill", dev, stream, world, K, args.warmup)
+    proj = run_projection_leg(gqa, dev, stream, world, K, args.warmup)
+    block = run_block_leg(gqa, dev, stream, world, K, args.warmup)
     # ---- the decode step that appends the new token first (its own timed region)
     app = run_decode_append(gqa, dev, stream, world, K, args.warmup)
     # ---- the batched decode on a paged copy of the same cache (its own timed region)
@@ -280,9 +300,18 @@ def run_ours(args, rank, world, local_rank):
     # cuBLAS measurement; the power-capped sustained figure is reported for context.
     tc = float(pk["bf16_tflops"])
     attn_tflops = flops * K / (attn_ms / 1e3) / 1e12
+    total_tflops = flops * K / prefill_s / 1e12
     dec_gbs = dbytes * K / dec_s / 1e9
-    traffic_attn = traffic_from_profiles("attn_fwd_kernel")
-    traffic_dec = traffic_from_profiles("decode_split_kernel")
+    traffic_attn = traffic_from_profiles("attn_fwd_kernel", PREFILL)
+    traffic_dec = traffic_from_profiles("decode_split_kernel", DECODE)
+    hbm_line = lambda leg: dict(leg, roofline=dict(leg["roofline"], peak=hbm,  # noqa: E731
+                                                   frac=round(leg["roofline"]["achieved"] / hbm, 4),
+                                                   peak_source=f"hbm_gbs of {pk_kind}"))
+    tc_line = lambda leg: dict(leg, roofline=dict(leg["roofline"], peak=tc,  # noqa: E731
+                                                  frac=round(leg["roofline"]["achieved"] / tc, 4),
+                                                  peak_source=f"bf16_tflops (burst) of {pk_kind}",
+                                                  **({"frac_incl_k_prologue": round(leg["value"] / world / tc, 4)}
+                                                     if "k_prologue_ms" in leg else {})))
     line = {
         "metric": METRIC,
         "value": round(whole_job_rate(flops * K, world, prefill_s) / 1e12, 2),
@@ -297,12 +326,12 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": "large prefill (B4 T4096 H32 Hkv8 D128, inputs x0.5, causal) + batched decode "
-                        "(64 seqs, cache len U[1024,32768], H32 Hkv8 D128)",
+            "workload": f"{WORKLOAD_TEXT[PREFILL]} + {WORKLOAD_TEXT[DECODE]}",
             "prefill": {"B": B, "T": T, "H": H, "Hkv": Hkv, "D": D, "flops_per_step": flops},
             "decode": {"B": dB, "H": dH, "Hkv": dHkv, "D": D, "cached_tokens": int(dec.seqlens.sum()),
                        "bytes_per_step": dbytes},
-            "l2": "inputs larger than L2 (prefill q/k/v/out 470 MB; decode KV cache 4.4 GB); no flush",
+            "l2": "inputs larger than L2 (prefill q/k/v/out 1.75 GB; decode KV cache 3.9 GB); no flush in the "
+                  "step; the extra legs write 256 MB between timed calls",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         },
         "prefill_ms": round(1e3 * prefill_s / K, 4),
@@ -316,18 +345,22 @@ def run_ours(args, rank, world, local_rank):
                          "peak_source": f"hbm_gbs of {pk_kind}"},
             "e2e": e2e["decode"],
         },
+        # value counts the k-hat prologue and the attention kernel; roofline is the
+        # attention kernel alone (the dominant kernel), frac_incl_k_prologue both.
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": tc, "unit": "TFLOP/s",
-                     "frac": round(attn_tflops / tc, 4), "traffic": traffic_attn, "kernel": "attn_fwd_kernel",
+                     "frac": round(attn_tflops / tc, 4), "frac_incl_k_prologue": round(total_tflops / tc, 4),
+                     "traffic": traffic_attn, "kernel": "attn_fwd_kernel",
                      "attn_ms": round(attn_ms / K, 4), "k_prologue_ms": round(pro_ms / K, 4),
                      "peak_source": f"bf16_tflops (burst) of {pk_kind}",
                      "peak_sustained": float(pk.get("bf16_tflops_sustained", tc))},
         "e2e": e2e["prefill"],
-        "decode_append": dict(app, roofline=dict(app["roofline"], peak=hbm,
-                                                 frac=round(app["roofline"]["achieved"] / hbm, 4),
-                                                 peak_source=f"hbm_gbs of {pk_kind}")),
-        "decode_paged": dict(paged, roofline=dict(paged["roofline"], peak=hbm,
-                                                  frac=round(paged["roofline"]["achieved"] / hbm, 4),
-                                                  peak_source=f"hbm_gbs of {pk_kind}")),
+        "large_prefill": tc_line(extra),
+        "varlen_prefill": tc_line(varlen),
+        "chunked_prefill": tc_line(chunked),
+        "projections": tc_line(proj),
+        "attn_block": tc_line(block),
+        "decode_append": hbm_line(app),
+        "decode_paged": hbm_line(paged),
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
@@ -336,10 +369,230 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+def timed_calls(call, stream, world, dev, K, W, flush=None):
+    """W untimed calls, then K calls each between its own pair of CUDA events on `stream`
+    (with `flush`, a 256 MB write between calls, outside the events); returns the summed
+    seconds per event pair (a list), maximum over ranks."""
+    for _ in range(W):
+        call(None)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    evs = []
+    for i in range(K):
+        if flush is not None:
+            flush.fill_(i & 255)
+        evs.append(call(stream))
+    torch.cuda.synchronize()
+    n = len(evs[0]) - 1
+    ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(n)]
+    return [x / 1e3 for x in max_over_ranks(ms, dev, world)]
+
+
+def run_prefill_leg(gqa, name, dev, stream, world, K, W):
+    """The k-hat prologue and attention kernel on the prefill workload `name`, inputs
+    resident, each call between CUDA events (prologue and attention separately), L2
+    flushed between calls."""
+    lib = gqa.load()
+    sh = stream.cuda_stream
+    w = synthetic.make(name)
+    B, T, H, D = w.q.shape
+    Hkv = w.k.shape[2]
+    q, k, v, pos, wq, wk = (x.to(dev) for x in (w.q, w.k, w.v, w.pos, w.wq, w.wk))
+    khat = torch.empty_like(k)
+    rope_cs = torch.empty(gqa.rope_table_numel(B * T, D), dtype=torch.float32, device=dev)
+    out = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ptr = lambda t: t.data_ptr()  # noqa: E731
+
+    def call(st_):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if st_ is not None else None
+        if ev:
+            ev[0].record(st_)
+        st = lib.gqa_attn_k_norm_rope(ptr(k), ptr(pos), ptr(wk), w.theta, w.eps, ptr(khat), ptr(rope_cs), B * T,
+                                      Hkv, D, sh)
+        if ev:
+            ev[1].record(st_)
+        st |= lib.gqa_attn_prefill_khat(ptr(q), ptr(khat), ptr(v), ptr(pos), ptr(rope_cs), ptr(wq), w.theta, w.eps,
+                                        ptr(out), B, T, H, Hkv, D, sh)
+        if ev:
+            ev[2].record(st_)
+        if st != 0:
+            raise RuntimeError(f"{name}: library call failed with status {st}")
+        return ev
+
+    pro_s, attn_s = timed_calls(call, stream, world, dev, K, W, flush)
+    if gqa.device_status() != 0:
+        raise RuntimeError(f"device status error in the {name} timing")
+    flops = prefill_flops(B, T, H, D)
+    del q, k, v, pos, khat, rope_cs, out, flush
+    return {"value": round(whole_job_rate(flops * K, world, pro_s + attn_s) / 1e12, 2), "unit": "TFLOP/s",
+            "ms": round(1e3 * (pro_s + attn_s) / K, 4), "attn_ms": round(1e3 * attn_s / K, 4),
+            "k_prologue_ms": round(1e3 * pro_s / K, 4), "workload": WORKLOAD_TEXT[name],
+            "flops_per_call": flops, "gpu_launches": 2 * K,
+            "roofline": {"bound": "tensor", "achieved": round(flops * K / attn_s / 1e12, 2), "unit": "TFLOP/s",
+                         "traffic": traffic_from_profiles("attn_fwd_kernel", name), "kernel": "attn_fwd_kernel"}}
+
+
+def packed_flops(lens, prefix, H, D=128):
+    """Algorithmic FLOPs of causal attention over packed sequences: chunk row t of
+    sequence b sees prefix[b] + t + 1 keys, 4 D FLOP each (QK^T and PV)."""
+    return sum(4 * D * H * (n * p + n * (n + 1) // 2) for n, p in zip(lens, prefix))
+
+
+def run_packed_leg(gqa, name, dev, stream, world, K, W):
+    """gqa_attn_prefill_varlen (no prefix) or gqa_attn_prefill_chunk (each sequence has
+    cached rows; the chunk is appended to the cache first) on a packed workload, inputs
+    resident, CUDA events around each call, L2 flushed between calls."""
+    lib = gqa.load()
+    sh = stream.cuda_stream
+    w = synthetic.make(name)
+    N, H, D = w.q.shape
+    Hkv = w.k.shape[1]
+    B = len(w.lens)
+    chunk = w.prefix is not None
+    t = {n: getattr(w, n).to(dev) for n in ("q", "k", "v", "pos", "cu", "wq", "wk")}
+    if chunk:
+        t.update({n: getattr(w, n).to(dev) for n in ("k_cache", "v_cache", "cache_offsets", "prefix")})
+        ws_n = lib.gqa_attn_prefill_chunk_workspace_size(N, D)
+    else:
+        ws_n = lib.gqa_attn_prefill_varlen_workspace_size(N, Hkv, D)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
+    out = torch.empty((N, H, D), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    rope = gqa.RopeConfig.make(theta=w.theta)
+    maxlen = max(w.lens)
+    ptr = lambda x: x.data_ptr()  # noqa: E731
+
+    def call(st_):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)] if st_ is not None else None
+        if ev:
+            ev[0].record(st_)
+        if chunk:
+            st = lib.gqa_attn_prefill_chunk(ptr(t["q"]), ptr(t["k"]), ptr(t["v"]), ptr(t["pos"]), ptr(t["cu"]),
+                                            ptr(t["k_cache"]), ptr(t["v_cache"]), ptr(t["cache_offsets"]),
+                                            ptr(t["prefix"]), t["k_cache"].shape[0], ptr(t["wq"]), ptr(t["wk"]),
+                                            ctypes.byref(rope), w.eps, ptr(out), B, N, H, Hkv, D, maxlen, ptr(ws),
+                                            ws.numel(), sh)
+        else:
+            st = lib.gqa_attn_prefill_varlen(ptr(t["q"]), ptr(t["k"]), ptr(t["v"]), ptr(t["pos"]), ptr(t["cu"]),
+                                             ptr(t["wq"]), ptr(t["wk"]), ctypes.byref(rope), w.eps, ptr(out), B, N,
+                                             H, Hkv, D, maxlen, ptr(ws), ws.numel(), sh)
+        if ev:
+            ev[1].record(st_)
+        if st != 0:
+            raise RuntimeError(f"{name}: library call failed with status {st}")
+        return ev
+
+    sec = timed_calls(call, stream, world, dev, K, W, flush)[0]
+    if gqa.device_status() != 0:
+        raise RuntimeError(f"device status error in the {name} timing")
+    prefix = w.prefix.tolist() if chunk else [0] * B
+    flops = packed_flops(w.lens, prefix, H, D)
+    del t, ws, out, flush
+    what = (f"{B} sequences, {prefix[0]} cached rows + a {w.lens[0]}-token chunk each, H{H} Hkv{Hkv} D{D}"
+            if chunk else f"{B} packed sequences, lengths U[256,8192] (N={N}), H{H} Hkv{Hkv} D{D}")
+    return {"value": round(whole_job_rate(flops * K, world, sec) / 1e12, 2), "unit": "TFLOP/s",
+            "ms": round(1e3 * sec / K, 4), "workload": what, "flops_per_call": flops, "gpu_launches": 2 * K,
+            "roofline": {"bound": "tensor", "achieved": round(flops * K / sec / 1e12, 2), "unit": "TFLOP/s",
+                         "traffic": None, "kernel": "k_prologue_kernel + attn_fwd_kernel (one call)"}}
+
+
+def run_projection_leg(gqa, dev, stream, world, K, W):
+    """gqa_linear as the fused QKV projection (16384 x 4096 -> 6144, bf16 out) and as the
+    output projection (16384 x 4096 -> 4096, fp32 out), each call between CUDA events, L2
+    flushed between calls."""
+    lib = gqa.load()
+    sh = stream.cuda_stream
+    w = synthetic.make("projections")
+    x, wqkv, wo = w.x.to(dev), w.w_qkv.to(dev), w.w_o.to(dev)
+    M, hidden = x.shape
+    Nq = wqkv.shape[0]
+    qkv = torch.empty((M, Nq), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((M, hidden), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def call(st_):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if st_ is not None else None
+        if ev:
+            ev[0].record(st_)
+        st = lib.gqa_linear(x.data_ptr(), wqkv.data_ptr(), qkv.data_ptr(), 0, M, Nq, hidden, sh)
+        if ev:
+            ev[1].record(st_)
+        # the output projection reads an [M, H D] bf16 operand (H D = hidden here); x stands
+        # in for the attention output (same shape and dtype)
+        st |= lib.gqa_linear(x.data_ptr(), wo.data_ptr(), y.data_ptr(), 1, M, hidden, hidden, sh)
+        if ev:
+            ev[2].record(st_)
+        if st != 0:
+            raise RuntimeError(f"gqa_linear failed with status {st}")
+        return ev
+
+    s_qkv, s_o = timed_calls(call, stream, world, dev, K, W, flush)
+    if gqa.device_status() != 0:
+        raise RuntimeError("device status error in the projection timing")
+    f_qkv, f_o = 2 * M * Nq * hidden, 2 * M * hidden * hidden
+    del x, wqkv, wo, qkv, y, flush
+    return {"value": round(whole_job_rate((f_qkv + f_o) * K, world, s_qkv + s_o) / 1e12, 2), "unit": "TFLOP/s",
+            "workload": f"qkv_proj {M}x{hidden} -> {Nq} (bf16 out) and o_proj {M}x{hidden} -> {hidden} (fp32 out)",
+            "qkv_ms": round(1e3 * s_qkv / K, 4), "o_proj_ms": round(1e3 * s_o / K, 4),
+            "qkv_tflops": round(f_qkv * K / s_qkv / 1e12, 2), "o_proj_tflops": round(f_o * K / s_o / 1e12, 2),
+            "gpu_launches": 2 * K,
+            "roofline": {"bound": "tensor", "achieved": round((f_qkv + f_o) * K / (s_qkv + s_o) / 1e12, 2),
+                         "unit": "TFLOP/s", "traffic": None, "kernel": "gemm_kernel"}}
+
+
+def run_block_leg(gqa, dev, stream, world, K, W):
+    """gqa_attn_block_prefill, the whole attention sub-block (qkv projection, q/k norm,
+    RoPE, causal GQA attention, output projection) on the large prefill's shape with
+    hidden 4096, CUDA events around each call, L2 flushed between calls."""
+    lib = gqa.load()
+    sh = stream.cuda_stream
+    B, T, H, Hkv, D, hidden = 4, 4096, 32, 8, 128, 4096
+    w = synthetic.projection_inputs(B * T, hidden, H, Hkv, seed=40)
+    x, wqkv, wo = w.x.to(dev), w.w_qkv.to(dev), w.w_o.to(dev)
+    pos = torch.arange(T, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+    g = torch.Generator().manual_seed(41)
+    wq = (torch.rand(D, generator=g) + 0.5).to(dev)
+    wk = (torch.rand(D, generator=g) + 0.5).to(dev)
+    y = torch.empty((B * T, hidden), dtype=torch.float32, device=dev)
+    ws = torch.empty(lib.gqa_attn_block_prefill_workspace_size(B, T, hidden, H, Hkv, D), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    rope = gqa.RopeConfig.make(theta=synthetic.THETA)
+
+    def call(st_):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)] if st_ is not None else None
+        if ev:
+            ev[0].record(st_)
+        st = lib.gqa_attn_block_prefill(x.data_ptr(), wqkv.data_ptr(), wo.data_ptr(), pos.data_ptr(), wq.data_ptr(),
+                                        wk.data_ptr(), ctypes.byref(rope), synthetic.EPS, y.data_ptr(), B, T, hidden,
+                                        H, Hkv, D, ws.data_ptr(), ws.numel(), sh)
+        if ev:
+            ev[1].record(st_)
+        if st != 0:
+            raise RuntimeError(f"gqa_attn_block_prefill failed with status {st}")
+        return ev
+
+    sec = timed_calls(call, stream, world, dev, K, W, flush)[0]
+    if gqa.device_status() != 0:
+        raise RuntimeError("device status error in the attention-block timing")
+    N = B * T
+    flops = 2 * N * (H + 2 * Hkv) * D * hidden + prefill_flops(B, T, H, D) + 2 * N * hidden * H * D
+    del x, wqkv, wo, y, ws, flush
+    return {"value": round(whole_job_rate(flops * K, world, sec) / 1e12, 2), "unit": "TFLOP/s",
+            "ms": round(1e3 * sec / K, 4), "flops_per_call": flops,
+            "workload": f"attention sub-block B{B} T{T} hidden {hidden} H{H} Hkv{Hkv} D{D}: qkv_proj, q/k norm, "
+                        "RoPE, causal GQA attention, o_proj", "gpu_launches": 4 * K,
+            "roofline": {"bound": "tensor", "achieved": round(flops * K / sec / 1e12, 2), "unit": "TFLOP/s",
+                         "traffic": None, "kernel": "gemm_kernel, k_prologue_kernel, attn_fwd_kernel, gemm_kernel"}}
+
+
 def run_decode_append(gqa, dev, stream, world, K, W):
     """gqa_attn_decode_append on the batched append workload (64 sequences with
-    1023..32767 cached rows, one new token each), inputs resident, CUDA events around K
-    calls after W warm-up calls.  Every call writes the same rows with the same values."""
+    1023..32767 cached rows, one new token each), inputs resident, CUDA events around each
+    of K calls after W warm-up calls, L2 flushed between calls.  Every call writes the
+    same rows with the same values."""
     lib = gqa.load()
     sh = stream.cuda_stream
     w = synthetic.make(DECODE_APPEND)
@@ -349,38 +602,35 @@ def run_decode_append(gqa, dev, stream, world, K, W):
                                                "wq", "wk")}
     out = torch.empty((B, H, D), dtype=torch.float32, device=dev)
     ws = torch.empty(gqa.decode_workspace_size(B, H, Hkv, w.max_len, D), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     ptr = lambda x: x.data_ptr()  # noqa: E731
 
-    def call():
+    def call(st_):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)] if st_ is not None else None
+        if ev:
+            ev[0].record(st_)
         st = lib.gqa_attn_decode_append(ptr(t["q"]), ptr(t["k_new"]), ptr(t["v_new"]), ptr(t["k_cache"]),
                                         ptr(t["v_cache"]), ptr(t["offsets"]), ptr(t["seqlens"]), None, ptr(t["wq"]),
                                         ptr(t["wk"]), w.theta, w.eps, ptr(out), B, H, Hkv, D, w.max_len, ptr(ws),
                                         ws.numel(), sh)
+        if ev:
+            ev[1].record(st_)
         if st != 0:
             raise RuntimeError(f"gqa_attn_decode_append failed with status {st}")
+        return ev
 
-    for _ in range(W):
-        call()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(K):
-        call()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    sec = timed_calls(call, stream, world, dev, K, W, flush)[0]
     if gqa.device_status() != 0:
         raise RuntimeError("device status error in the append-step timing")
-    sec = max_over_ranks([e0.elapsed_time(e1)], dev, world)[0] / 1e3
     nbytes = decode_append_bytes(w.seqlens.tolist(), H, Hkv, D)
     gbs = nbytes * K / sec / 1e9
-    del t, out, ws
+    del t, out, ws, flush
     return {"value": round(whole_job_rate(nbytes * K, world, sec) / 1e9, 1), "unit": "GB/s",
             "ms": round(1e3 * sec / K, 4),
             "workload": "64 sequences, cached rows U[1023,32767] + 1 appended, H32 Hkv8 D128",
-            "bytes_per_call": nbytes, "gpu_launches": 3 * K,
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s", "traffic": None,
+            "bytes_per_call": nbytes, "gpu_launches": 3 * K, "l2": "256 MB written between timed calls",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s",
+                         "traffic": traffic_from_profiles("decode_split_kernel", DECODE_APPEND),
                          "kernel": "decode_append_kernel + decode_split_kernel + decode_merge_kernel (one call)"}}
 
 
@@ -407,7 +657,7 @@ def paged_layout(lens, offs, page_size, seed=30):
 def run_decode_paged(gqa, dec, dq, kc, vc, sl, dwq, dev, stream, world, K, W, page_size=64):
     """gqa_attn_decode_paged on the batched decode workload, its cache copied on the
     device into pages of page_size rows handed out in a seeded random order; CUDA events
-    around K calls after W warm-up calls."""
+    around each of K calls after W warm-up calls, L2 flushed between calls."""
     lib = gqa.load()
     sh = stream.cuda_stream
     B, H, D = dec.q.shape
@@ -425,36 +675,34 @@ def run_decode_paged(gqa, dec, dq, kc, vc, sl, dwq, dev, stream, world, K, W, pa
     ws = torch.empty(gqa.decode_workspace_size(B, H, Hkv, dec.max_len, D), dtype=torch.uint8, device=dev)
     rope = gqa.RopeConfig.make(theta=dec.theta)
 
-    def call():
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def call(st_):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)] if st_ is not None else None
+        if ev:
+            ev[0].record(st_)
         st = lib.gqa_attn_decode_paged(dq.data_ptr(), kp.data_ptr(), vp.data_ptr(), tab.data_ptr(), num_pages,
                                        page_size, tab.shape[1], sl.data_ptr(), None, dwq.data_ptr(),
                                        ctypes.byref(rope), dec.eps, out.data_ptr(), B, H, Hkv, D, dec.max_len,
                                        ws.data_ptr(), ws.numel(), sh)
+        if ev:
+            ev[1].record(st_)
         if st != 0:
             raise RuntimeError(f"gqa_attn_decode_paged failed with status {st}")
+        return ev
 
-    for _ in range(W):
-        call()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(K):
-        call()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    sec = timed_calls(call, stream, world, dev, K, W, flush)[0]
     if gqa.device_status() != 0:
         raise RuntimeError("device status error in the paged-decode timing")
-    sec = max_over_ranks([e0.elapsed_time(e1)], dev, world)[0] / 1e3
     nbytes = decode_bytes(lens, H, Hkv, D)
     gbs = nbytes * K / sec / 1e9
-    del kp, vp, tab, out, ws
+    del kp, vp, tab, out, ws, flush
     return {"value": round(whole_job_rate(nbytes * K, world, sec) / 1e9, 1), "unit": "GB/s",
             "ms": round(1e3 * sec / K, 4), "page_size": page_size, "num_pages": num_pages,
             "workload": "the batched decode (64 seqs, cache len U[1024,32768], H32 Hkv8 D128) in shuffled pages",
-            "bytes_per_call": nbytes, "gpu_launches": 2 * K,
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s", "traffic": None,
+            "bytes_per_call": nbytes, "gpu_launches": 2 * K, "l2": "256 MB written between timed calls",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s",
+                         "traffic": traffic_from_profiles("decode_split_kernel<paged>", "batched_decode_paged64"),
                          "kernel": "decode_split_kernel (paged) + decode_merge_kernel (one call)"}}
 
 
@@ -577,8 +825,8 @@ def cpu_baseline(pin, dec, budget_s=20.0):
         m = min(len(order), m * 2)
         by, dsec = oracle_decode_sample(dec, np.sort(order[:m]))
     return {"value": round(fl / sec / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"prefill: {n} random output rows (b, head, i) of the large prefill, {sec:.1f} s; "
-                      f"fp64 C, OpenMP",
+            "sample": f"prefill: {n} random output rows (b, head, i) of the {WORKLOAD_TEXT[PREFILL]}, "
+                      f"{sec:.1f} s; fp64 C, OpenMP",
             "decode": {"value": round(by / dsec / 1e9, 4), "unit": "GB/s",
                        "sample": f"decode: the {m} shortest sequences of the batched decode, all heads, {dsec:.1f} s"}}
 
@@ -609,8 +857,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * (sec_t + dsec_t) / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "large prefill (B4 T4096 H32 Hkv8 D128, inputs x0.5, causal) + batched decode "
-                               "(64 seqs, cache len U[1024,32768], H32 Hkv8 D128)",
+        "config": {"workload": f"{WORKLOAD_TEXT[PREFILL]} + {WORKLOAD_TEXT[DECODE]}",
                    "sample_per_step": f"{rows_per_step} prefill output rows + 1 decode sequence (all heads)"},
         "decode": {"value": round(by_t / dsec_t / 1e9, 4), "unit": "GB/s"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",

@@ -26,9 +26,26 @@ EXPORTS = ("gqa_status_string", "gqa_attn_prefill_workspace_size", "gqa_attn_pre
            "gqa_attn_decode", "gqa_attn_decode_append", "gqa_attn_decode_noalloc",
            "gqa_attn_device_status", "gqa_attn_prefill_ex", "gqa_attn_k_norm_rope_ex",
            "gqa_attn_prefill_khat_ex", "gqa_attn_decode_ex", "gqa_attn_decode_append_ex",
-           "gqa_attn_decode_paged", "gqa_attn_decode_append_paged")
+           "gqa_attn_decode_paged", "gqa_attn_decode_append_paged", "gqa_attn_prefill_varlen_workspace_size",
+           "gqa_attn_prefill_varlen", "gqa_attn_prefill_chunk_workspace_size", "gqa_attn_prefill_chunk",
+           "gqa_linear", "gqa_attn_block_prefill_workspace_size", "gqa_attn_block_prefill",
+           "gqa_attn_test_stall")
+
+
+def _header_scratch_bytes() -> int:
+    """GQA_NOALLOC_SCRATCH_BYTES as include/gqa_attn.h defines it (the library is compiled
+    from the same header), so the two cannot drift apart."""
+    import re
+    path = os.path.join(os.path.dirname(_PKG), "include", "gqa_attn.h")
+    with open(path, encoding="utf-8") as f:
+        m = re.search(r"#define\s+GQA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", f.read())
+    if m is None:
+        raise RuntimeError(f"GQA_NOALLOC_SCRATCH_BYTES not found in {path}")
+    return int(m.group(1)) << int(m.group(2))
+
+
 # Size of the library's built-in scratch used by gqa_attn_decode_noalloc.
-NOALLOC_SCRATCH_BYTES = 32 << 20
+NOALLOC_SCRATCH_BYTES = _header_scratch_bytes()
 
 
 class RopeConfig(ctypes.Structure):
@@ -104,8 +121,24 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, P, P, R, F, P, I, I, I, I, I, P, Z, P]
     lib.gqa_attn_decode_append_paged.argtypes = [P, P, P, P, P, P, I, I, I, P, P, P, P, R, F, P, I, I, I, I, I, P, Z,
                                                  P]
+    L = ctypes.c_int64
+    lib.gqa_attn_prefill_varlen_workspace_size.argtypes = [L, I, I]
+    lib.gqa_attn_prefill_varlen_workspace_size.restype = Z
+    lib.gqa_attn_prefill_varlen.argtypes = [P, P, P, P, P, P, P, R, F, P, I, L, I, I, I, I, P, Z, P]
+    lib.gqa_attn_prefill_chunk_workspace_size.argtypes = [L, I]
+    lib.gqa_attn_prefill_chunk_workspace_size.restype = Z
+    lib.gqa_attn_prefill_chunk.argtypes = [P, P, P, P, P, P, P, P, P, L, P, P, R, F, P, I, L, I, I, I, I, P, Z, P]
+    lib.gqa_attn_test_stall.argtypes = [I]
+    lib.gqa_attn_test_stall.restype = None
+    lib.gqa_linear.argtypes = [P, P, P, I, L, I, I, P]
+    lib.gqa_linear.restype = I
+    lib.gqa_attn_block_prefill_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.gqa_attn_block_prefill_workspace_size.restype = Z
+    lib.gqa_attn_block_prefill.argtypes = [P, P, P, P, P, P, R, F, P, I, I, I, I, I, I, P, Z, P]
+    lib.gqa_attn_block_prefill.restype = I
     for n in ("gqa_attn_prefill_ex", "gqa_attn_k_norm_rope_ex", "gqa_attn_prefill_khat_ex", "gqa_attn_decode_ex",
-              "gqa_attn_decode_append_ex", "gqa_attn_decode_paged", "gqa_attn_decode_append_paged"):
+              "gqa_attn_decode_append_ex", "gqa_attn_decode_paged", "gqa_attn_decode_append_paged",
+              "gqa_attn_prefill_varlen", "gqa_attn_prefill_chunk"):
         getattr(lib, n).restype = I
     _lib = lib
     return lib
@@ -242,6 +275,135 @@ def prefill_khat(q, k_hat, v, pos, qnorm_w, theta: float = 1.0e6, eps: float = 1
     st = fn(_ptr(q), _ptr(k_hat), _ptr(v), _ptr(pos), _ptr(rope_cs), _ptr(qnorm_w), th, float(eps), _ptr(out), B,
             T, H, Hkv, D, _stream_handle(stream))
     _raise(st, "gqa_attn_prefill_khat")
+    return out
+
+
+def prefill_varlen(q, k, v, pos, cu_seqlens, qnorm_w, knorm_w, max_seqlen: int, eps: float = 1e-6,
+                   rope: Optional[RopeConfig] = None, out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Packed variable-length causal prefill.  q [N,H,D], k/v [N,Hkv,D] bf16, pos [N]
+    int32, cu_seqlens [B+1] int64 (device) -> out [N,H,D] fp32; each sequence attends
+    causally within itself.  rope defaults to the plain RoPE of base 1e6."""
+    lib = load()
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    _check(pos, "pos", torch.int32, 1)
+    _check(cu_seqlens, "cu_seqlens", torch.int64, 1)
+    _check(qnorm_w, "qnorm_w", torch.float32, 1)
+    _check(knorm_w, "knorm_w", torch.float32, 1)
+    N, H, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if k.shape != (N, Hkv, D) or v.shape != k.shape or pos.shape != (N,) or B < 0:
+        raise ValueError("shape mismatch between q, k, v, pos, cu_seqlens")
+    rope = rope if rope is not None else RopeConfig.make()
+    if out is None:
+        out = torch.empty((N, H, D), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 3)
+    need = int(lib.gqa_attn_prefill_varlen_workspace_size(N, Hkv, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib.gqa_attn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(cu_seqlens), _ptr(qnorm_w),
+                                     _ptr(knorm_w), ctypes.byref(rope), float(eps), _ptr(out), B, N, H, Hkv, D,
+                                     int(max_seqlen), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream_handle(stream))
+    _raise(st, "gqa_attn_prefill_varlen")
+    return out
+
+
+def prefill_chunk(q, k, v, pos, cu_seqlens, k_cache, v_cache, cache_offsets, prefix_len, qnorm_w, knorm_w,
+                  max_chunk_len: int, eps: float = 1e-6, rope: Optional[RopeConfig] = None,
+                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Chunked prefill after a cached prefix: the N chunk tokens (q [N,H,D], k/v
+    [N,Hkv,D] raw, pos [N], packed per cu_seqlens [B+1]) are appended to the cache
+    (k_cache/v_cache [rows,Hkv,D], sequence b at cache_offsets[b] with prefix_len[b] rows
+    cached) and attend to it -> out [N,H,D] fp32."""
+    lib = load()
+    for t, n, dt, d in ((q, "q", torch.bfloat16, 3), (k, "k", torch.bfloat16, 3), (v, "v", torch.bfloat16, 3),
+                        (pos, "pos", torch.int32, 1), (cu_seqlens, "cu_seqlens", torch.int64, 1),
+                        (k_cache, "k_cache", torch.bfloat16, 3), (v_cache, "v_cache", torch.bfloat16, 3),
+                        (cache_offsets, "cache_offsets", torch.int64, 1), (prefix_len, "prefix_len", torch.int32, 1),
+                        (qnorm_w, "qnorm_w", torch.float32, 1), (knorm_w, "knorm_w", torch.float32, 1)):
+        _check(t, n, dt, d)
+    N, H, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if (k.shape != (N, Hkv, D) or v.shape != k.shape or pos.shape != (N,) or k_cache.shape[1:] != (Hkv, D)
+            or v_cache.shape != k_cache.shape or cache_offsets.shape != (B + 1,) or prefix_len.shape != (B,)):
+        raise ValueError("shape mismatch")
+    rope = rope if rope is not None else RopeConfig.make()
+    if out is None:
+        out = torch.empty((N, H, D), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 3)
+    need = int(lib.gqa_attn_prefill_chunk_workspace_size(N, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib.gqa_attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(cu_seqlens), _ptr(k_cache),
+                                    _ptr(v_cache), _ptr(cache_offsets), _ptr(prefix_len), k_cache.shape[0],
+                                    _ptr(qnorm_w), _ptr(knorm_w), ctypes.byref(rope), float(eps), _ptr(out), B, N, H,
+                                    Hkv, D, int(max_chunk_len), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _raise(st, "gqa_attn_prefill_chunk")
+    return out
+
+
+def linear(x, w, out_dtype: torch.dtype = torch.bfloat16, out: Optional[torch.Tensor] = None,
+           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Projection without bias, y = x W^T: x [..., K] bf16, w [N, K] bf16 -> y [..., N]
+    in bf16 or fp32 (fp32 accumulation)."""
+    lib = load()
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() < 1:
+        raise ValueError("x must be a contiguous CUDA bf16 tensor [..., K]")
+    _check(w, "w", torch.bfloat16, 2)
+    N, K = w.shape
+    if x.shape[-1] != K:
+        raise ValueError("x and w disagree on K")
+    M = x.numel() // K if K else 0
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bf16 or fp32")
+    if out is None:
+        out = torch.empty(x.shape[:-1] + (N,), dtype=out_dtype, device=x.device)
+    if out.dtype != out_dtype or not out.is_contiguous() or out.numel() != M * N:
+        raise ValueError("out must be a contiguous tensor of the output shape and dtype")
+    st = lib.gqa_linear(_ptr(x), _ptr(w), _ptr(out), 1 if out_dtype == torch.float32 else 0, M, N, K,
+                        _stream_handle(stream))
+    _raise(st, "gqa_linear")
+    return out
+
+
+def attn_block_prefill(x, w_qkv, w_o, pos, qnorm_w, knorm_w, H: int, Hkv: int, eps: float = 1e-6,
+                       rope: Optional[RopeConfig] = None, out: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None,
+                       stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The attention sub-block for a prefill: x [B,T,hidden] bf16, w_qkv [(H+2Hkv)D,
+    hidden], w_o [hidden, H D] bf16, pos [B,T] -> y [B,T,hidden] fp32 (qkv projection,
+    q/k norm, RoPE, causal GQA attention, output projection)."""
+    lib = load()
+    _check(x, "x", torch.bfloat16, 3)
+    _check(w_qkv, "w_qkv", torch.bfloat16, 2)
+    _check(w_o, "w_o", torch.bfloat16, 2)
+    _check(pos, "pos", torch.int32, 2)
+    _check(qnorm_w, "qnorm_w", torch.float32, 1)
+    _check(knorm_w, "knorm_w", torch.float32, 1)
+    B, T, hidden = x.shape
+    D = qnorm_w.shape[0]
+    if w_qkv.shape != ((H + 2 * Hkv) * D, hidden) or w_o.shape != (hidden, H * D) or pos.shape != (B, T):
+        raise ValueError("shape mismatch between x, w_qkv, w_o, pos")
+    rope = rope if rope is not None else RopeConfig.make()
+    if out is None:
+        out = torch.empty((B, T, hidden), dtype=torch.float32, device=x.device)
+    _check(out, "out", torch.float32, 3)
+    need = int(lib.gqa_attn_block_prefill_workspace_size(B, T, hidden, H, Hkv, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    st = lib.gqa_attn_block_prefill(_ptr(x), _ptr(w_qkv), _ptr(w_o), _ptr(pos), _ptr(qnorm_w), _ptr(knorm_w),
+                                    ctypes.byref(rope), float(eps), _ptr(out), B, T, hidden, H, Hkv, D,
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream_handle(stream))
+    _raise(st, "gqa_attn_block_prefill")
     return out
 
 

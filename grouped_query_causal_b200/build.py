@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libgqa_attn.so")
 SOURCES = ["gqa_attn.cu"]
-DEPS = ["gqa_attn.cu", "prefill.cuh", "decode.cuh", "ptx.cuh", "rope.cuh", "gqa_attn.map"]
+DEPS = ["gqa_attn.cu", "prefill.cuh", "decode.cuh", "gemm.cuh", "ptx.cuh", "rope.cuh", "gqa_attn.map"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -138,32 +138,26 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     const int k1 = min(len, k0 + kChunk);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    __shared__ int s_bad;   // a warp met a page id out of range
+    if (tid == 0) s_bad = 0;
     const int32_t *ptab = PAGED ? p.pages + static_cast<size_t>(b) * p.max_pages : nullptr;
-    if constexpr (PAGED) {
-        // every page this chunk reads must exist; otherwise the chunk reads nothing and
-        // poisons its partial sums so that the merged output of the sequence is NaN
-        bool bad = false;
-        for (int pg = k0 / p.page_size + tid; pg <= (k1 - 1) / p.page_size; pg += 128) {
-            const int id = ptab[pg];
-            bad |= id < 0 || id >= p.num_pages;
-        }
-        if (__syncthreads_or(bad)) {
-            const size_t slot0 = (static_cast<size_t>(b) * p.maxC + c) * p.H + static_cast<size_t>(g) * p.hpg;
-            if (tid < HG && jbase + tid < p.hpg) {
-                p.part_ml[2 * (slot0 + jbase + tid)] = 0.f;
-                p.part_ml[2 * (slot0 + jbase + tid) + 1] = __int_as_float(0x7fc00000);
-            }
-            if (tid == 0) atomicOr(p.err, kErrInput);
-            return;
-        }
-    }
+    const int kw0 = k0 + warp * kWarpKeys;
+    int kw1 = min(k1, kw0 + kWarpKeys);
     // Page ids of this warp's rows (at most 17 pages of >= 16 rows cover its 256 rows),
     // one per lane, so a batch finds its page with a shuffle rather than a dependent load.
-    const int wpg0 = PAGED ? (k0 + warp * kWarpKeys) / p.page_size : 0;
+    // A warp whose pages include an id outside [0, num_pages) reads no rows and poisons the
+    // chunk's partial sums, so that the merged output of the sequence is NaN.
+    const int wpg0 = PAGED ? kw0 / p.page_size : 0;
     int my_page = 0;
+    bool warp_bad = false;
     if constexpr (PAGED) {
-        const int last = (min(k1, k0 + (warp + 1) * kWarpKeys) - 1) / p.page_size;
-        if (wpg0 + lane <= last) my_page = ptab[wpg0 + lane];
+        if (kw0 < kw1) {
+            const int last = (kw1 - 1) / p.page_size;
+            const bool mine = wpg0 + lane <= last;
+            if (mine) my_page = ptab[wpg0 + lane];
+            warp_bad = __any_sync(0xffffffffu, mine && (my_page < 0 || my_page >= p.num_pages));
+            if (warp_bad) kw1 = kw0;
+        }
     }
     // Physical row of the 16-row batch that starts at logical row `base` (16-aligned: a
     // batch never crosses a page, whose size is a multiple of 16).  Warp-uniform.
@@ -176,6 +170,42 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
             return base;
         }
     };
+
+    const int sub = lane & 15;    // elements 8*sub .. 8*sub+7 of a row
+    const int rsel = lane >> 4;   // which row of the pair
+    const int nrow = max(0, kw1 - kw0);
+    float *sw = sbuf[warp];
+    const size_t row_stride = static_cast<size_t>(p.Hkv) * kHeadDim;
+    const uint16_t *kbase = p.kc + (static_cast<size_t>(off) * p.Hkv + g) * kHeadDim + 8 * sub;
+    const uint16_t *vbase = p.vc + (static_cast<size_t>(off) * p.Hkv + g) * kHeadDim + 8 * sub;
+    const bool writer = (lane & ((16 >> LG) - 1)) == 0;
+    const int my_head = decode_head_of_lane<HG>(lane);
+
+    // Loads of the 16-row batch that starts at logical row `base` (rows past kw1 read
+    // as zero).  Contiguous caches index rows directly; paged ones look the page up once
+    // per batch.
+    auto load_batch = [&](const uint16_t *rbase, int base, uint4 (&dst)[kRowPairs]) {
+        if constexpr (PAGED) {
+            if (base >= kw1) return;
+            const long long pr = batch_row(base);
+#pragma unroll
+            for (int u = 0; u < kRowPairs; ++u) {
+                const int row = base + 2 * u + rsel;
+                dst[u] = row < kw1 ? ldg_stream_v4(rbase + static_cast<size_t>(pr + 2 * u + rsel) * row_stride)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < kRowPairs; ++u) {
+                const int row = base + 2 * u + rsel;
+                dst[u] = row < kw1 ? ldg_stream_v4(rbase + static_cast<size_t>(row) * row_stride)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    };
+    // the first batch of keys is in flight while the query is prepared
+    uint4 kn[kRowPairs];
+    load_batch(kbase, kw0, kn);
 
     // ---- q prologue: RMSNorm + RoPE at the query position, scaled into base-2 logits
     {
@@ -205,50 +235,15 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
         }
     }
     __syncthreads();
+    if (warp_bad && lane == 0) s_bad = 1;
 
-    const int sub = lane & 15;    // elements 8*sub .. 8*sub+7 of a row
-    const int rsel = lane >> 4;   // which row of the pair
     float2 qr[HG][4];   // pairs of query elements, for packed two-lane FMAs
 #pragma unroll
     for (int jj = 0; jj < HG; ++jj)
 #pragma unroll
         for (int e = 0; e < 4; ++e) qr[jj][e] = make_float2(sq[jj][8 * sub + 2 * e], sq[jj][8 * sub + 2 * e + 1]);
 
-    const int kw0 = k0 + warp * kWarpKeys;
-    const int kw1 = min(k1, kw0 + kWarpKeys);
-    const int nrow = max(0, kw1 - kw0);
-    float *sw = sbuf[warp];
-    const size_t row_stride = static_cast<size_t>(p.Hkv) * kHeadDim;
-    const uint16_t *kbase = p.kc + (static_cast<size_t>(off) * p.Hkv + g) * kHeadDim + 8 * sub;
-    const uint16_t *vbase = p.vc + (static_cast<size_t>(off) * p.Hkv + g) * kHeadDim + 8 * sub;
-    const bool writer = (lane & ((16 >> LG) - 1)) == 0;
-    const int my_head = decode_head_of_lane<HG>(lane);
-
     // ---- K sweep: base-2 logits of the HG heads for each key of this warp
-    // Loads of the 16-row batch that starts at logical row `base` (rows past kw1 read
-    // as zero).  Contiguous caches index rows directly; paged ones look the page up once
-    // per batch.
-    auto load_batch = [&](const uint16_t *rbase, int base, uint4 (&dst)[kRowPairs]) {
-        if constexpr (PAGED) {
-            if (base >= kw1) return;
-            const long long pr = batch_row(base);
-#pragma unroll
-            for (int u = 0; u < kRowPairs; ++u) {
-                const int row = base + 2 * u + rsel;
-                dst[u] = row < kw1 ? ldg_stream_v4(rbase + static_cast<size_t>(pr + 2 * u + rsel) * row_stride)
-                                   : make_uint4(0u, 0u, 0u, 0u);
-            }
-        } else {
-#pragma unroll
-            for (int u = 0; u < kRowPairs; ++u) {
-                const int row = base + 2 * u + rsel;
-                dst[u] = row < kw1 ? ldg_stream_v4(rbase + static_cast<size_t>(row) * row_stride)
-                                   : make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
-    };
-    uint4 kn[kRowPairs];
-    load_batch(kbase, kw0, kn);
     for (int base = kw0; base < kw1; base += 2 * kRowPairs) {
         uint4 kv[kRowPairs];
 #pragma unroll
@@ -346,6 +341,14 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
 
     // ---- merge the four warps; thread tid owns element d = tid
     const size_t slot0 = (static_cast<size_t>(b) * p.maxC + c) * p.H + static_cast<size_t>(g) * p.hpg;
+    if (PAGED && s_bad) {
+        if (tid < HG && jbase + tid < p.hpg) {
+            p.part_ml[2 * (slot0 + jbase + tid)] = 0.f;
+            p.part_ml[2 * (slot0 + jbase + tid) + 1] = __int_as_float(0x7fc00000);
+        }
+        if (tid == 0) atomicOr(p.err, kErrInput);
+        return;
+    }
 #pragma unroll 1
     for (int jj = 0; jj < HG; ++jj) {
         const int j = jbase + jj;

@@ -15,6 +15,7 @@
 
 #include "gqa_attn.h"
 #include "decode.cuh"
+#include "gemm.cuh"
 #include "prefill.cuh"
 
 namespace gqa {
@@ -25,6 +26,9 @@ __device__ unsigned g_device_error = 0;
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// Failure-path test switch (gqa_attn_test_stall): read at every attention launch.
+std::atomic<int> g_test_stall{0};
 
 int current_device() {
     int dev = -1;
@@ -59,16 +63,17 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 4-D bf16 tensor [d3][d2][d1][d0] (d0 innermost, contiguous), box (64, 1, 128, 1),
-// 128-byte swizzle, zero fill outside the tensor.
-bool make_bf16_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3) {
+// 3-D bf16 tensor [rows][heads][128] (head vectors contiguous, `row_bytes` between rows),
+// box (64, 1, 128): half a head vector of 128 consecutive rows, 128-byte swizzle, zero
+// fill outside the tensor.
+bool make_rows_map(CUtensorMap *m, const void *base, uint64_t heads, uint64_t rows, uint64_t row_bytes) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
-    const cuuint64_t dims[4] = {d0, d1, d2, d3};
-    const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), heads, rows};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2, row_bytes};
+    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -209,17 +214,40 @@ bool params_ok(float theta, float eps) {
 
 bool eps_ok(float eps) { return eps >= 0.f && std::isfinite(eps); }
 
-// Enqueue the k-hat prologue (arguments already validated).
-gqa_status launch_k_norm_rope(const void *k, const int32_t *pos, const float *knorm_w, const RopeSpec &rs,
-                              float eps, void *k_hat, float *rope_cs, long long ntok, int Hkv, cudaStream_t st) {
+// Where the k-hat prologue writes: row n (cu == nullptr), or, per sequence, after the
+// rows already cached (the chunked-prefill append).
+struct KRows {
+    const int64_t *cu = nullptr, *cache_off = nullptr;
+    const int32_t *prefix = nullptr;
+    int B = 0;
+    long long rows = 0;   // rows of the destination buffers
+};
+
+// Enqueue the k-hat prologue (arguments already validated).  k rows are k_stride
+// elements apart; v (optional) is copied beside k-hat into vout.
+gqa_status launch_k_norm_rope(const void *k, long long k_stride, const void *v, long long v_stride, const int32_t *pos,
+                              const float *knorm_w, const RopeSpec &rs, float eps, void *k_hat, void *vout,
+                              float *rope_cs, long long ntok, int Hkv, const KRows &dst, cudaStream_t st) {
+    unsigned *err = device_error_word();
+    if (!err) return GQA_ERR_CUDA;
     KPrologueParams kp;
     kp.k = static_cast<const uint16_t *>(k);
+    kp.v = static_cast<const uint16_t *>(v);
     kp.pos = pos;
     kp.wk = knorm_w;
     kp.khat = static_cast<uint16_t *>(k_hat);
+    kp.vout = static_cast<uint16_t *>(vout);
     kp.rope_cs = rope_cs;
+    kp.cu = dst.cu;
+    kp.cache_off = dst.cache_off;
+    kp.prefix = dst.prefix;
+    kp.err = err;
     kp.ntok = ntok;
+    kp.k_stride = k_stride;
+    kp.v_stride = v_stride;
+    kp.rows = dst.cu ? dst.rows : ntok;
     kp.Hkv = Hkv;
+    kp.B = dst.B;
     kp.eps = eps;
     kp.rf = rs.rf;
     long long blocks = (ntok + 7) / 8;   // one warp per token, 8 warps per block
@@ -232,15 +260,29 @@ gqa_status launch_k_norm_rope(const void *k, const int32_t *pos, const float *kn
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
+// Sequence geometry of an attention launch (AttnParams): dense (arrays null: B
+// sequences of T tokens) or per sequence from device arrays.
+struct AttnGeom {
+    int B = 0, T = 0;                  // T: the dense length, or the longest sequence
+    long long nq_rows = 0, nkv_rows = 0;
+    long long q_row_elems = 0;         // elements between consecutive q rows (H*D unless strided)
+    long long kv_row_elems = 0;        // elements between consecutive k-hat rows
+    long long v_row_elems = 0;         // elements between consecutive v rows (0: as k-hat)
+    bool out_bf16 = false;             // bf16 output (the input of the output projection)
+    const int64_t *cu_q = nullptr, *kv_off = nullptr;
+    const int32_t *prefix = nullptr;
+};
+
 // Enqueue the attention kernel (arguments already validated).
 gqa_status launch_attention(const void *q, const void *k_hat, const void *v, const int32_t *pos,
-                            const float *rope_cs, const float *qnorm_w, const RopeSpec &rs, float eps, float *out,
-                            int B, int T, int H, int Hkv, cudaStream_t st) {
+                            const float *rope_cs, const float *qnorm_w, const RopeSpec &rs, float eps, void *out,
+                            const AttnGeom &gm, int H, int Hkv, cudaStream_t st) {
     unsigned *err = device_error_word();
     if (!err) return GQA_ERR_CUDA;
     CUtensorMap tm_q, tm_k, tm_v;
-    if (!make_bf16_map(&tm_q, q, kHeadDim, H, T, B) || !make_bf16_map(&tm_k, k_hat, kHeadDim, Hkv, T, B) ||
-        !make_bf16_map(&tm_v, v, kHeadDim, Hkv, T, B))
+    if (!make_rows_map(&tm_q, q, H, gm.nq_rows, gm.q_row_elems * 2) ||
+        !make_rows_map(&tm_k, k_hat, Hkv, gm.nkv_rows, gm.kv_row_elems * 2) ||
+        !make_rows_map(&tm_v, v, Hkv, gm.nkv_rows, (gm.v_row_elems ? gm.v_row_elems : gm.kv_row_elems) * 2))
         return GQA_ERR_CUDA;
     if (!attn_smem_attr_set()) return GQA_ERR_CUDA;
     AttnParams ap;
@@ -249,24 +291,43 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
     ap.wq = qnorm_w;
     ap.out = out;
     ap.err = err;
-    ap.B = B;
-    ap.T = T;
+    ap.cu_q = gm.cu_q;
+    ap.kv_off = gm.kv_off;
+    ap.prefix = gm.prefix;
+    ap.nq_rows = gm.nq_rows;
+    ap.nkv_rows = gm.nkv_rows;
+    ap.B = gm.B;
+    ap.T = gm.T;
     ap.H = H;
     ap.Hkv = Hkv;
     ap.hpg = H / Hkv;
-    ap.nqb = (T + kBM - 1) / kBM;
+    ap.nqb = (gm.T + kBM - 1) / kBM;
     ap.npairs = (ap.hpg + 1) / 2;
+    ap.out_bf16 = gm.out_bf16 ? 1 : 0;
+    ap.test_stall = g_test_stall.load(std::memory_order_relaxed);
     ap.eps = eps;
     ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim))) * rs.logit_mult;
     ap.rf = rs.rf;
-    const long long jobs = static_cast<long long>(ap.nqb) * B * Hkv * ap.npairs;
-    if (jobs <= 0 || jobs > 0x7fffffffLL) return GQA_ERR_INVALID_ARG;
+    const long long units = static_cast<long long>(ap.nqb) * gm.B * Hkv * ap.npairs;
+    if (units <= 0) return GQA_OK;
+    if (units > 0x7fffffffLL) return GQA_ERR_INVALID_ARG;
+    ap.nunits = static_cast<int>(units);
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(units, attn_sm_count()));
     if (rs.pairing == kPairHalf)
-        attn_fwd_kernel<kPairHalf><<<static_cast<unsigned>(jobs), kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
+        attn_fwd_kernel<kPairHalf><<<grid, kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
     else
-        attn_fwd_kernel<kPairAdjacent><<<static_cast<unsigned>(jobs), kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v,
-                                                                                                   ap);
+        attn_fwd_kernel<kPairAdjacent><<<grid, kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+AttnGeom dense_geom(int B, int T, int H, int Hkv) {
+    AttnGeom g;
+    g.B = B;
+    g.T = T;
+    g.nq_rows = g.nkv_rows = static_cast<long long>(B) * T;
+    g.q_row_elems = static_cast<long long>(H) * kHeadDim;
+    g.kv_row_elems = static_cast<long long>(Hkv) * kHeadDim;
+    return g;
 }
 
 }  // namespace
@@ -290,7 +351,8 @@ gqa_status k_norm_rope_impl(const void *k, const int32_t *pos, const float *knor
         const size_t tb = round_up(static_cast<size_t>(N), 128) * kHeadDim * sizeof(float);
         if ((c < b + bytes && b < c + tb) || (c < a + bytes && a < c + tb)) return GQA_ERR_INVALID_ARG;
     }
-    return launch_k_norm_rope(k, pos, knorm_w, rs, eps, k_hat, rope_cs, N, Hkv, static_cast<cudaStream_t>(stream));
+    return launch_k_norm_rope(k, static_cast<long long>(Hkv) * kHeadDim, nullptr, 0, pos, knorm_w, rs, eps, k_hat,
+                              nullptr, rope_cs, N, Hkv, KRows{}, static_cast<cudaStream_t>(stream));
 }
 
 gqa_status prefill_khat_impl(const void *q, const void *k_hat, const void *v, const int32_t *pos,
@@ -303,7 +365,7 @@ gqa_status prefill_khat_impl(const void *q, const void *k_hat, const void *v, co
     if (!aligned(q, 16) || !aligned(k_hat, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(qnorm_w, 16) ||
         !aligned(pos, 4) || (rope_cs && !aligned(rope_cs, 16)))
         return GQA_ERR_INVALID_ARG;
-    return launch_attention(q, k_hat, v, pos, rope_cs, qnorm_w, rs, eps, out, B, T, H, Hkv,
+    return launch_attention(q, k_hat, v, pos, rope_cs, qnorm_w, rs, eps, out, dense_geom(B, T, H, Hkv), H, Hkv,
                             static_cast<cudaStream_t>(stream));
 }
 
@@ -322,10 +384,11 @@ gqa_status prefill_impl(const void *q, const void *k, const void *v, const int32
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float *table = reinterpret_cast<float *>(static_cast<char *>(workspace) + khat_bytes(B, T, Hkv));
-    gqa_status s =
-        launch_k_norm_rope(k, pos, knorm_w, rs, eps, workspace, table, static_cast<long long>(B) * T, Hkv, st);
+    gqa_status s = launch_k_norm_rope(k, static_cast<long long>(Hkv) * kHeadDim, nullptr, 0, pos, knorm_w, rs, eps,
+                                      workspace, nullptr, table, static_cast<long long>(B) * T, Hkv, KRows{}, st);
     if (s != GQA_OK) return s;
-    return launch_attention(q, workspace, v, pos, table, qnorm_w, rs, eps, out, B, T, H, Hkv, st);
+    return launch_attention(q, workspace, v, pos, table, qnorm_w, rs, eps, out, dense_geom(B, T, H, Hkv), H, Hkv,
+                            st);
 }
 
 }  // namespace
@@ -381,6 +444,253 @@ extern "C" gqa_status gqa_attn_prefill_ex(const void *q, const void *k, const vo
                         stream);
 }
 
+// ---------------------------------------------------------------- packed and chunked prefill
+namespace {
+
+bool ragged_shape_ok(int B, int64_t N, int H, int Hkv, int max_len) {
+    if (B < 0 || N < 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0 || max_len < 0) return false;
+    if (N > (1LL << 31) - 256 || max_len > (1 << 30)) return false;
+    return true;
+}
+
+}  // namespace
+
+extern "C" size_t gqa_attn_prefill_varlen_workspace_size(int64_t N, int Hkv, int D) {
+    if (D != kHeadDim || N <= 0 || Hkv <= 0 || N > (1LL << 31) - 256) return 0;
+    return khat_bytes(1, static_cast<int>(N), Hkv) + rope_table_bytes(1, static_cast<int>(N));
+}
+
+extern "C" gqa_status gqa_attn_prefill_varlen(const void *q, const void *k, const void *v, const int32_t *pos,
+                                              const int64_t *cu_seqlens, const float *qnorm_w, const float *knorm_w,
+                                              const gqa_rope_config *rope, float eps, float *out, int B, int64_t N,
+                                              int H, int Hkv, int D, int max_seqlen, void *workspace,
+                                              size_t workspace_bytes, void *stream) {
+    RopeSpec rs;
+    if (!rope_spec(rope, rs) || !eps_ok(eps)) return GQA_ERR_INVALID_ARG;
+    if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
+    if (!ragged_shape_ok(B, N, H, Hkv, max_seqlen)) return GQA_ERR_INVALID_ARG;
+    if (B == 0 || N == 0 || max_seqlen == 0) return GQA_OK;
+    if (!q || !k || !v || !pos || !cu_seqlens || !qnorm_w || !knorm_w || !out) return GQA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(qnorm_w, 16) ||
+        !aligned(knorm_w, 16) || !aligned(pos, 4) || !aligned(cu_seqlens, 8))
+        return GQA_ERR_INVALID_ARG;
+    const size_t need = gqa_attn_prefill_varlen_workspace_size(N, Hkv, D);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void *khat = workspace;
+    float *table = reinterpret_cast<float *>(static_cast<char *>(workspace) + khat_bytes(1, static_cast<int>(N), Hkv));
+    gqa_status s = launch_k_norm_rope(k, static_cast<long long>(Hkv) * kHeadDim, nullptr, 0, pos, knorm_w, rs, eps,
+                                      khat, nullptr, table, N, Hkv, KRows{}, st);
+    if (s != GQA_OK) return s;
+    AttnGeom gm;
+    gm.B = B;
+    gm.T = max_seqlen;
+    gm.nq_rows = gm.nkv_rows = N;
+    gm.q_row_elems = static_cast<long long>(H) * kHeadDim;
+    gm.kv_row_elems = static_cast<long long>(Hkv) * kHeadDim;
+    gm.cu_q = cu_seqlens;
+    return launch_attention(q, khat, v, pos, table, qnorm_w, rs, eps, out, gm, H, Hkv, st);
+}
+
+extern "C" size_t gqa_attn_prefill_chunk_workspace_size(int64_t N, int D) {
+    if (D != kHeadDim || N <= 0 || N > (1LL << 31) - 256) return 0;
+    return rope_table_bytes(1, static_cast<int>(N));
+}
+
+extern "C" gqa_status gqa_attn_prefill_chunk(const void *q, const void *k, const void *v, const int32_t *pos,
+                                             const int64_t *cu_seqlens, void *k_cache, void *v_cache,
+                                             const int64_t *cache_offsets, const int32_t *prefix_len,
+                                             int64_t cache_rows, const float *qnorm_w, const float *knorm_w,
+                                             const gqa_rope_config *rope, float eps, float *out, int B, int64_t N,
+                                             int H, int Hkv, int D, int max_chunk_len, void *workspace,
+                                             size_t workspace_bytes, void *stream) {
+    RopeSpec rs;
+    if (!rope_spec(rope, rs) || !eps_ok(eps)) return GQA_ERR_INVALID_ARG;
+    if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
+    if (!ragged_shape_ok(B, N, H, Hkv, max_chunk_len)) return GQA_ERR_INVALID_ARG;
+    if (cache_rows < 0 || cache_rows > (1LL << 31) - 256) return GQA_ERR_INVALID_ARG;
+    if (B == 0 || N == 0 || max_chunk_len == 0) return GQA_OK;
+    if (!q || !k || !v || !pos || !cu_seqlens || !k_cache || !v_cache || !cache_offsets || !prefix_len ||
+        !qnorm_w || !knorm_w || !out || cache_rows == 0)
+        return GQA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(qnorm_w, 16) ||
+        !aligned(knorm_w, 16) || !aligned(pos, 4) || !aligned(cu_seqlens, 8) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16) || !aligned(cache_offsets, 8) || !aligned(prefix_len, 4))
+        return GQA_ERR_INVALID_ARG;
+    const size_t need = gqa_attn_prefill_chunk_workspace_size(N, D);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *table = static_cast<float *>(workspace);
+    // the chunk's k-hat and v go into the cache after each sequence's cached rows ...
+    KRows dst;
+    dst.cu = cu_seqlens;
+    dst.cache_off = cache_offsets;
+    dst.prefix = prefix_len;
+    dst.B = B;
+    dst.rows = cache_rows;
+    const long long kv = static_cast<long long>(Hkv) * kHeadDim;
+    gqa_status s = launch_k_norm_rope(k, kv, v, kv, pos, knorm_w, rs, eps, k_cache, v_cache, table, N, Hkv, dst, st);
+    if (s != GQA_OK) return s;
+    // ... and the chunk's queries attend to all of them
+    AttnGeom gm;
+    gm.B = B;
+    gm.T = max_chunk_len;
+    gm.nq_rows = N;
+    gm.nkv_rows = cache_rows;
+    gm.q_row_elems = static_cast<long long>(H) * kHeadDim;
+    gm.kv_row_elems = kv;
+    gm.cu_q = cu_seqlens;
+    gm.kv_off = cache_offsets;
+    gm.prefix = prefix_len;
+    return launch_attention(q, k_cache, v_cache, pos, table, qnorm_w, rs, eps, out, gm, H, Hkv, st);
+}
+
+// ---------------------------------------------------------------- projections
+namespace {
+
+// 2-D bf16 matrix [rows][cols] (row stride ld elements), box (64 cols, box_rows rows),
+// 128-byte swizzle, zero fill outside.
+bool make_matrix_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool gemm_smem_attr_set() {
+    static std::atomic<int> done[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0) return false;
+    if (done[dev].load()) return true;
+    if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kGemmSmemBytes)) != cudaSuccess)
+        return false;
+    done[dev].store(1);
+    return true;
+}
+
+// y[M, N] = x[M, K] w[N, K]^T (arguments validated): x rows ldx elements apart, y rows ldy.
+gqa_status launch_gemm(const void *x, long long ldx, const void *w, void *y, long long ldy, bool y_fp32, int M, int N,
+                       int K, cudaStream_t st) {
+    unsigned *err = device_error_word();
+    if (!err) return GQA_ERR_CUDA;
+    CUtensorMap tm_x, tm_w;
+    if (!make_matrix_map(&tm_x, x, M, K, ldx, kGemmBM) || !make_matrix_map(&tm_w, w, N, K, K, kGemmBN))
+        return GQA_ERR_CUDA;
+    if (!gemm_smem_attr_set()) return GQA_ERR_CUDA;
+    GemmParams gp;
+    gp.y = y;
+    gp.err = err;
+    gp.M = M;
+    gp.N = N;
+    gp.K = K;
+    gp.ldy = ldy;
+    gp.y_fp32 = y_fp32 ? 1 : 0;
+    gp.mblocks = (M + kGemmBM - 1) / kGemmBM;
+    gp.nblocks = (N + kGemmBN - 1) / kGemmBN;
+    const long long tiles = static_cast<long long>(gp.mblocks) * gp.nblocks;
+    if (tiles <= 0) return GQA_OK;
+    if (tiles > 0x7fffffffLL) return GQA_ERR_INVALID_ARG;
+    gp.ntiles = static_cast<int>(tiles);
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(tiles, attn_sm_count()));
+    gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_x, tm_w, gp);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+bool linear_shape_ok(long long M, long long N, long long K) {
+    return M >= 0 && N > 0 && K > 0 && N % 32 == 0 && K % 8 == 0 && M < (1LL << 31) && N < (1LL << 24) &&
+           K < (1LL << 24);
+}
+
+}  // namespace
+
+extern "C" gqa_status gqa_linear(const void *x, const void *w, void *y, int y_dtype, int64_t M, int N, int K,
+                                 void *stream) {
+    if (y_dtype != GQA_DTYPE_BF16 && y_dtype != GQA_DTYPE_F32) return GQA_ERR_INVALID_ARG;
+    if (!linear_shape_ok(M, N, K)) return GQA_ERR_INVALID_ARG;
+    if (M == 0) return GQA_OK;
+    if (!x || !w || !y || !aligned(x, 16) || !aligned(w, 16) || !aligned(y, 16)) return GQA_ERR_INVALID_ARG;
+    return launch_gemm(x, K, w, y, N, y_dtype == GQA_DTYPE_F32, static_cast<int>(M), N, K,
+                       static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------- the whole attention sub-block
+namespace {
+
+struct BlockLayout {
+    size_t qkv, khat, table, o, total;
+};
+
+bool block_layout(int B, int T, int H, int Hkv, BlockLayout &l) {
+    if (!prefill_shape_ok(B, T, H, Hkv) || B == 0 || T == 0) return false;
+    const size_t n = static_cast<size_t>(B) * T;
+    l.qkv = 0;
+    l.khat = round_up(n * (H + 2 * Hkv) * kHeadDim * 2, 256);
+    l.table = l.khat + khat_bytes(B, T, Hkv);
+    l.o = l.table + rope_table_bytes(B, T);
+    l.total = l.o + round_up(n * H * kHeadDim * 2, 256);
+    return true;
+}
+
+}  // namespace
+
+extern "C" size_t gqa_attn_block_prefill_workspace_size(int B, int T, int hidden, int H, int Hkv, int D) {
+    BlockLayout l;
+    if (D != kHeadDim || hidden <= 0 || !block_layout(B, T, H, Hkv, l)) return 0;
+    return l.total;
+}
+
+extern "C" gqa_status gqa_attn_block_prefill(const void *x, const void *w_qkv, const void *w_o, const int32_t *pos,
+                                             const float *qnorm_w, const float *knorm_w, const gqa_rope_config *rope,
+                                             float eps, float *y, int B, int T, int hidden, int H, int Hkv, int D,
+                                             void *workspace, size_t workspace_bytes, void *stream) {
+    RopeSpec rs;
+    if (!rope_spec(rope, rs) || !eps_ok(eps)) return GQA_ERR_INVALID_ARG;
+    if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
+    if (!prefill_shape_ok(B, T, H, Hkv)) return GQA_ERR_INVALID_ARG;
+    const long long n = static_cast<long long>(B) * T;
+    const int nqkv = (H + 2 * Hkv) * kHeadDim;
+    if (hidden <= 0 || !linear_shape_ok(n, nqkv, hidden) || !linear_shape_ok(n, hidden, H * kHeadDim))
+        return GQA_ERR_INVALID_ARG;
+    if (n == 0) return GQA_OK;
+    if (!x || !w_qkv || !w_o || !pos || !qnorm_w || !knorm_w || !y) return GQA_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_qkv, 16) || !aligned(w_o, 16) || !aligned(y, 16) || !aligned(qnorm_w, 16) ||
+        !aligned(knorm_w, 16) || !aligned(pos, 4))
+        return GQA_ERR_INVALID_ARG;
+    BlockLayout l;
+    if (!block_layout(B, T, H, Hkv, l)) return GQA_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < l.total) return GQA_ERR_WORKSPACE;
+    char *ws = static_cast<char *>(workspace);
+    uint16_t *qkv = reinterpret_cast<uint16_t *>(ws + l.qkv);
+    void *khat = ws + l.khat;
+    float *table = reinterpret_cast<float *>(ws + l.table);
+    void *o = ws + l.o;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // (1) qkv = x W_qkv^T, bf16 [n, H + 2 Hkv, D]: q, k, v of a token side by side
+    gqa_status s = launch_gemm(x, hidden, w_qkv, qkv, nqkv, false, static_cast<int>(n), nqkv, hidden, st);
+    if (s != GQA_OK) return s;
+    // (2) k-hat from the k section, read in place
+    s = launch_k_norm_rope(qkv + static_cast<size_t>(H) * kHeadDim, nqkv, nullptr, 0, pos, knorm_w, rs, eps, khat,
+                           nullptr, table, n, Hkv, KRows{}, st);
+    if (s != GQA_OK) return s;
+    // (3) attention on the q and v sections in place, bf16 output [n, H, D]
+    AttnGeom gm = dense_geom(B, T, H, Hkv);
+    gm.q_row_elems = nqkv;
+    gm.v_row_elems = nqkv;
+    gm.out_bf16 = true;
+    s = launch_attention(qkv, khat, qkv + static_cast<size_t>(H + Hkv) * kHeadDim, pos, table, qnorm_w, rs, eps, o, gm,
+                         H, Hkv, st);
+    if (s != GQA_OK) return s;
+    // (4) y = o W_o^T over the concatenated heads, fp32 [n, hidden]
+    return launch_gemm(o, static_cast<long long>(H) * kHeadDim, w_o, y, hidden, true, static_cast<int>(n), hidden,
+                       H * kHeadDim, st);
+}
+
 extern "C" size_t gqa_attn_decode_workspace_size(int B, int H, int Hkv, int D, int max_len) {
     if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0 || D != kHeadDim || max_len <= 0) return 0;
     const size_t slots = decode_slots(B, H, max_len);
@@ -413,16 +723,21 @@ struct PagedCache {
     int num_pages, page_size, max_pages;
 };
 
-gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
-                       const int64_t *cache_offsets, const PagedCache *paged, const int32_t *seqlens,
-                       const int32_t *q_pos,
-                       const float *qnorm_w, const float *knorm_w, const RopeSpec &rs, float eps, float *out, int B,
-                       int H, int Hkv, int D, int max_len, void *workspace, size_t workspace_bytes, void *stream) {
+// Host-side argument checks of the decode entry points, everything except the
+// workspace.  Sets `empty` for B == 0 (a no-op).
+gqa_status decode_check(const void *q, const void *k_new, const void *v_new, const void *k_cache,
+                        const void *v_cache, const int64_t *cache_offsets, const PagedCache *paged,
+                        const int32_t *seqlens, const int32_t *q_pos, const float *qnorm_w, const float *knorm_w,
+                        float eps, const float *out, int B, int H, int Hkv, int D, int max_len, bool &empty) {
+    empty = false;
     const bool append = k_new != nullptr || v_new != nullptr || knorm_w != nullptr;
     if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
     if (B < 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0) return GQA_ERR_INVALID_ARG;
     if (!eps_ok(eps)) return GQA_ERR_INVALID_ARG;
-    if (B == 0) return GQA_OK;
+    if (B == 0) {
+        empty = true;
+        return GQA_OK;
+    }
     if (max_len <= 0) return GQA_ERR_INVALID_ARG;
     if ((static_cast<long long>(max_len) + kChunk - 1) / kChunk > 65535) return GQA_ERR_INVALID_ARG;
     if (static_cast<long long>(B) * Hkv > 0x7fffffffLL || static_cast<long long>(B) * H > 0x7fffffffLL)
@@ -441,6 +756,19 @@ gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void
         return GQA_ERR_INVALID_ARG;
     if (append && (!k_new || !v_new || !knorm_w || !aligned(k_new, 8) || !aligned(v_new, 8) || !aligned(knorm_w, 16)))
         return GQA_ERR_INVALID_ARG;
+    return GQA_OK;
+}
+
+gqa_status decode_impl(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                       const int64_t *cache_offsets, const PagedCache *paged, const int32_t *seqlens,
+                       const int32_t *q_pos,
+                       const float *qnorm_w, const float *knorm_w, const RopeSpec &rs, float eps, float *out, int B,
+                       int H, int Hkv, int D, int max_len, void *workspace, size_t workspace_bytes, void *stream) {
+    const bool append = k_new != nullptr || v_new != nullptr || knorm_w != nullptr;
+    bool empty = false;
+    const gqa_status chk = decode_check(q, k_new, v_new, k_cache, v_cache, cache_offsets, paged, seqlens, q_pos,
+                                        qnorm_w, knorm_w, eps, out, B, H, Hkv, D, max_len, empty);
+    if (chk != GQA_OK || empty) return chk;
     const size_t need = gqa_attn_decode_workspace_size(B, H, Hkv, D, max_len);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
     unsigned *err = device_error_word();
@@ -613,19 +941,21 @@ extern "C" gqa_status gqa_attn_decode_noalloc(const void *q, const void *k_cache
                                               const int32_t *q_pos, const float *qnorm_w, float theta, float eps,
                                               float *out, int B, int H, int Hkv, int D, int max_len,
                                               void *stream) {
-    if (D == kHeadDim && B > 0 && H > 0 && Hkv > 0 && H % Hkv == 0 && max_len > 0 &&
-        gqa_attn_decode_workspace_size(B, H, Hkv, D, max_len) > GQA_NOALLOC_SCRATCH_BYTES)
-        return GQA_ERR_WORKSPACE;
-    // Every other argument check is gqa_attn_decode's; the scratch address is only
-    // looked up when there is work to launch.
-    if (D != kHeadDim || B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0 || max_len <= 0)
-        return gqa_attn_decode(q, k_cache, v_cache, cache_offsets, seqlens, q_pos, qnorm_w, theta, eps, out, B, H,
-                               Hkv, D, max_len, nullptr, 0, stream);
+    // gqa_attn_decode's argument checks first, then the size limit of the built-in
+    // scratch; its device address is only looked up when there is work to launch.
+    if (!params_ok(theta, eps)) return GQA_ERR_INVALID_ARG;
+    bool empty = false;
+    const gqa_status chk = decode_check(q, nullptr, nullptr, k_cache, v_cache, cache_offsets, nullptr, seqlens, q_pos,
+                                        qnorm_w, nullptr, eps, out, B, H, Hkv, D, max_len, empty);
+    if (chk != GQA_OK || empty) return chk;
+    if (gqa_attn_decode_workspace_size(B, H, Hkv, D, max_len) > GQA_NOALLOC_SCRATCH_BYTES) return GQA_ERR_WORKSPACE;
     void *scratch = noalloc_scratch_address();
     if (!scratch) return GQA_ERR_CUDA;
     return gqa_attn_decode(q, k_cache, v_cache, cache_offsets, seqlens, q_pos, qnorm_w, theta, eps, out, B, H, Hkv,
                            D, max_len, scratch, GQA_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+extern "C" void gqa_attn_test_stall(int enable) { g_test_stall.store(enable ? 1 : 0, std::memory_order_relaxed); }
 
 extern "C" gqa_status gqa_attn_device_status(void *stream) {
     unsigned *err = device_error_word();

@@ -40,16 +40,43 @@ __host__ __device__ __forceinline__ size_t rope_table_index(long long n, int i2)
 }
 
 struct KPrologueParams {
-    const uint16_t *k;     // bf16 [ntok, Hkv, D]
+    const uint16_t *k;     // bf16: the Hkv head vectors of token n start at k + n * k_stride
+    const uint16_t *v;     // bf16 values copied beside k-hat (v + n * v_stride), or nullptr
     const int32_t *pos;    // [ntok]
     const float *wk;       // [D]
-    uint16_t *khat;        // bf16 [ntok, Hkv, D]
+    uint16_t *khat;        // bf16 [rows, Hkv, D]: token n goes to row dst_row(n)
+    uint16_t *vout;        // bf16 [rows, Hkv, D] (with v), or nullptr
     float *rope_cs;        // RoPE cos/sin of every token in the blocked table layout (rope_table_index), or nullptr
-    long long ntok;
-    int Hkv;
+    // Destination rows.  cu == nullptr: token n -> row n.  Otherwise token n of sequence b
+    // (cu[b] <= n < cu[b+1]) -> row cache_off[b] + prefix[b] + n - cu[b], which must lie
+    // inside the sequence's rows cache_off[b] .. cache_off[b+1] - 1 (else the token is not
+    // written and the device status records an input error).
+    const int64_t *cu;        // [B + 1]
+    const int64_t *cache_off; // [B + 1]
+    const int32_t *prefix;    // [B]
+    unsigned *err;
+    long long ntok, k_stride, v_stride, rows;
+    int Hkv, B;
     float eps;
     RopeFreqs rf;
 };
+
+// Destination row of token n, or -1 if the sequence geometry puts it out of range.
+__device__ __forceinline__ long long k_prologue_row(const KPrologueParams &p, long long n) {
+    if (p.cu == nullptr) return n;
+    int lo = 0, hi = p.B;   // largest b with cu[b] <= n
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (p.cu[mid] <= n) lo = mid;
+        else hi = mid;
+    }
+    const long long c0 = p.cu[lo], c1 = p.cu[lo + 1];
+    const long long r0 = p.cache_off[lo], r1 = p.cache_off[lo + 1];
+    const long long pre = p.prefix[lo];
+    const long long row = r0 + pre + (n - c0);
+    if (!(c0 <= n && n < c1 && pre >= 0 && r0 >= 0 && row < r1 && r1 <= p.rows)) return -1;
+    return row;
+}
 
 // One warp per token at a time; each half-warp transforms one head vector, each lane
 // eight consecutive elements.  Adjacent pairing: the lane's elements are four RoPE pairs.
@@ -76,6 +103,11 @@ __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__
     const int f0 = half_pairs ? 8 * (sub & 7) + 4 * (sub >> 3) : 4 * sub;
 
     for (; tok < p.ntok; tok += nwarps) {
+        const long long drow = k_prologue_row(p, tok);
+        if (drow < 0) {
+            if (lane == 0) atomicOr(p.err, kErrInput);
+            continue;
+        }
         const int ps = p.pos[tok];
         float cs[8], sn[8];
 #pragma unroll
@@ -117,7 +149,8 @@ __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__
                 const int hh = h0 + 2 * u + half;
                 raw[u] = make_uint4(0u, 0u, 0u, 0u);
                 if (hh < p.Hkv)
-                    raw[u] = *reinterpret_cast<const uint4 *>(p.k + (static_cast<size_t>(tok) * p.Hkv + hh) * kHeadDim + 8 * sub);
+                    raw[u] = *reinterpret_cast<const uint4 *>(p.k + static_cast<size_t>(tok) * p.k_stride +
+                                                              static_cast<size_t>(hh) * kHeadDim + 8 * sub);
             }
 #pragma unroll
             for (int u = 0; u < kPairs; ++u) {
@@ -157,9 +190,15 @@ __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__
                     for (int i = 0; i < 4; ++i) outw[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
                 }
                 if (hh < p.Hkv)
-                    *reinterpret_cast<uint4 *>(p.khat + (static_cast<size_t>(tok) * p.Hkv + hh) * kHeadDim + 8 * sub) =
+                    *reinterpret_cast<uint4 *>(p.khat + (static_cast<size_t>(drow) * p.Hkv + hh) * kHeadDim + 8 * sub) =
                         make_uint4(outw[0], outw[1], outw[2], outw[3]);
             }
+        }
+        if (p.v != nullptr) {   // the token's values go beside its keys
+            for (int hh = half; hh < p.Hkv; hh += 2)
+                *reinterpret_cast<uint4 *>(p.vout + (static_cast<size_t>(drow) * p.Hkv + hh) * kHeadDim + 8 * sub) =
+                    *reinterpret_cast<const uint4 *>(p.v + static_cast<size_t>(tok) * p.v_stride +
+                                                     static_cast<size_t>(hh) * kHeadDim + 8 * sub);
         }
     }
 }
@@ -176,14 +215,17 @@ constexpr uint32_t kOffBar = kOffKV + kStages * kTileBytes;
 enum {
     BAR_Q_FULL = 0,    // [2] TMA -> softmax WG: raw Q tile landed
     BAR_Q_READY = 2,   // [2] softmax WG -> MMA: Q tile normed + rotated in place (128 arrivals)
-    BAR_KV_FULL = 4,   // [kStages] TMA -> MMA (only K_0, in slot 0, uses it)
-    BAR_KV_EMPTY = 4 + kStages,      // [kStages] MMA (commit) -> TMA
-    BAR_S_FULL = 4 + 2 * kStages,    // [2] MMA (commit) -> softmax WG: S of the next tile is in TMEM
-    BAR_P_FULL = 6 + 2 * kStages,    // [2] softmax WG -> MMA: P written over S in TMEM, O rescaled (128 arrivals)
-    BAR_O_FULL = 8 + 2 * kStages,    // [2] MMA (commit) -> softmax WG: last P V finished
-    BAR_DRAIN = 10 + 2 * kStages,    // MMA drains its own work before TMEM is released
-    BAR_STEP_FULL = 11 + 2 * kStages,  // [3] TMA -> MMA: V_j and K_{j+1} landed (one wait per tile)
-    NUM_BARS = 14 + 2 * kStages
+    BAR_Q_EMPTY = 4,   // [2] MMA (commit) -> TMA: the unit's last Q K^T on the slot finished
+    BAR_K0_FULL = 6,   // TMA -> MMA: the first K tile of a unit landed
+    BAR_KV_EMPTY = 7,                // [kStages] MMA (commit) -> TMA
+    BAR_S_FULL = 7 + kStages,        // [2] MMA (commit) -> softmax WG: S of the next tile is in TMEM
+    BAR_P_FULL = 9 + kStages,        // [2] softmax WG -> MMA: P written over S in TMEM, O rescaled (128 arrivals)
+    BAR_O_FULL = 11 + kStages,       // [2] MMA (commit) -> softmax WG: the unit's last P V finished
+    BAR_O_EMPTY = 13 + kStages,      // [2] softmax WG -> MMA: O read out by the epilogue (128 arrivals)
+    BAR_DRAIN = 15 + kStages,        // MMA drains its own work before TMEM is released
+    BAR_STEP_FULL = 16 + kStages,    // [3] TMA -> MMA: V_j and K_{j+1} landed (one wait per tile)
+    BAR_NEVER = 19 + kStages,        // never signalled: the failure-path test waits on it
+    NUM_BARS = 20 + kStages
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + NUM_BARS * 8;
 constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align the base to 1024
@@ -192,18 +234,80 @@ constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align t
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAttnThreads = 384;     // warp 0 TMA, warp 1 MMA, warps 4-7 / 8-11 softmax
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+// Registers per thread: launched at kRegsLaunch (384 threads x 168 = 64512 of the SM's
+// 65536), then warpgroup 0 (TMA, MMA and two idle warps) gives up registers to the two
+// softmax warpgroups, whose 128-column score rows need them.
+constexpr uint32_t kRegsLaunch = 168, kRegsCtl = 120, kRegsSoftmax = 192;
+static_assert(kRegsCtl * 128 + 2 * kRegsSoftmax * 128 <= kRegsLaunch * kAttnThreads, "register split");
 
+// Geometry of a prefill launch.  Sequence b has len(b) query tokens, rows q0(b) ..
+// q0(b) + len(b) - 1 of q / pos / out, and prefix(b) + len(b) keys, rows kv0(b) .. of
+// k-hat / v, the first prefix(b) of them cached before these queries.  Query row t of
+// the sequence is token prefix(b) + t and sees keys 0 .. prefix(b) + t (causal on the
+// token index).  Dense prefill: q0 = kv0 = b T, len = T, prefix = 0 (no arrays).
 struct AttnParams {
-    const int32_t *pos;    // [B, T]
-    const float *rope_cs;  // RoPE cos/sin table over the B*T tokens (rope_table_index), or nullptr (evaluate here)
+    const int32_t *pos;    // [Nq]
+    const float *rope_cs;  // RoPE cos/sin table over the Nq query tokens (rope_table_index), or nullptr (evaluate here)
     const float *wq;       // [D]
-    float *out;            // fp32 [B, T, H, D]
+    void *out;             // [Nq, H, D], fp32 or (out_bf16) bf16
     unsigned *err;
-    int B, T, H, Hkv, hpg, nqb, npairs;
+    const int64_t *cu_q;   // [B + 1] query-row offsets, or nullptr: b T
+    const int64_t *kv_off; // [B] first K/V row, or nullptr: the query-row offset
+    const int32_t *prefix; // [B] cached keys before the first query token, or nullptr: 0
+    long long nq_rows;     // rows of q / pos / out
+    long long nkv_rows;    // rows of k-hat / v
+    int B, T, H, Hkv, hpg, nqb, npairs, nunits;
+    int out_bf16;          // 1: the output is rounded to bf16 (the input of the output projection)
+    int test_stall;        // 1 (failure-path test only): the MMA thread first waits on BAR_NEVER
     float eps;
     float scale_log2;      // log2(e) / sqrt(D) times the RoPE variant's logit factor: softmax runs in base 2
     RopeFreqs rf;
 };
+
+// One work unit: a 128-row query block of one sequence and a pair of query heads of a
+// KV group.  Units are numbered heaviest (latest query block) first.
+struct AttnUnit {
+    long long q0;     // query row of block row 0 (q0(b) + qb * 128)
+    long long kv0;    // K/V row of key 0
+    int b, g, hq0, nslots;
+    int rows;         // valid rows of the block (<= 128)
+    int key0;         // token index of block row 0 (prefix + qb * 128)
+    int n_kv;         // K/V tiles the block reads: keys 0 .. key0 + rows - 1
+};
+
+// Decode unit u; false when it has no work (a query block past the end of a shorter
+// sequence, or a sequence whose device-side geometry is out of range).
+__device__ __forceinline__ bool attn_unit(const AttnParams &p, int u, AttnUnit &w, bool &bad) {
+    bad = false;
+    const int per_qb = p.B * p.Hkv * p.npairs;
+    const int qb = p.nqb - 1 - u / per_qb;
+    int rem = u % per_qb;
+    const int pair = rem % p.npairs;
+    rem /= p.npairs;
+    w.g = rem % p.Hkv;
+    w.b = rem / p.Hkv;
+    long long q0 = static_cast<long long>(w.b) * p.T, len = p.T;
+    if (p.cu_q != nullptr) {
+        q0 = p.cu_q[w.b];
+        len = p.cu_q[w.b + 1] - q0;
+    }
+    const long long kv0 = p.kv_off != nullptr ? p.kv_off[w.b] : q0;
+    const long long pre = p.prefix != nullptr ? p.prefix[w.b] : 0;
+    if (q0 < 0 || len < 0 || q0 + len > p.nq_rows || len > static_cast<long long>(p.nqb) * kBM || pre < 0 ||
+        kv0 < 0 || kv0 + pre + len > p.nkv_rows || pre + len > 0x7fff0000LL) {
+        bad = true;
+        return false;
+    }
+    if (static_cast<long long>(qb) * kBM >= len) return false;
+    w.q0 = q0 + static_cast<long long>(qb) * kBM;
+    w.kv0 = kv0;
+    w.rows = static_cast<int>(min(static_cast<long long>(kBM), len - static_cast<long long>(qb) * kBM));
+    w.key0 = static_cast<int>(pre) + qb * kBM;
+    w.n_kv = (w.key0 + w.rows - 1) / kBN + 1;
+    w.nslots = min(2, p.hpg - 2 * pair);
+    w.hq0 = w.g * p.hpg + 2 * pair;
+    return true;
+}
 
 // Shared-memory address of 16-byte chunk c (0..15, i.e. elements 8c..8c+7) of row r of
 // a 128x128 bf16 tile stored as two 128B-swizzled boxes of 64 columns.
@@ -340,19 +444,75 @@ __device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, cons
     }
 }
 
+// Exponentials per score tile: of every 4 pairs of scores, the first kExpPolyPairs are
+// evaluated on the FMA pipes (exp2_poly2) and the rest by the MUFU ex2 instruction, so
+// that the two pipes share the work (the MUFU rate alone, 16 per clock per SM, equals the
+// tensor cores' rate of keys at D = 128).
+constexpr int kExpPolyPairs = 0;
+
+// 2^x for a pair of scores on the FMA pipes, after the Cody-Waite range reduction
+// x = j + f with j = rint(x) (adding and subtracting 1.5 * 2^23), |f| <= 1/2, and a
+// degree-3 polynomial for 2^f fitted here for least maximum relative error on [-1/2, 1/2]
+// (7.5e-5, far below the 2^-9 of the bf16 the result is rounded to); 2^j goes into the
+// exponent field by an integer add.  x is clamped to -125 (2^-125 rounds to a harmless
+// 2.4e-38), so tiles with masked (-inf) scores use ex2 instead.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+    const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
+    const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+    float2 p = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.24261114f, 0.24261114f));
+    p = __ffma2_rn(p, f, make_float2(0.693260968f, 0.693260968f));
+    p = __ffma2_rn(p, f, make_float2(0.999928057f, 0.999928057f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // 2^(x*scale + negm) of 64 consecutive scores, packed as bf16 pairs into 32 words; their
-// (unrounded) sum goes into eight partial sums.
+// (unrounded) sum goes into eight partial sums.  NPOLY: pairs out of every 4 evaluated on
+// the FMA pipes.
+template <int NPOLY>
 __device__ __forceinline__ void exp_pack64(const float *x, float scale, float negm, uint32_t *pk, float (&sp)[8]) {
+    const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(negm, negm);
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
-        const float e0 = ex2_approx(fmaf(x[2 * c], scale, negm));
-        const float e1 = ex2_approx(fmaf(x[2 * c + 1], scale, negm));
+        float e0, e1;
+        if ((c & 3) < NPOLY) {
+            const float2 e = exp2_poly2(__ffma2_rn(make_float2(x[2 * c], x[2 * c + 1]), sc2, nm2));
+            e0 = e.x;
+            e1 = e.y;
+        } else {
+            e0 = ex2_approx(fmaf(x[2 * c], scale, negm));
+            e1 = ex2_approx(fmaf(x[2 * c + 1], scale, negm));
+        }
         sp[(2 * c) & 7] += e0;
         sp[(2 * c + 1) & 7] += e1;
         pk[c] = pack_bf16x2(e0, e1);
     }
 }
 
+// P of a 128-key tile into TMEM (over S): keys 0-63, then 64-127.
+template <int NPOLY>
+__device__ __forceinline__ void exp_tile(const float *x, float scale, float negm, uint32_t tS, float (&sp)[8]) {
+    {
+        uint32_t pk[32];
+        exp_pack64<NPOLY>(x, scale, negm, pk, sp);
+        tmem_st32(tS, reinterpret_cast<const float *>(pk));
+    }
+    {
+        uint32_t pk[32];
+        exp_pack64<NPOLY>(x + 64, scale, negm, pk, sp);
+        tmem_st32(tS + 32, reinterpret_cast<const float *>(pk));
+    }
+}
+
+// Persistent flash-style causal GQA attention: one CTA per SM walks the work units
+// blockIdx.x, blockIdx.x + gridDim.x, ... (heaviest first).  The K/V ring, the barrier
+// phases and the TMEM buffers carry over from unit to unit, so that the next unit's Q
+// and first K/V tiles load, and its Q tile is normed and rotated, while the current
+// unit's last P V and epilogue run.
 template <int PAIRING>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -367,20 +527,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int warp = tid >> 5;
     const int lane = tid & 31;
 
-    // ---- work unit: heaviest (latest) query blocks are scheduled first
-    const int per_qb = p.B * p.Hkv * p.npairs;
-    const int job = blockIdx.x;
-    const int qb = p.nqb - 1 - job / per_qb;
-    int rem = job % per_qb;
-    const int pair = rem % p.npairs;
-    rem /= p.npairs;
-    const int g = rem % p.Hkv;
-    const int b = rem / p.Hkv;
-    const int j0 = 2 * pair;
-    const int nslots = min(2, p.hpg - j0);
-    const int hq0 = g * p.hpg + j0;
-    const int n_kv = qb + 1;  // causal: K/V tiles 0 .. qb
-
     const uint32_t sQ0 = sbase + kOffQ, sKV0 = sbase + kOffKV;
     const uint32_t bar0 = sbase + kOffBar;
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
@@ -389,18 +535,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(BAR(BAR_Q_FULL + s), 1);
             mbar_init(BAR(BAR_Q_READY + s), kBM);
+            mbar_init(BAR(BAR_Q_EMPTY + s), 1);
             mbar_init(BAR(BAR_S_FULL + s), 1);
             mbar_init(BAR(BAR_P_FULL + s), kBM);
             mbar_init(BAR(BAR_O_FULL + s), 1);
+            mbar_init(BAR(BAR_O_EMPTY + s), kBM);
         }
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(BAR(BAR_KV_FULL + i), 1);
-            mbar_init(BAR(BAR_KV_EMPTY + i), 1);
-        }
-        for (int i = 0; i < 3; ++i) {
-            mbar_init(BAR(BAR_STEP_FULL + i), 1);
-        }
+        mbar_init(BAR(BAR_K0_FULL), 1);
+        for (int i = 0; i < kStages; ++i) mbar_init(BAR(BAR_KV_EMPTY + i), 1);
+        for (int i = 0; i < 3; ++i) mbar_init(BAR(BAR_STEP_FULL + i), 1);
         mbar_init(BAR(BAR_DRAIN), 1);
+        mbar_init(BAR(BAR_NEVER), 1);
         fence_mbarrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -416,99 +561,145 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
-
+    if (warp < 4) {
+    regs_dec<kRegsCtl>();
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             bool ok = true;
-            if (p.rope_cs != nullptr) {   // the table blocks holding this query block's tokens
-                const long long n0 = static_cast<long long>(b) * p.T + qb * kBM;
-                const long long n1 = n0 + min(kBM, p.T - qb * kBM) - 1;
-                for (long long blk = n0 >> 7; blk <= (n1 >> 7); ++blk)
-                    prefetch_l2_bulk(p.rope_cs + rope_table_index(blk << 7, 0) * 4, 32 * 128 * 16);
-            }
-            for (int s = 0; s < nslots; ++s) {
-                const uint32_t dst = sQ0 + s * kTileBytes;
-                mbar_arrive_expect_tx(BAR(BAR_Q_FULL + s), kTileBytes);
-                tma_load_4d(dst, &tm_q, 0, hq0 + s, qb * kBM, b, BAR(BAR_Q_FULL + s));
-                tma_load_4d(dst + kBoxBytes, &tm_q, 64, hq0 + s, qb * kBM, b, BAR(BAR_Q_FULL + s));
-            }
-            int issued = 0;
-            for (int it = 0; it < 2 * n_kv; ++it) {   // K0, V0, K1, V1, ...
-                const int buf = it % kStages, use = it / kStages;
-                if (use > 0 && !mbar_wait(BAR(BAR_KV_EMPTY + buf), (use - 1) & 1, p.err)) {
-                    ok = false;
-                    break;
+            uint32_t q_uses[2] = {0u, 0u};   // Q loads per slot so far
+            uint32_t k0_uses = 0;            // units so far (first K tiles)
+            uint32_t it = 0;                 // K/V ring items so far (K0 V0 K1 V1 ... per unit)
+            uint32_t gs = 0;                 // steps so far (one per K/V tile pair)
+            uint32_t step_arms[3] = {0u, 0u, 0u};   // phases armed on each step barrier
+            for (int u = blockIdx.x; u < p.nunits && ok; u += gridDim.x) {
+                AttnUnit w;
+                bool bad;
+                if (!attn_unit(p, u, w, bad)) {
+                    if (bad) atomicOr(p.err, kErrInput);
+                    continue;
                 }
-                const CUtensorMap *m = (it & 1) ? &tm_v : &tm_k;
-                const uint32_t dst = sKV0 + buf * kTileBytes;
-                const int row0 = (it >> 1) * kBN;
-                // K_0 signals its slot; V_j and K_{j+1} both signal step barrier j % 3,
-                // armed once for both when V_j is issued
-                const int jstep = (it - 1) >> 1;
-                const uint32_t bar = it == 0 ? BAR(BAR_KV_FULL + 0) : BAR(BAR_STEP_FULL + jstep % 3);
-                if (it == 0)
-                    mbar_arrive_expect_tx(bar, kTileBytes);
-                else if (it & 1)
-                    mbar_arrive_expect_tx(bar, jstep + 1 < n_kv ? 2 * kTileBytes : kTileBytes);
-                tma_load_4d(dst, m, 0, g, row0, b, bar);
-                tma_load_4d(dst + kBoxBytes, m, 64, g, row0, b, bar);
-                issued = it + 1;
+                if (p.rope_cs != nullptr) {   // the table blocks holding this query block's tokens
+                    for (long long blk = w.q0 >> 7; blk <= ((w.q0 + w.rows - 1) >> 7); ++blk)
+                        prefetch_l2_bulk(p.rope_cs + rope_table_index(blk << 7, 0) * 4, 32 * 128 * 16);
+                }
+                for (int s = 0; s < w.nslots && ok; ++s) {
+                    // the slot is free once the previous unit's last Q K^T on it has finished
+                    if (q_uses[s] > 0 && !mbar_wait(BAR(BAR_Q_EMPTY + s), (q_uses[s] - 1) & 1, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t dst = sQ0 + s * kTileBytes;
+                    mbar_arrive_expect_tx(BAR(BAR_Q_FULL + s), kTileBytes);
+                    tma_load_3d(dst, &tm_q, 0, w.hq0 + s, static_cast<int>(w.q0), BAR(BAR_Q_FULL + s));
+                    tma_load_3d(dst + kBoxBytes, &tm_q, 64, w.hq0 + s, static_cast<int>(w.q0), BAR(BAR_Q_FULL + s));
+                    ++q_uses[s];
+                }
+                for (int k = 0; k < 2 * w.n_kv && ok; ++k, ++it) {   // K0, V0, K1, V1, ...
+                    const uint32_t buf = it % kStages, use = it / kStages;
+                    if (use > 0 && !mbar_wait(BAR(BAR_KV_EMPTY + buf), (use - 1) & 1, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const CUtensorMap *m = (k & 1) ? &tm_v : &tm_k;
+                    const uint32_t dst = sKV0 + buf * kTileBytes;
+                    const int row = static_cast<int>(w.kv0 + static_cast<long long>(k >> 1) * kBN);
+                    // K_0 signals its own barrier; V_j and K_{j+1} both signal step barrier
+                    // (gs + j) % 3, armed once for both when V_j is issued
+                    const int j = (k - 1) >> 1;
+                    const uint32_t bar = k == 0 ? BAR(BAR_K0_FULL) : BAR(BAR_STEP_FULL + (gs + j) % 3);
+                    if (k == 0) {
+                        mbar_arrive_expect_tx(bar, kTileBytes);
+                        ++k0_uses;
+                    } else if (k & 1) {
+                        mbar_arrive_expect_tx(bar, j + 1 < w.n_kv ? 2 * kTileBytes : kTileBytes);
+                        ++step_arms[(gs + j) % 3];
+                    }
+                    tma_load_3d(dst, m, 0, w.g, row, bar);
+                    tma_load_3d(dst + kBoxBytes, m, 64, w.g, row, bar);
+                }
+                if (ok) gs += w.n_kv;
             }
             if (!ok) {
-                // Failure path: let every copy still in flight land before the CTA exits.
-                for (int s = 0; s < nslots; ++s) mbar_wait(BAR(BAR_Q_FULL + s), 0, p.err);
-                if (issued > 0) mbar_wait(BAR(BAR_KV_FULL + 0), 0, p.err);
-                for (int j = max(0, (issued - kStages - 1) >> 1); 2 * j + 1 < issued; ++j)
-                    mbar_wait(BAR(BAR_STEP_FULL + j % 3), (j / 3) & 1, p.err);
+                // Failure path: let every copy still in flight land before the CTA exits.  No
+                // barrier is re-armed before its previous phase completed, so waiting for the
+                // last armed phase of each covers every copy (a step barrier armed for two
+                // tiles of which only one was issued gives up after the bounded wait).
+                for (int s = 0; s < 2; ++s)
+                    if (q_uses[s] > 0) mbar_wait(BAR(BAR_Q_FULL + s), (q_uses[s] - 1) & 1, p.err);
+                if (k0_uses > 0) mbar_wait(BAR(BAR_K0_FULL), (k0_uses - 1) & 1, p.err);
+                for (int i = 0; i < 3; ++i)
+                    if (step_arms[i] > 0) mbar_wait(BAR(BAR_STEP_FULL + i), (step_arms[i] - 1) & 1, p.err);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         // In-order program with blocking (suspending) waits, heads interleaved:
-        //   Q K_0^T (both heads), then for every tile j and head s: P_j V_j as soon as
-        //   the softmax has written P_j over S_j, immediately followed by Q K_{j+1}^T
-        //   (which overwrites P_j: tcgen05.mma operations of one thread run in issue
-        //   order).  While head 0's softmax works on S_{j+1}, the tensor core runs head
-        //   1's P V and Q K^T, and vice versa.
+        //   per unit: Q K_0^T for each head as soon as its Q tile is ready; then for every
+        //   tile j and head s: P_j V_j once the softmax has written P_j over S_j,
+        //   immediately followed by Q K_{j+1}^T (which overwrites P_j: tcgen05.mma
+        //   operations of one thread run in issue order).  While head 0's softmax works on
+        //   S_{j+1}, the tensor core runs head 1's P V and Q K^T, and vice versa.  The
+        //   first P V of a unit (accumulate off) waits until the epilogue has read O out.
         // The issuing thread is on the critical path: its queue of MMAs is shallow, so
         // every wait it makes idles the tensor core.  Its waits carry a short suspend hint
         // (a default try_wait can wake up ~900 cycles after the phase completes), and V_j
         // and K_{j+1} share one barrier so that each tile costs one wait for data.
-#define MMA_WAIT(b_, par_, e_) mbar_wait_hint((b_), (par_), 20u, (e_))
+#define MMA_WAIT(b_, par_) mbar_wait_hint((b_), (par_), 20u, p.err)
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16_f32(kBM, kBN, false);
             const uint32_t id_pv = idesc_bf16_f32(kBM, kHeadDim, true);
             bool ok = true;
-            for (int s = 0; s < nslots && ok; ++s) ok = mbar_wait(BAR(BAR_Q_READY + s), 0, p.err);
-            if (ok) ok = mbar_wait(BAR(BAR_KV_FULL + 0), 0, p.err);   // K_0 is ring item 0
-            if (ok) {
-                tc_fence_after();
-                for (int s = 0; s < nslots; ++s) {
-                    issue_qk(tmem + s * 128, sQ0 + s * kTileBytes, sKV0, id_qk);
-                    umma_commit(BAR(BAR_S_FULL + s));
-                }
-                umma_commit(BAR(BAR_KV_EMPTY + 0));
-            }
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int iv = 2 * j + 1, ik = 2 * j + 2;   // ring items of V_j and K_{j+1}
-                const bool more = j + 1 < n_kv;
-                if (!MMA_WAIT(BAR(BAR_STEP_FULL + j % 3), (j / 3) & 1, p.err)) { ok = false; break; }
-                for (int s = 0; s < nslots; ++s) {
-                    if (!MMA_WAIT(BAR(BAR_P_FULL + s), j & 1, p.err)) { ok = false; break; }
+            uint32_t q_uses[2] = {0u, 0u}, tiles[2] = {0u, 0u}, units[2] = {0u, 0u};
+            uint32_t k0_uses = 0, it = 0, gs = 0;
+            // failure-path test: a wait that nothing ends gives up after 100 us
+            if (p.test_stall) ok = mbar_wait(BAR(BAR_NEVER), 0, p.err, 100000ull);
+            for (int u = blockIdx.x; u < p.nunits && ok; u += gridDim.x) {
+                AttnUnit w;
+                bool bad;
+                if (!attn_unit(p, u, w, bad)) continue;
+                const uint32_t k0_item = it;
+                if (!MMA_WAIT(BAR(BAR_K0_FULL), k0_uses & 1)) { ok = false; break; }
+                ++k0_uses;
+                for (int s = 0; s < w.nslots; ++s) {
+                    if (!MMA_WAIT(BAR(BAR_Q_READY + s), q_uses[s] & 1)) { ok = false; break; }
+                    ++q_uses[s];
                     tc_fence_after();
-                    issue_pv(tmem + 256 + s * 128, tmem + s * 128, sKV0 + (iv % kStages) * kTileBytes, id_pv, j > 0);
-                    if (more) {
-                        issue_qk(tmem + s * 128, sQ0 + s * kTileBytes, sKV0 + (ik % kStages) * kTileBytes, id_qk);
-                        umma_commit(BAR(BAR_S_FULL + s));
-                    } else {
-                        umma_commit(BAR(BAR_O_FULL + s));
-                    }
+                    issue_qk(tmem + s * 128, sQ0 + s * kTileBytes, sKV0 + (k0_item % kStages) * kTileBytes, id_qk);
+                    umma_commit(BAR(BAR_S_FULL + s));
+                    if (w.n_kv == 1) umma_commit(BAR(BAR_Q_EMPTY + s));
                 }
                 if (!ok) break;
-                umma_commit(BAR(BAR_KV_EMPTY + iv % kStages));
-                if (more) umma_commit(BAR(BAR_KV_EMPTY + ik % kStages));
+                umma_commit(BAR(BAR_KV_EMPTY + k0_item % kStages));
+                for (int j = 0; j < w.n_kv && ok; ++j) {
+                    const uint32_t iv = k0_item + 2 * j + 1, ik = k0_item + 2 * j + 2;   // ring items of V_j, K_{j+1}
+                    const bool more = j + 1 < w.n_kv;
+                    if (!MMA_WAIT(BAR(BAR_STEP_FULL + (gs + j) % 3), ((gs + j) / 3) & 1)) { ok = false; break; }
+                    for (int s = 0; s < w.nslots; ++s) {
+                        if (!MMA_WAIT(BAR(BAR_P_FULL + s), tiles[s] & 1)) { ok = false; break; }
+                        ++tiles[s];
+                        if (j == 0 && units[s] > 0 && !MMA_WAIT(BAR(BAR_O_EMPTY + s), (units[s] - 1) & 1)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_pv(tmem + 256 + s * 128, tmem + s * 128, sKV0 + (iv % kStages) * kTileBytes, id_pv, j > 0);
+                        if (more) {
+                            issue_qk(tmem + s * 128, sQ0 + s * kTileBytes, sKV0 + (ik % kStages) * kTileBytes, id_qk);
+                            umma_commit(BAR(BAR_S_FULL + s));
+                            if (j + 2 == w.n_kv) umma_commit(BAR(BAR_Q_EMPTY + s));
+                        } else {
+                            umma_commit(BAR(BAR_O_FULL + s));
+                            ++units[s];
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit(BAR(BAR_KV_EMPTY + iv % kStages));
+                    if (more) umma_commit(BAR(BAR_KV_EMPTY + ik % kStages));
+                }
+                it += 2 * w.n_kv;
+                gs += w.n_kv;
             }
             // Every MMA issued above must finish before TMEM can be released.
             umma_commit(BAR(BAR_DRAIN));
@@ -516,34 +707,91 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
 #undef MMA_WAIT
         __syncwarp();
-    } else if (warp >= 4) {
+    }
+    } else {
+        regs_inc<kRegsSoftmax>();
         // ------------------------------------------------------------ softmax warpgroups
+        // Per unit: norm + rotate the Q tile, then the online softmax of every S tile.
+        // The epilogue of a unit (O / l to global) runs after the next unit's Q tile has
+        // been transformed, so that the next unit's first Q K^T overlaps it.
         const int s = (warp - 4) >> 2;
         const int r = tid - 128 * (1 + s);   // query row in the tile == TMEM lane
-        if (s < nslots) {
-            const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-            const uint32_t tS = tmem + lane_base + s * 128;
-            const uint32_t tO = tmem + lane_base + 256 + s * 128;
-            const int t = qb * kBM + r;
-            const bool valid = t < p.T;
-            const int hq = hq0 + s;
-
-            bool ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_Q_FULL + s), 0, p.err));
-            if (ok) {
-                const long long tok = static_cast<long long>(b) * p.T + t;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + s * 128;
+        const uint32_t tO = tmem + lane_base + 256 + s * 128;
+        bool ok = true;
+        uint32_t q_uses = 0, tiles = 0, units = 0;
+        // the unit whose epilogue is pending
+        bool pend = false;
+        float pend_l = 1.f;
+        long long pend_row = -1;   // element offset of this thread's output row, or -1
+        int u = blockIdx.x;
+        while (ok) {
+            AttnUnit w;
+            bool have = false, bad;
+            for (; u < p.nunits; u += gridDim.x)
+                if (attn_unit(p, u, w, bad) && s < w.nslots) {
+                    have = true;
+                    break;
+                }
+            if (have) {
+                ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_Q_FULL + s), q_uses & 1, p.err));
+                if (!ok) break;
+                ++q_uses;
+                const bool valid = r < w.rows;
+                const long long tok = w.q0 + r;
                 const int ps = valid ? p.pos[tok] : 0;
                 transform_q_row<PAIRING>(sQ0 + s * kTileBytes, r, ps, valid ? p.rope_cs : nullptr, tok, p.wq, p.eps,
                                          p.rf);
                 fence_proxy_async_smem();
                 mbar_arrive(BAR(BAR_Q_READY + s));
             }
+            if (pend) {
+                ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_O_FULL + s), units & 1, p.err));
+                if (!ok) break;
+                ++units;
+                tc_fence_after();
+                const float inv_l = 1.0f / pend_l;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float o[32];
+                    tmem_ld32(tO + 32 * c, o);
+                    tmem_wait_ld();
+                    if (pend_row >= 0) {
+                        if (p.out_bf16) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + pend_row + 32 * c);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                dst[e] = make_uint4(pack_bf16x2(o[8 * e] * inv_l, o[8 * e + 1] * inv_l),
+                                                    pack_bf16x2(o[8 * e + 2] * inv_l, o[8 * e + 3] * inv_l),
+                                                    pack_bf16x2(o[8 * e + 4] * inv_l, o[8 * e + 5] * inv_l),
+                                                    pack_bf16x2(o[8 * e + 6] * inv_l, o[8 * e + 7] * inv_l));
+                        } else {
+                            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + pend_row + 32 * c);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                dst[e] = make_float4(o[4 * e] * inv_l, o[4 * e + 1] * inv_l, o[4 * e + 2] * inv_l,
+                                                     o[4 * e + 3] * inv_l);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(BAR(BAR_O_EMPTY + s));
+                pend = false;
+            }
+            if (!have) break;
 
+            // what the epilogue needs, computed now so that only n_kv and rowkey stay live
+            const long long orow = r < w.rows ? ((w.q0 + r) * p.H + w.hq0 + s) * kHeadDim : -1;
+            const int n_kv = w.n_kv;
+            const int rowkey = w.key0 + r;   // token index of this row: sees keys 0 .. rowkey
             float m_run = -INFINITY;   // running max of scaled scores (base 2), possibly stale by < 8
             float l_run = 0.f;         // running sum of 2^(score - m_run)
             for (int j = 0; j < n_kv && ok; ++j) {
                 // S_FULL of tile j also means P_{j-1} V_{j-1} has finished (issued before Q K_j^T).
-                ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_S_FULL + s), j & 1, p.err));
+                ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_S_FULL + s), tiles & 1, p.err));
                 if (!ok) break;
+                ++tiles;
                 tc_fence_after();
                 float x[128];
                 tmem_ld32(tS, x);
@@ -551,15 +799,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tmem_ld32(tS + 64, x + 64);
                 tmem_ld32(tS + 96, x + 96);
                 tmem_wait_ld();
-                if (j == qb) {   // diagonal tile: key c is visible to row r iff c <= r
+                const int lim = rowkey - j * kBN;   // keys c <= lim of this tile are visible
+                const bool masked = lim < kBN - 1;
+                if (masked) {
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
-                        if (c > r) x[c] = -INFINITY;
+                        if (c > lim) x[c] = -INFINITY;
                 }
                 // row max with eight independent partial maxima (short dependency chains)
                 float mp[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) mp[u] = x[u];
+                for (int e = 0; e < 8; ++e) mp[e] = x[e];
 #pragma unroll
                 for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
                 const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
@@ -567,22 +817,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const float m_new = fmaxf(m_run, mx * p.scale_log2);
                 // Only move the reference max when it grows by more than 2^8; the final
                 // O / l is exact either way because O and l always share the reference.
+                // A row with no visible key yet (only past the end of its sequence) keeps
+                // -inf and adds nothing.
                 const bool need = m_new > m_run + 8.0f;
                 const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
                 if (need) m_run = m_new;
                 l_run *= alpha;
-                const float negm = -m_run;
+                const float negm = m_run == -INFINITY ? 0.f : -m_run;
                 float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                {
-                    uint32_t pk[32];
-                    exp_pack64(x, p.scale_log2, negm, pk, sp);
-                    tmem_st32(tS, reinterpret_cast<const float *>(pk));          // P keys 0..63
-                }
-                {
-                    uint32_t pk[32];
-                    exp_pack64(x + 64, p.scale_log2, negm, pk, sp);
-                    tmem_st32(tS + 32, reinterpret_cast<const float *>(pk));     // P keys 64..127
-                }
+                if (kExpPolyPairs > 0 && !__any_sync(0xffffffffu, masked))
+                    exp_tile<kExpPolyPairs>(x, p.scale_log2, negm, tS, sp);
+                else
+                    exp_tile<0>(x, p.scale_log2, negm, tS, sp);
                 // Rescale this row of O if the reference moved (rare after the first tiles).
                 // O is stable: P_{j-1} V_{j-1} finished before S_j was signalled.
                 if (__any_sync(0xffffffffu, need) && j > 0) {
@@ -592,7 +838,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         tmem_ld32(tO + 32 * c, o);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int u = 0; u < 32; ++u) o[u] *= alpha;
+                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
                         tmem_st32(tO + 32 * c, o);
                     }
                 }
@@ -601,27 +847,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 mbar_arrive(BAR(BAR_P_FULL + s));
                 l_run += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
             }
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_O_FULL + s), 0, p.err));
-            if (ok) {
-                tc_fence_after();
-                const float inv_l = 1.0f / l_run;
-                float *orow = p.out + ((static_cast<size_t>(b) * p.T + t) * p.H + hq) * kHeadDim;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float o[32];
-                    tmem_ld32(tO + 32 * c, o);
-                    tmem_wait_ld();
-                    if (valid) {
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            reinterpret_cast<float4 *>(orow + 32 * c)[u] =
-                                make_float4(o[4 * u] * inv_l, o[4 * u + 1] * inv_l, o[4 * u + 2] * inv_l,
-                                            o[4 * u + 3] * inv_l);
-                    }
-                }
-            }
-            tc_fence_before();
+            pend = true;
+            pend_l = l_run;
+            pend_row = orow;
+            u += gridDim.x;
         }
+        tc_fence_before();
     }
 #undef BAR
     __syncthreads();

@@ -11,6 +11,9 @@ so that a CPU check and the GPU path see the same bits.
 * positions: 0 .. T-1 per sequence (int32).
 * decode: per-sequence cache lengths uniform on [len_lo, len_hi]; K and V cache
   rows N(0, 1) bf16, packed sequence after sequence as [rows, Hkv, D].
+* packed prefill: sequence lengths uniform on [len_lo, len_hi], tokens packed; a
+  chunk after a cached prefix adds a cache whose prefix rows are N(0, 1) bf16.
+* projections: hidden states N(0, 1) bf16, weights N(0, 1/fan-in) bf16.
 """
 from __future__ import annotations
 
@@ -187,6 +190,74 @@ def page_cache(k_rows: torch.Tensor, v_rows: torch.Tensor, offsets, capacities, 
     return PagedCache(kp, vp, table, page_size)
 
 
+@dataclass
+class PackedInputs:
+    """Sequences packed token after token: q [N,H,D], k/v [N,Hkv,D] raw bf16, positions
+    [N] (each sequence from prefix[b] on), cu [B+1] token offsets; for a chunk after a
+    cached prefix also the cache (k-hat / v rows of the prefix, room for the chunk)."""
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    pos: torch.Tensor
+    cu: torch.Tensor
+    wq: torch.Tensor
+    wk: torch.Tensor
+    prefix: torch.Tensor = None      # int32 [B] cached rows (chunk workloads)
+    k_cache: torch.Tensor = None     # bf16 [rows, Hkv, D]
+    v_cache: torch.Tensor = None
+    cache_offsets: torch.Tensor = None   # int64 [B+1]
+    theta: float = THETA
+    eps: float = EPS
+
+    @property
+    def lens(self):
+        return (self.cu[1:] - self.cu[:-1]).tolist()
+
+
+def packed_inputs(lens, H: int, Hkv: int, D: int = HEAD_DIM, seed: int = 0, prefix=None) -> PackedInputs:
+    """Packed sequences of the given lengths, N(0,1) bf16 q/k/v, U(0.5, 1.5) norm weights.
+    With prefix (rows already cached per sequence), a cache of prefix[b] + lens[b] rows
+    per sequence is added whose first prefix[b] rows hold N(0,1) bf16 values (they stand
+    in for cached k-hat and v, as in the decode workloads)."""
+    B = len(lens)
+    N = int(sum(lens))
+    cu = torch.zeros(B + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(torch.as_tensor(lens, dtype=torch.int64), 0)
+    pre = [0] * B if prefix is None else [int(p) for p in prefix]
+    pos = torch.cat([torch.arange(p, p + n, dtype=torch.int32) for p, n in zip(pre, lens)]) if N else \
+        torch.zeros(0, dtype=torch.int32)
+    out = PackedInputs(_normal_bf16((N, H, D), seed), _normal_bf16((N, Hkv, D), seed + 1),
+                       _normal_bf16((N, Hkv, D), seed + 2), pos, cu, _uniform((D,), seed + 3, 0.5, 1.5),
+                       _uniform((D,), seed + 4, 0.5, 1.5))
+    if prefix is not None:
+        caps = torch.as_tensor([p + n for p, n in zip(pre, lens)], dtype=torch.int64)
+        offs = torch.zeros(B + 1, dtype=torch.int64)
+        offs[1:] = torch.cumsum(caps, 0)
+        out.prefix = torch.as_tensor(pre, dtype=torch.int32)
+        out.k_cache = _normal_bf16((int(offs[-1]), Hkv, D), seed + 5)
+        out.v_cache = _normal_bf16((int(offs[-1]), Hkv, D), seed + 6)
+        out.cache_offsets = offs
+    return out
+
+
+@dataclass
+class ProjectionInputs:
+    """Hidden states x [N, hidden] bf16 N(0,1) and projection weights scaled by
+    1/sqrt(fan-in): w_qkv [(H + 2 Hkv) D, hidden], w_o [hidden, H D]."""
+    x: torch.Tensor
+    w_qkv: torch.Tensor
+    w_o: torch.Tensor
+    H: int
+    Hkv: int
+
+
+def projection_inputs(N: int, hidden: int, H: int, Hkv: int, D: int = HEAD_DIM, seed: int = 0) -> ProjectionInputs:
+    x = _normal_bf16((N, hidden), seed)
+    w_qkv = _normal_bf16(((H + 2 * Hkv) * D, hidden), seed + 1, 1.0 / hidden ** 0.5)
+    w_o = _normal_bf16((hidden, H * D), seed + 2, 1.0 / (H * D) ** 0.5)
+    return ProjectionInputs(x, w_qkv, w_o, H, Hkv)
+
+
 # The documented workloads, by name.
 WORKLOADS = {
     "prefill_correctness": dict(kind="prefill", B=1, T=128, H=16, Hkv=8),
@@ -198,6 +269,12 @@ WORKLOADS = {
     "batched_decode": dict(kind="decode", B=64, H=32, Hkv=8, len_lo=1024, len_hi=32768),
     "long_context_prefill": dict(kind="prefill", B=1, T=32768, H=64, Hkv=8),
     "batched_decode_append": dict(kind="decode_append", B=64, H=32, Hkv=8, len_lo=1023, len_hi=32767),
+    # 16 packed sequences, lengths U{256..8192}
+    "varlen_prefill": dict(kind="packed", B=16, H=32, Hkv=8, len_lo=256, len_hi=8192),
+    # 8 sequences with 8192 cached rows each and a new chunk of 2048 tokens
+    "chunked_prefill": dict(kind="chunk", B=8, H=32, Hkv=8, prefix=8192, chunk=2048),
+    # the projections around the large prefill's attention: 16384 tokens, hidden 4096
+    "projections": dict(kind="projection", N=16384, hidden=4096, H=32, Hkv=8),
 }
 
 
@@ -208,4 +285,11 @@ def make(name: str, seed: int = 0):
         return prefill_inputs(seed=seed, **w)
     if kind == "decode_append":
         return decode_append_inputs(seed=seed, **w)
+    if kind == "packed":
+        lens = torch.randint(w["len_lo"], w["len_hi"] + 1, (w["B"],), generator=_gen(seed + 10)).tolist()
+        return packed_inputs(lens, w["H"], w["Hkv"], seed=seed)
+    if kind == "chunk":
+        return packed_inputs([w["chunk"]] * w["B"], w["H"], w["Hkv"], seed=seed, prefix=[w["prefix"]] * w["B"])
+    if kind == "projection":
+        return projection_inputs(w["N"], w["hidden"], w["H"], w["Hkv"], seed=seed)
     return decode_inputs(seed=seed, **w)

@@ -206,7 +206,8 @@ gqa_status gqa_attn_decode_append(const void *q, const void *k_new, const void *
  * workspace: the split-KV partial results go to a scratch array that is part of the
  * library itself (GQA_NOALLOC_SCRATCH_BYTES of device memory that every GPU which
  * loads the library holds until the process exits).  No call allocates or frees.
- *   - Problems whose partials need more than GQA_NOALLOC_SCRATCH_BYTES, i.e.
+ *   - Every argument check of gqa_attn_decode runs first, with the same status codes.
+ *     Then problems whose partials need more than GQA_NOALLOC_SCRATCH_BYTES, i.e.
  *     gqa_attn_decode_workspace_size(B, H, Hkv, D, max_len) > GQA_NOALLOC_SCRATCH_BYTES,
  *     are rejected with GQA_ERR_WORKSPACE before anything is launched.
  *   - The first call on a device looks up the scratch array's device address (once per
@@ -307,6 +308,66 @@ gqa_status gqa_attn_decode_append_ex(const void *q, const void *k_new, const voi
                                      int H, int Hkv, int D, int max_len, void *workspace,
                                      size_t workspace_bytes, void *stream);
 
+/* ----------------------------------------------------------------- packed and chunked prefill
+ *
+ * Variable-length prefill: B sequences of different lengths packed one after another
+ * ("Qwen3系列1" D1-5: the causal mask applies within each sequence; "Qwen3" walkthrough,
+ * "Attention 的 Forward 流程": the q/k/v of a batch arrive as one [N, heads, D] tensor).
+ *
+ *   q         bf16 [N, H, D]      raw queries of all N tokens, sequence after sequence
+ *   k, v      bf16 [N, Hkv, D]    raw keys (normed and rotated here) and values
+ *   pos       int32 [N]           RoPE position of every token
+ *   cu_seqlens int64 [B + 1]      device: sequence b is tokens cu_seqlens[b] ..
+ *                                 cu_seqlens[b+1] - 1 (0 = cu_seqlens[0] <= ... <=
+ *                                 cu_seqlens[B] = N; empty sequences are allowed)
+ *   qnorm_w, knorm_w, rope, eps   as for gqa_attn_prefill_ex (rope must not be NULL)
+ *   out       fp32 [N, H, D]      row t of sequence b attends to keys 0 .. t of b only
+ *   max_seqlen host-side bound on every sequence's length (sizes the launch)
+ *   workspace >= gqa_attn_prefill_varlen_workspace_size(N, Hkv, D) bytes, 256-byte
+ *             aligned (k-hat of the N tokens and their RoPE cos/sin).
+ * Sequence bounds are read on the device: a sequence that breaks them (or is longer than
+ * max_seqlen, whose tail then goes unwritten) is skipped and sets GQA_ERR_DEVICE_INPUT;
+ * its output rows are undefined.  B = 0, N = 0 or max_seqlen = 0 is a no-op.
+ */
+size_t gqa_attn_prefill_varlen_workspace_size(int64_t N, int Hkv, int D);
+gqa_status gqa_attn_prefill_varlen(const void *q, const void *k, const void *v, const int32_t *pos,
+                                   const int64_t *cu_seqlens, const float *qnorm_w,
+                                   const float *knorm_w, const gqa_rope_config *rope, float eps,
+                                   float *out, int B, int64_t N, int H, int Hkv, int D,
+                                   int max_seqlen, void *workspace, size_t workspace_bytes,
+                                   void *stream);
+
+/*
+ * Chunked prefill: each sequence already has prefix_len[b] rows in the KV cache (from an
+ * earlier prefill or chunk) and a new chunk of tokens arrives ("Qwen3系列1" D2-3: the
+ * keys and values of earlier tokens live in the per-layer cache, which grows along the
+ * tokens; K/V are written into it before attention).  The call first writes the chunk's
+ * k-hat (RMSNorm + RoPE at pos) and v into the cache, right after the cached rows, then
+ * chunk row t of sequence b (token prefix_len[b] + t) attends to cache rows
+ * 0 .. prefix_len[b] + t of that sequence.
+ *
+ *   q, k, v, pos, cu_seqlens, out  the N chunk tokens, packed as for gqa_attn_prefill_varlen
+ *   k_cache, v_cache  bf16 [cache_rows, Hkv, D]; sequence b owns rows cache_offsets[b] ..
+ *                     cache_offsets[b+1] - 1 and must have room for prefix_len[b] +
+ *                     chunk length rows; the chunk's rows are written in place
+ *   cache_offsets     int64 [B + 1], device, non-decreasing
+ *   prefix_len        int32 [B], device, rows already cached (0 = plain prefill of the chunk)
+ *   max_chunk_len     host-side bound on every chunk's length
+ *   workspace >= gqa_attn_prefill_chunk_workspace_size(N, D) bytes, 256-byte aligned
+ *             (the chunk tokens' RoPE cos/sin).
+ * A chunk token whose cache row falls outside its sequence's rows is not written and
+ * sets GQA_ERR_DEVICE_INPUT (that sequence's output is then undefined); the same for
+ * sequence bounds out of range.  prefix_len is not advanced (the caller does that).
+ */
+size_t gqa_attn_prefill_chunk_workspace_size(int64_t N, int D);
+gqa_status gqa_attn_prefill_chunk(const void *q, const void *k, const void *v, const int32_t *pos,
+                                  const int64_t *cu_seqlens, void *k_cache, void *v_cache,
+                                  const int64_t *cache_offsets, const int32_t *prefix_len,
+                                  int64_t cache_rows, const float *qnorm_w, const float *knorm_w,
+                                  const gqa_rope_config *rope, float eps, float *out, int B,
+                                  int64_t N, int H, int Hkv, int D, int max_chunk_len,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
 /* ----------------------------------------------------------------- paged KV cache
  *
  * The decode cache may also live in fixed-size pages (the layout of paged-attention
@@ -340,6 +401,51 @@ gqa_status gqa_attn_decode_append_paged(const void *q, const void *k_new, const 
                                         int H, int Hkv, int D, int max_len, void *workspace,
                                         size_t workspace_bytes, void *stream);
 
+/* ----------------------------------------------------------------- projections
+ *
+ * The dense contractions around the attention ("Qwen3" walkthrough, "Attention 的
+ * Forward 流程": step 1 qkv = qkv_proj(hidden_states), split and viewed per head in
+ * steps 2-3; step 7 output = o_proj(o.flatten(1, -1)); "Qwen3系列1" D1-2: a linear layer
+ * is Y = XW + b and Qwen3's projections have no b; D1-4 Q4/Q5: the heads are
+ * concatenated, then multiplied by W_O):
+ *
+ *     y[m][n] = sum_k x[m][k] w[n][k]          (nn.Linear: y = x W^T, no bias)
+ *
+ *   x   bf16 [M, K] row-major      w  bf16 [N, K] row-major (one output feature per row)
+ *   y   [M, N] row-major, bf16 (GQA_DTYPE_BF16, rounded to nearest even) or fp32
+ *       (GQA_DTYPE_F32); fp32 accumulation on the tensor cores either way
+ *   N must be a multiple of 32 and K of 8; M >= 0 (0 is a no-op).  All pointers 16-byte
+ *   aligned device memory.  The fused QKV projection is gqa_linear with w = [W_q; W_k;
+ *   W_v] ((H + 2 Hkv) D rows): its output [M, H + 2 Hkv, D] is read in place by
+ *   gqa_attn_block_prefill.
+ */
+typedef enum { GQA_DTYPE_BF16 = 0, GQA_DTYPE_F32 = 1 } gqa_dtype;
+
+gqa_status gqa_linear(const void *x, const void *w, void *y, int y_dtype, int64_t M, int N, int K,
+                      void *stream);
+
+/*
+ * The whole attention sub-block of a decoder layer for a prefill (the seven steps of the
+ * "Qwen3" walkthrough's Qwen3Attention.forward): qkv = x W_qkv^T (bf16), split into
+ * q [.., H, D], k [.., Hkv, D], v [.., Hkv, D]; q/k RMSNorm; RoPE; causal GQA attention
+ * (bf16 output, the dtype the projection reads); y = o W_o^T over the concatenated heads.
+ *
+ *   x      bf16 [B*T, hidden]          hidden states of B sequences of T tokens
+ *   w_qkv  bf16 [(H + 2 Hkv) D, hidden] = [W_q; W_k; W_v]
+ *   w_o    bf16 [hidden, H D]
+ *   pos, qnorm_w, knorm_w, rope, eps   as for gqa_attn_prefill_ex (rope not NULL)
+ *   y      fp32 [B*T, hidden]
+ *   workspace >= gqa_attn_block_prefill_workspace_size(...) bytes, 256-byte aligned:
+ *          qkv, k-hat, the RoPE table and the attention output.
+ * hidden must be a multiple of 32.  B = 0 or T = 0 is a no-op.
+ */
+size_t gqa_attn_block_prefill_workspace_size(int B, int T, int hidden, int H, int Hkv, int D);
+gqa_status gqa_attn_block_prefill(const void *x, const void *w_qkv, const void *w_o, const int32_t *pos,
+                                  const float *qnorm_w, const float *knorm_w,
+                                  const gqa_rope_config *rope, float eps, float *y, int B, int T,
+                                  int hidden, int H, int Hkv, int D, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
 /*
  * Device status: waits for `stream` (a cudaStream_t as void*, NULL = legacy default
  * stream), then reads and clears the library's device error word on the current
@@ -348,6 +454,17 @@ gqa_status gqa_attn_decode_append_paged(const void *q, const void *k_new, const 
  * broke its length bounds), or GQA_ERR_CUDA.  This is the only synchronizing call.
  */
 gqa_status gqa_attn_device_status(void *stream);
+
+/*
+ * Test switch for the failure path, not for production use: while enabled (non-zero),
+ * every attention launch makes its MMA-issuing thread first wait on a barrier that
+ * nothing signals.  That wait gives up after 100 us and records GQA_ERR_DEVICE_TIMEOUT;
+ * the thread then issues nothing, and the CTA's other roles give up their own waits
+ * after the usual 2 s limit, let their copies in flight land and release tensor memory,
+ * so the launch ends (after a few seconds) with garbage output and the device usable.
+ * Call with 0 to switch it off.  It affects launches enqueued while it is on.
+ */
+void gqa_attn_test_stall(int enable);
 
 #ifdef __cplusplus
 }

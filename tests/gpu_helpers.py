@@ -35,18 +35,21 @@ def oracle_prefill_args(inp: synthetic.PrefillInputs):
             inp.theta, inp.eps)
 
 
-def sample_rows(B, T, H, n_random, seed=0):
-    """(b, hq, i) rows: tile edges, the first and last rows, and random ones."""
-    rng = np.random.default_rng(seed)
+def strided_rows(B, T, H, stride, edges=(), tail_heads=(), tail=0, whole_heads=()):
+    """(b, hq, i) rows for a full-size prefill check: every `stride`-th row of every head
+    (the phase shifts from head to head, so that together the heads cover every row
+    offset inside a 128-row tile), the rows `edges` of every head, the last `tail` rows
+    of every head in `tail_heads`, and every row of the (b, hq) heads in `whole_heads`."""
     rows = set()
-    edges = [0, 1, 126, 127, 128, 129, 255, 256, T // 2, T - 129, T - 128, T - 2, T - 1]
     for b in range(B):
-        for i in edges:
-            if 0 <= i < T:
-                rows.add((b, int(rng.integers(H)), i))
-                rows.add((b, H - 1, i))
-    for _ in range(n_random):
-        rows.add((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(T))))
+        for hq in range(H):
+            phase = (7 * hq + 3 * b) % stride
+            rows.update((b, hq, i) for i in range(phase, T, stride))
+            rows.update((b, hq, i) for i in edges if 0 <= i < T)
+            if hq in tail_heads:
+                rows.update((b, hq, i) for i in range(max(0, T - tail), T))
+    for b, hq in whole_heads:
+        rows.update((b, hq, i) for i in range(T))
     return np.array(sorted(rows), dtype=np.int64)
 
 

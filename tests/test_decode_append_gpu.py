@@ -87,19 +87,14 @@ def test_explicit_positions(gqa):
 
 def test_batched_decode_append_config(gqa):
     """64 sequences with 1023..32767 cached rows, H=32, Hkv=8: the append-step workload
-    the benchmark times.  Outputs checked on a sample of sequences, every cache row
-    checked."""
+    the benchmark times.  Every sequence's output and every cache row checked."""
     inp = synthetic.make("batched_decode_append")
     out, kc, vc = _run(gqa, inp)
     gqa.check_device_status()
-    sl = inp.seqlens.numpy()
-    rng = np.random.default_rng(1)
-    idx = sorted(set([int(sl.argmin()), int(sl.argmax())] + rng.choice(64, 8, replace=False).tolist()))
-    ref, _ = _oracle(inp, idx)
-    assert_close(out[idx], ref, "batched_decode_append")
     assert np.isfinite(out).all()
+    ref, kh = _oracle(inp)
+    assert_close(out, ref, "batched_decode_append, all 64 sequences")
     # the written keys: k-hat of every new key at its position (the sequence length)
-    kh = oracle.qk_transform(bits(inp.k_new), sl.astype(np.int32), inp.wk.numpy(), inp.theta, inp.eps)
     _check_cache(inp, kc, vc, kh)
 
 

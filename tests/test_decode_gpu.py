@@ -42,17 +42,12 @@ def _oracle(inp, idx=None, q_pos=None):
 
 def test_batched_decode_config(gqa):
     """64 sequences, len ~ U[1024, 32768], H=32, Hkv=8, query at position len: the
-    launch the benchmark times.  Checked on a sample of sequences (the shortest, the
-    longest and random ones) against the oracle, all 32 heads each."""
+    launch the benchmark times, every sequence and every head against the oracle."""
     inp = synthetic.make("batched_decode")
     got = _run(gqa, inp)
     gqa.check_device_status()
-    sl = inp.seqlens.numpy()
-    rng = np.random.default_rng(0)
-    idx = sorted(set([int(sl.argmin()), int(sl.argmax())] + rng.choice(64, 10, replace=False).tolist()))
-    ref = _oracle(inp, idx)
-    assert_close(got[idx], ref, "batched_decode")
     assert np.isfinite(got).all()
+    assert_close(got, _oracle(inp), "batched_decode, all 64 sequences")
 
 
 @pytest.mark.parametrize("H,Hkv", [(16, 16), (16, 8), (16, 4), (16, 1), (12, 4), (10, 2), (32, 8)])

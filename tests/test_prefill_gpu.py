@@ -6,7 +6,7 @@ import torch
 
 from oracle import oracle
 from grouped_query_causal_b200 import synthetic
-from tests.gpu_helpers import (assert_close, bits as bits_of, oracle_prefill_args, sample_rows, to_dev)
+from tests.gpu_helpers import (assert_close, bits as bits_of, oracle_prefill_args, strided_rows, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,25 +72,35 @@ def test_deterministic(gqa):
     np.testing.assert_array_equal(a, b)
 
 
-def test_large_prefill_sampled_rows(gqa):
+def test_large_prefill_strided_rows(gqa):
     """B=4, T=4096, H=32, Hkv=8, inputs x0.5, in the launch configuration the benchmark
-    times; checked on sampled rows the oracle computes one by one."""
+    times.  Checked element by element against the oracle on every 16th row of every
+    head (phase shifted per head, so every row offset of a tile is covered), the tile
+    edges of every head, and every row of three whole heads (among them the last KV
+    head of the last sequence and its last query block)."""
     inp = synthetic.make("large_prefill")
     got = _run(gqa, inp)
-    rows = sample_rows(4, 4096, 32, n_random=96, seed=1)
-    ref = oracle.prefill_rows(*oracle_prefill_args(inp), rows)
-    assert_close(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, "large_prefill rows")
     assert np.isfinite(got).all()
+    T = 4096
+    rows = strided_rows(4, T, 32, 16, edges=(0, 1, 126, 127, 128, 129, 2047, 2048, T - 129, T - 128, T - 1),
+                        whole_heads=((3, 31), (0, 0), (2, 13)))
+    ref = oracle.prefill_rows(*oracle_prefill_args(inp), rows)
+    assert_close(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, f"large_prefill, {len(rows)} rows")
 
 
-def test_long_context_prefill_sampled_rows(gqa):
-    """B=1, T=32768, H=64, Hkv=8: sampled rows (incl. the last, longest ones)."""
+def test_long_context_prefill_strided_rows(gqa):
+    """B=1, T=32768, H=64, Hkv=8, in the benchmark's launch configuration: every 64th
+    row of every head (phase shifted per head), tile and half-sequence edges of every
+    head, and the last 256 rows of every head of the last KV group (the longest causal
+    sweeps, over all 256 key tiles)."""
     inp = synthetic.make("long_context_prefill")
     got = _run(gqa, inp)
-    rows = sample_rows(1, 32768, 64, n_random=24, seed=2)
-    ref = oracle.prefill_rows(*oracle_prefill_args(inp), rows)
-    assert_close(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, "long_context rows")
     assert np.isfinite(got).all()
+    T = 32768
+    rows = strided_rows(1, T, 64, 64, edges=(0, 1, 127, 128, 129, 16383, 16384, T - 129, T - 128, T - 1),
+                        tail_heads=range(56, 64), tail=256)
+    ref = oracle.prefill_rows(*oracle_prefill_args(inp), rows)
+    assert_close(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, f"long_context, {len(rows)} rows")
 
 
 def test_empty_problem_is_noop(gqa):
