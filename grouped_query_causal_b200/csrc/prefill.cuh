@@ -444,49 +444,13 @@ __device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, cons
     }
 }
 
-// Exponentials per score tile: of every 4 pairs of scores, the first kExpPolyPairs are
-// evaluated on the FMA pipes (exp2_poly2) and the rest by the MUFU ex2 instruction, so
-// that the two pipes share the work (the MUFU rate alone, 16 per clock per SM, equals the
-// tensor cores' rate of keys at D = 128).
-constexpr int kExpPolyPairs = 0;
-
-// 2^x for a pair of scores on the FMA pipes, after the Cody-Waite range reduction
-// x = j + f with j = rint(x) (adding and subtracting 1.5 * 2^23), |f| <= 1/2, and a
-// degree-3 polynomial for 2^f fitted here for least maximum relative error on [-1/2, 1/2]
-// (7.5e-5, far below the 2^-9 of the bf16 the result is rounded to); 2^j goes into the
-// exponent field by an integer add.  x is clamped to -125 (2^-125 rounds to a harmless
-// 2.4e-38), so tiles with masked (-inf) scores use ex2 instead.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-    x.x = fmaxf(x.x, -125.0f);
-    x.y = fmaxf(x.y, -125.0f);
-    const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-    const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
-    const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
-    float2 p = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.24261114f, 0.24261114f));
-    p = __ffma2_rn(p, f, make_float2(0.693260968f, 0.693260968f));
-    p = __ffma2_rn(p, f, make_float2(0.999928057f, 0.999928057f));
-    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
 // 2^(x*scale + negm) of 64 consecutive scores, packed as bf16 pairs into 32 words; their
-// (unrounded) sum goes into eight partial sums.  NPOLY: pairs out of every 4 evaluated on
-// the FMA pipes.
-template <int NPOLY>
+// (unrounded) sum goes into eight partial sums.
 __device__ __forceinline__ void exp_pack64(const float *x, float scale, float negm, uint32_t *pk, float (&sp)[8]) {
-    const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(negm, negm);
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
-        float e0, e1;
-        if ((c & 3) < NPOLY) {
-            const float2 e = exp2_poly2(__ffma2_rn(make_float2(x[2 * c], x[2 * c + 1]), sc2, nm2));
-            e0 = e.x;
-            e1 = e.y;
-        } else {
-            e0 = ex2_approx(fmaf(x[2 * c], scale, negm));
-            e1 = ex2_approx(fmaf(x[2 * c + 1], scale, negm));
-        }
+        const float e0 = ex2_approx(fmaf(x[2 * c], scale, negm));
+        const float e1 = ex2_approx(fmaf(x[2 * c + 1], scale, negm));
         sp[(2 * c) & 7] += e0;
         sp[(2 * c + 1) & 7] += e1;
         pk[c] = pack_bf16x2(e0, e1);
@@ -494,22 +458,29 @@ __device__ __forceinline__ void exp_pack64(const float *x, float scale, float ne
 }
 
 // P of a 128-key tile into TMEM (over S): keys 0-63, then 64-127.
-template <int NPOLY>
 __device__ __forceinline__ void exp_tile(const float *x, float scale, float negm, uint32_t tS, float (&sp)[8]) {
     {
         uint32_t pk[32];
-        exp_pack64<NPOLY>(x, scale, negm, pk, sp);
+        exp_pack64(x, scale, negm, pk, sp);
         tmem_st32(tS, reinterpret_cast<const float *>(pk));
     }
     {
         uint32_t pk[32];
-        exp_pack64<NPOLY>(x + 64, scale, negm, pk, sp);
+        exp_pack64(x + 64, scale, negm, pk, sp);
         tmem_st32(tS + 32, reinterpret_cast<const float *>(pk));
     }
 }
 
-// Persistent flash-style causal GQA attention: one CTA per SM walks the work units
-// blockIdx.x, blockIdx.x + gridDim.x, ... (heaviest first).  The K/V ring, the barrier
+// The work unit of round r for this CTA.  Units are numbered heaviest first; the rounds
+// alternate their direction over the CTAs (snake order), so that each pair of rounds
+// gives every CTA about the same causal length.
+__device__ __forceinline__ int attn_unit_of_round(int r) {
+    const int G = gridDim.x, c = blockIdx.x;
+    return r * G + ((r & 1) ? G - 1 - c : c);
+}
+
+// Persistent flash-style causal GQA attention: one CTA per SM walks one work unit per
+// round (attn_unit_of_round).  The K/V ring, the barrier
 // phases and the TMEM buffers carry over from unit to unit, so that the next unit's Q
 // and first K/V tiles load, and its Q tile is normed and rotated, while the current
 // unit's last P V and epilogue run.
@@ -572,7 +543,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t it = 0;                 // K/V ring items so far (K0 V0 K1 V1 ... per unit)
             uint32_t gs = 0;                 // steps so far (one per K/V tile pair)
             uint32_t step_arms[3] = {0u, 0u, 0u};   // phases armed on each step barrier
-            for (int u = blockIdx.x; u < p.nunits && ok; u += gridDim.x) {
+            for (int r = 0; ok; ++r) {
+                const int u = attn_unit_of_round(r);
+                if (u >= p.nunits) break;
                 AttnUnit w;
                 bool bad;
                 if (!attn_unit(p, u, w, bad)) {
@@ -655,7 +628,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t k0_uses = 0, it = 0, gs = 0;
             // failure-path test: a wait that nothing ends gives up after 100 us
             if (p.test_stall) ok = mbar_wait(BAR(BAR_NEVER), 0, p.err, 100000ull);
-            for (int u = blockIdx.x; u < p.nunits && ok; u += gridDim.x) {
+            for (int r = 0; ok; ++r) {
+                const int u = attn_unit_of_round(r);
+                if (u >= p.nunits) break;
                 AttnUnit w;
                 bool bad;
                 if (!attn_unit(p, u, w, bad)) continue;
@@ -725,15 +700,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bool pend = false;
         float pend_l = 1.f;
         long long pend_row = -1;   // element offset of this thread's output row, or -1
-        int u = blockIdx.x;
+        int rnd = 0;
         while (ok) {
             AttnUnit w;
             bool have = false, bad;
-            for (; u < p.nunits; u += gridDim.x)
+            for (;; ++rnd) {
+                const int u = attn_unit_of_round(rnd);
+                if (u >= p.nunits) break;
                 if (attn_unit(p, u, w, bad) && s < w.nslots) {
                     have = true;
                     break;
                 }
+            }
             if (have) {
                 ok = __all_sync(0xffffffffu, mbar_wait(BAR(BAR_Q_FULL + s), q_uses & 1, p.err));
                 if (!ok) break;
@@ -800,8 +778,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tmem_ld32(tS + 96, x + 96);
                 tmem_wait_ld();
                 const int lim = rowkey - j * kBN;   // keys c <= lim of this tile are visible
-                const bool masked = lim < kBN - 1;
-                if (masked) {
+                if (lim < kBN - 1) {
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
                         if (c > lim) x[c] = -INFINITY;
@@ -825,10 +802,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 l_run *= alpha;
                 const float negm = m_run == -INFINITY ? 0.f : -m_run;
                 float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                if (kExpPolyPairs > 0 && !__any_sync(0xffffffffu, masked))
-                    exp_tile<kExpPolyPairs>(x, p.scale_log2, negm, tS, sp);
-                else
-                    exp_tile<0>(x, p.scale_log2, negm, tS, sp);
+                exp_tile(x, p.scale_log2, negm, tS, sp);
                 // Rescale this row of O if the reference moved (rare after the first tiles).
                 // O is stable: P_{j-1} V_{j-1} finished before S_j was signalled.
                 if (__any_sync(0xffffffffu, need) && j > 0) {
@@ -850,7 +824,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             pend = true;
             pend_l = l_run;
             pend_row = orow;
-            u += gridDim.x;
+            ++rnd;
         }
         tc_fence_before();
     }

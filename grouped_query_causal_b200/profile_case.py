@@ -1,11 +1,14 @@
-"""Run one prefill or decode workload a few times on cuda:0 (for profilers such as ncu).
+"""Run one prefill, decode, paged-decode or projection workload a few times on cuda:0 (for
+profilers such as ncu).
 
     python -m grouped_query_causal_b200.profile_case prefill --B 2 --T 4096 --H 32 --Hkv 8 --iters 2
     python -m grouped_query_causal_b200.profile_case decode --B 16 --len 16384 --H 32 --Hkv 8 --iters 2
+    python -m grouped_query_causal_b200.profile_case paged --B 16 --len 16384 --H 32 --Hkv 8 --iters 2
+    python -m grouped_query_causal_b200.profile_case linear --M 4096 --N 6144 --K 4096 --iters 2
 
 Inputs are random on the device (their values do not matter for timing or counters);
 each iteration is one full library call: k-hat prologue + attention for prefill,
-split + merge for decode.  Prints the CUDA-event time of each iteration.
+split + merge for decode, one GEMM for linear.  Prints the CUDA-event time of each iteration.
 """
 from __future__ import annotations
 
@@ -18,7 +21,11 @@ from . import binding
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kind", choices=["prefill", "decode"])
+    ap.add_argument("kind", choices=["prefill", "decode", "paged", "linear"])
+    ap.add_argument("--M", type=int, default=4096)
+    ap.add_argument("--N", type=int, default=6144)
+    ap.add_argument("--K", type=int, default=4096)
+    ap.add_argument("--page", type=int, default=64, help="paged: rows per page")
     ap.add_argument("--B", type=int, default=2)
     ap.add_argument("--T", type=int, default=4096)
     ap.add_argument("--len", type=int, default=16384, help="decode: cached tokens per sequence")
@@ -43,6 +50,28 @@ def main(argv=None):
         run = lambda: binding.prefill(q, k, v, pos, wq, wk, out=out, workspace=ws)  # noqa: E731
         flops = a.B * a.H * 2 * D * a.T * (a.T + 1)
         unit, scale = "TFLOP/s", 1e12
+    elif a.kind == "linear":
+        x = torch.randn(a.M, a.K, device=dev, generator=g).to(torch.bfloat16)
+        w = (torch.randn(a.N, a.K, device=dev, generator=g) / a.K ** 0.5).to(torch.bfloat16)
+        out = torch.empty(a.M, a.N, dtype=torch.bfloat16, device=dev)
+        run = lambda: binding.linear(x, w, out=out)  # noqa: E731
+        flops = 2 * a.M * a.N * a.K
+        unit, scale = "TFLOP/s", 1e12
+    elif a.kind == "paged":
+        # every sequence's pages in a shuffled order over one pool
+        npg = (a.len + a.page - 1) // a.page
+        q = torch.randn(a.B, a.H, D, device=dev, generator=g).to(torch.bfloat16)
+        kp = torch.randn(a.B * npg, a.page, a.Hkv, D, device=dev, generator=g).to(torch.bfloat16)
+        vp = torch.randn(a.B * npg, a.page, a.Hkv, D, device=dev, generator=g).to(torch.bfloat16)
+        table = torch.randperm(a.B * npg, device=dev, generator=g).to(torch.int32).view(a.B, npg)
+        sl = torch.full((a.B,), a.len, dtype=torch.int32, device=dev)
+        out = torch.empty(a.B, a.H, D, device=dev)
+        ws = torch.empty(binding.decode_workspace_size(a.B, a.H, a.Hkv, a.len), dtype=torch.uint8, device=dev)
+        rope = binding.RopeConfig.make()
+        run = lambda: binding.decode_paged(q, kp, vp, table, sl, wq, a.len, rope=rope, out=out,  # noqa: E731
+                                           workspace=ws)
+        flops = a.B * a.len * a.Hkv * D * 2 * 2   # bytes, for decode
+        unit, scale = "GB/s", 1e9
     else:
         rows = a.B * a.len
         q = torch.randn(a.B, a.H, D, device=dev, generator=g).to(torch.bfloat16)
