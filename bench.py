@@ -287,8 +287,10 @@ def run_ours(args, rank, world, local_rank):
     chunked = run_packed_leg(gqa, "chunked_prefill", dev, stream, world, K, args.warmup)
     proj = run_projection_leg(gqa, dev, stream, world, K, args.warmup)
     block = run_block_leg(gqa, dev, stream, world, K, args.warmup)
-    # ---- the decode step that appends the new token first (its own timed region)
+    # ---- the decode step that appends the new token first, and the plain decode, each in
+    # its own timed region (the in-step decode runs after the long prefill)
     app = run_decode_append(gqa, dev, stream, world, K, args.warmup)
+    dalone = run_decode_alone(gqa, dec, dq, kc, vc, offs, sl, dwq, dws, dout, dev, stream, world, K, args.warmup)
     # ---- the batched decode on a paged copy of the same cache (its own timed region)
     paged = run_decode_paged(gqa, dec, dq, kc, vc, sl, dwq, dev, stream, world, K, args.warmup)
 
@@ -308,6 +310,10 @@ def run_ours(args, rank, world, local_rank):
     dec_gbs = dbytes * K / dec_s / 1e9
     traffic_attn = traffic_from_profiles("attn_fwd_kernel", PREFILL)
     traffic_dec = traffic_from_profiles("decode_split_kernel", DECODE)
+    for key, legd in (("large_prefill", extra), ("varlen_prefill", varlen), ("chunked_prefill", chunked),
+                      ("projections", proj), ("attn_block", block), ("decode_append", app),
+                      ("decode_paged", paged), ("decode_alone", dalone)):
+        legd["clocks"] = LEG_CLOCKS.get(key)
     hbm_line = lambda leg: dict(leg, roofline=dict(leg["roofline"], peak=hbm,  # noqa: E731
                                                    frac=round(leg["roofline"]["achieved"] / hbm, 4),
                                                    peak_source=f"hbm_gbs of {pk_kind}"))
@@ -366,6 +372,7 @@ def run_ours(args, rank, world, local_rank):
         "projections": tc_line(proj),
         "attn_block": tc_line(block),
         "decode_append": hbm_line(app),
+        "decode_alone": hbm_line(dalone),
         "decode_paged": hbm_line(paged),
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
@@ -375,10 +382,18 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
-def timed_calls(call, stream, world, dev, K, W, flush=None):
+LEG_CLOCKS = {}   # clocks sampled during each extra leg's timed calls, by leg name
+
+
+def timed_calls(call, stream, world, dev, K, W, flush=None, leg=None):
     """W untimed calls, then K calls each between its own pair of CUDA events on `stream`
     (with `flush`, a 256 MB write between calls, outside the events); returns the summed
-    seconds per event pair (a list), maximum over ranks."""
+    seconds per event pair (a list), maximum over ranks.  With `leg`, the SM clocks seen
+    during the timed calls go to LEG_CLOCKS[leg] (rank 0)."""
+    sampler = ClockSampler(dev.index or 0) if (leg and int(os.environ.get("RANK", "0")) == 0) else None
+    if sampler:   # started ahead of the warm-up so that nvidia-smi is sampling by the timed calls
+        sampler.start()
+        time.sleep(0.3)
     for _ in range(W):
         call(None)
     torch.cuda.synchronize()
@@ -390,6 +405,8 @@ def timed_calls(call, stream, world, dev, K, W, flush=None):
             flush.fill_(i & 255)
         evs.append(call(stream))
     torch.cuda.synchronize()
+    if sampler:
+        LEG_CLOCKS[leg] = sampler.stop()
     n = len(evs[0]) - 1
     ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(n)]
     return [x / 1e3 for x in max_over_ranks(ms, dev, world)]
@@ -427,7 +444,7 @@ def run_prefill_leg(gqa, name, dev, stream, world, K, W):
             raise RuntimeError(f"{name}: library call failed with status {st}")
         return ev
 
-    pro_s, attn_s = timed_calls(call, stream, world, dev, K, W, flush)
+    pro_s, attn_s = timed_calls(call, stream, world, dev, K, W, flush, leg=name)
     if gqa.device_status() != 0:
         raise RuntimeError(f"device status error in the {name} timing")
     flops = prefill_flops(B, T, H, D)
@@ -490,7 +507,7 @@ def run_packed_leg(gqa, name, dev, stream, world, K, W):
             raise RuntimeError(f"{name}: library call failed with status {st}")
         return ev
 
-    sec = timed_calls(call, stream, world, dev, K, W, flush)[0]
+    sec = timed_calls(call, stream, world, dev, K, W, flush, leg=name)[0]
     if gqa.device_status() != 0:
         raise RuntimeError(f"device status error in the {name} timing")
     prefix = w.prefix.tolist() if chunk else [0] * B
@@ -534,7 +551,7 @@ def run_projection_leg(gqa, dev, stream, world, K, W):
             raise RuntimeError(f"gqa_linear failed with status {st}")
         return ev
 
-    s_qkv, s_o = timed_calls(call, stream, world, dev, K, W, flush)
+    s_qkv, s_o = timed_calls(call, stream, world, dev, K, W, flush, leg="projections")
     if gqa.device_status() != 0:
         raise RuntimeError("device status error in the projection timing")
     f_qkv, f_o = 2 * M * Nq * hidden, 2 * M * hidden * hidden
@@ -580,7 +597,7 @@ def run_block_leg(gqa, dev, stream, world, K, W):
             raise RuntimeError(f"gqa_attn_block_prefill failed with status {st}")
         return ev
 
-    sec = timed_calls(call, stream, world, dev, K, W, flush)[0]
+    sec = timed_calls(call, stream, world, dev, K, W, flush, leg="attn_block")[0]
     if gqa.device_status() != 0:
         raise RuntimeError("device status error in the attention-block timing")
     N = B * T
@@ -592,6 +609,41 @@ def run_block_leg(gqa, dev, stream, world, K, W):
                         "RoPE, causal GQA attention, o_proj", "gpu_launches": 4 * K,
             "roofline": {"bound": "tensor", "achieved": round(flops * K / sec / 1e12, 2), "unit": "TFLOP/s",
                          "traffic": None, "kernel": "gemm_kernel, k_prologue_kernel, attn_fwd_kernel, gemm_kernel"}}
+
+
+def run_decode_alone(gqa, dec, dq, kc, vc, offs, sl, dwq, dws, dout, dev, stream, world, K, W):
+    """gqa_attn_decode on the batched decode workload in its own timed region (CUDA events
+    around each call, L2 flushed between calls), away from the prefill of the step."""
+    lib = gqa.load()
+    sh = stream.cuda_stream
+    B, H, D = dec.q.shape
+    Hkv = dec.k_cache.shape[1]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ptr = lambda t: t.data_ptr()  # noqa: E731
+
+    def call(st_):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)] if st_ is not None else None
+        if ev:
+            ev[0].record(st_)
+        st = lib.gqa_attn_decode(ptr(dq), ptr(kc), ptr(vc), ptr(offs), ptr(sl), None, ptr(dwq), dec.theta, dec.eps,
+                                 ptr(dout), B, H, Hkv, D, dec.max_len, ptr(dws), dws.numel(), sh)
+        if ev:
+            ev[1].record(st_)
+        if st != 0:
+            raise RuntimeError(f"gqa_attn_decode failed with status {st}")
+        return ev
+
+    sec = timed_calls(call, stream, world, dev, K, W, flush, leg="decode_alone")[0]
+    if gqa.device_status() != 0:
+        raise RuntimeError("device status error in the decode timing")
+    nbytes = decode_bytes(dec.seqlens.tolist(), H, Hkv, D)
+    del flush
+    return {"value": round(whole_job_rate(nbytes * K, world, sec) / 1e9, 1), "unit": "GB/s",
+            "ms": round(1e3 * sec / K, 4), "workload": WORKLOAD_TEXT[DECODE], "bytes_per_call": nbytes,
+            "gpu_launches": 2 * K, "l2": "256 MB written between timed calls",
+            "roofline": {"bound": "hbm", "achieved": round(nbytes * K / sec / 1e9, 1), "unit": "GB/s",
+                         "traffic": traffic_from_profiles("decode_split_kernel", DECODE),
+                         "kernel": "decode_split_kernel + decode_merge_kernel (one call)"}}
 
 
 def run_decode_append(gqa, dev, stream, world, K, W):
@@ -625,7 +677,7 @@ def run_decode_append(gqa, dev, stream, world, K, W):
             raise RuntimeError(f"gqa_attn_decode_append failed with status {st}")
         return ev
 
-    sec = timed_calls(call, stream, world, dev, K, W, flush)[0]
+    sec = timed_calls(call, stream, world, dev, K, W, flush, leg="decode_append")[0]
     if gqa.device_status() != 0:
         raise RuntimeError("device status error in the append-step timing")
     nbytes = decode_append_bytes(w.seqlens.tolist(), H, Hkv, D)
@@ -697,7 +749,7 @@ def run_decode_paged(gqa, dec, dq, kc, vc, sl, dwq, dev, stream, world, K, W, pa
             raise RuntimeError(f"gqa_attn_decode_paged failed with status {st}")
         return ev
 
-    sec = timed_calls(call, stream, world, dev, K, W, flush)[0]
+    sec = timed_calls(call, stream, world, dev, K, W, flush, leg="decode_paged")[0]
     if gqa.device_status() != 0:
         raise RuntimeError("device status error in the paged-decode timing")
     nbytes = decode_bytes(lens, H, Hkv, D)

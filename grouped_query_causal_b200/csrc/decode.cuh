@@ -117,7 +117,7 @@ __device__ __forceinline__ int decode_head_of_lane(int lane) {
 }
 
 template <int HG, bool PAGED>
-__global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(128, (HG <= 4 ? 4 : 1)) decode_split_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int LG = HeadsLog2<HG>::value;
     __shared__ __align__(16) float sq[HG][kHeadDim];
     __shared__ __align__(16) float sbuf[4][kWarpKeys * HG];   // scores / probabilities, then partial O
@@ -159,17 +159,11 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
             if (warp_bad) kw1 = kw0;
         }
     }
-    // Physical row of the 16-row batch that starts at logical row `base` (16-aligned: a
-    // batch never crosses a page, whose size is a multiple of 16).  Warp-uniform.
-    auto batch_row = [&](int base) -> long long {
-        if constexpr (PAGED) {
-            const int pg = base / p.page_size;
-            const int id = __shfl_sync(0xffffffffu, my_page, pg - wpg0);
-            return static_cast<long long>(id) * p.page_size + (base - pg * p.page_size);
-        } else {
-            return base;
-        }
-    };
+    // Paged: the next 16-row batch's page (relative to wpg0) and row inside that page.
+    // The batches of a sweep are loaded in order, 16 rows apart, and a batch never crosses
+    // a page (page_size is a multiple of 16), so the cursor advances without a division.
+    const int off0 = PAGED ? kw0 - wpg0 * p.page_size : 0;
+    int cur_pg = 0, cur_off = off0;
 
     const int sub = lane & 15;    // elements 8*sub .. 8*sub+7 of a row
     const int rsel = lane >> 4;   // which row of the pair
@@ -182,12 +176,18 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     const int my_head = decode_head_of_lane<HG>(lane);
 
     // Loads of the 16-row batch that starts at logical row `base` (rows past kw1 read
-    // as zero).  Contiguous caches index rows directly; paged ones look the page up once
-    // per batch.
+    // as zero).  Contiguous caches index rows directly; paged ones take the page id of the
+    // cursor from the lane that holds it.
     auto load_batch = [&](const uint16_t *rbase, int base, uint4 (&dst)[kRowPairs]) {
         if constexpr (PAGED) {
             if (base >= kw1) return;
-            const long long pr = batch_row(base);
+            const int id = __shfl_sync(0xffffffffu, my_page, cur_pg);   // warp-uniform
+            const long long pr = static_cast<long long>(id) * p.page_size + cur_off;
+            cur_off += 2 * kRowPairs;
+            if (cur_off == p.page_size) {
+                cur_off = 0;
+                ++cur_pg;
+            }
 #pragma unroll
             for (int u = 0; u < kRowPairs; ++u) {
                 const int row = base + 2 * u + rsel;
@@ -269,6 +269,8 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
         }
     }
     uint4 vn[kRowPairs];
+    cur_pg = 0;   // the V sweep reads the same rows again
+    cur_off = off0;
     load_batch(vbase, kw0, vn);
     __syncwarp();
 

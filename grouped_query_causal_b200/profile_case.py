@@ -5,6 +5,10 @@ profilers such as ncu).
     python -m grouped_query_causal_b200.profile_case decode --B 16 --len 16384 --H 32 --Hkv 8 --iters 2
     python -m grouped_query_causal_b200.profile_case paged --B 16 --len 16384 --H 32 --Hkv 8 --iters 2
     python -m grouped_query_causal_b200.profile_case linear --M 4096 --N 6144 --K 4096 --iters 2
+    python -m grouped_query_causal_b200.profile_case workload --name long_context_prefill --iters 2
+
+`workload` runs one of the named synthetic workloads exactly as the benchmark does (same
+inputs and launch), so that counters taken on it are per bench launch.
 
 Inputs are random on the device (their values do not matter for timing or counters);
 each iteration is one full library call: k-hat prologue + attention for prefill,
@@ -21,7 +25,8 @@ from . import binding
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kind", choices=["prefill", "decode", "paged", "linear"])
+    ap.add_argument("kind", choices=["prefill", "decode", "paged", "linear", "workload"])
+    ap.add_argument("--name", default="long_context_prefill", help="workload: a name from synthetic.WORKLOADS")
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=6144)
     ap.add_argument("--K", type=int, default=4096)
@@ -50,6 +55,30 @@ def main(argv=None):
         run = lambda: binding.prefill(q, k, v, pos, wq, wk, out=out, workspace=ws)  # noqa: E731
         flops = a.B * a.H * 2 * D * a.T * (a.T + 1)
         unit, scale = "TFLOP/s", 1e12
+    elif a.kind == "workload":
+        from . import synthetic
+        w = synthetic.make(a.name)
+        kind = synthetic.WORKLOADS[a.name]["kind"]
+        if kind == "prefill":
+            t = [x.to(dev) for x in (w.q, w.k, w.v, w.pos, w.wq, w.wk)]
+            B, T, H, D = w.q.shape
+            Hkv = w.k.shape[2]
+            out = torch.empty(B, T, H, D, device=dev)
+            ws = torch.empty(binding.prefill_workspace_size(B, T, H, Hkv), dtype=torch.uint8, device=dev)
+            run = lambda: binding.prefill(*t, w.theta, w.eps, out=out, workspace=ws)  # noqa: E731
+            flops = B * H * 2 * D * T * (T + 1)
+            unit, scale = "TFLOP/s", 1e12
+        elif kind == "decode":
+            q, kc, vc, offs, sl, dwq = (x.to(dev) for x in (w.q, w.k_cache, w.v_cache, w.offsets, w.seqlens, w.wq))
+            B, H, D = w.q.shape
+            Hkv = w.k_cache.shape[1]
+            out = torch.empty(B, H, D, device=dev)
+            ws = torch.empty(binding.decode_workspace_size(B, H, Hkv, w.max_len), dtype=torch.uint8, device=dev)
+            run = lambda: binding.decode(q, kc, vc, offs, sl, dwq, w.max_len, out=out, workspace=ws)  # noqa: E731
+            flops = int(w.seqlens.sum()) * Hkv * D * 2 * 2
+            unit, scale = "GB/s", 1e9
+        else:
+            raise SystemExit(f"workload {a.name}: kind {kind} is not run here")
     elif a.kind == "linear":
         x = torch.randn(a.M, a.K, device=dev, generator=g).to(torch.bfloat16)
         w = (torch.randn(a.N, a.K, device=dev, generator=g) / a.K ** 0.5).to(torch.bfloat16)
