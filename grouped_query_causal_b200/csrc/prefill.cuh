@@ -206,12 +206,14 @@ __global__ void __launch_bounds__(256) k_prologue_kernel(const __grid_constant__
 // ============================================================================ attention
 constexpr int kBM = 128;                       // query rows per tile (one per softmax thread)
 constexpr int kBN = 128;                       // keys per K/V tile
-constexpr int kStages = 5;                     // K/V ring depth (tiles)
+constexpr int kStages = 4;                     // K/V ring depth (tiles)
 constexpr uint32_t kTileBytes = 128 * 128 * 2; // one bf16 128x128 tile
 constexpr uint32_t kBoxBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-byte swizzle span)
+constexpr uint32_t kStageBytes = 128 * 32 * 4; // epilogue staging per head: 128 rows x 32 fp32 columns
 constexpr uint32_t kOffQ = 0;                                   // 2 tiles
 constexpr uint32_t kOffKV = kOffQ + 2 * kTileBytes;             // kStages tiles
-constexpr uint32_t kOffBar = kOffKV + kStages * kTileBytes;
+constexpr uint32_t kOffStage = kOffKV + kStages * kTileBytes;   // 2 staging buffers
+constexpr uint32_t kOffBar = kOffStage + 2 * kStageBytes;
 enum {
     BAR_Q_FULL = 0,    // [2] TMA -> softmax WG: raw Q tile landed
     BAR_Q_READY = 2,   // [2] softmax WG -> MMA: Q tile normed + rotated in place (128 arrivals)
@@ -225,7 +227,8 @@ enum {
     BAR_DRAIN = 15 + kStages,        // MMA drains its own work before TMEM is released
     BAR_STEP_FULL = 16 + kStages,    // [3] TMA -> MMA: V_j and K_{j+1} landed (one wait per tile)
     BAR_NEVER = 19 + kStages,        // never signalled: the failure-path test waits on it
-    NUM_BARS = 20 + kStages
+    BAR_STG = 20 + kStages,          // [2] softmax WG internal: epilogue chunk staged / copied out (128 arrivals)
+    NUM_BARS = 22 + kStages
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + NUM_BARS * 8;
 constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align the base to 1024
@@ -517,6 +520,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int i = 0; i < 3; ++i) mbar_init(BAR(BAR_STEP_FULL + i), 1);
         mbar_init(BAR(BAR_DRAIN), 1);
         mbar_init(BAR(BAR_NEVER), 1);
+        for (int i = 0; i < 2; ++i) mbar_init(BAR(BAR_STG + i), kBM);
         fence_mbarrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -696,10 +700,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t tO = tmem + lane_base + 256 + s * 128;
         bool ok = true;
         uint32_t q_uses = 0, tiles = 0, units = 0;
-        // the unit whose epilogue is pending
+        // the unit whose epilogue is pending: its query rows, their count and the head
         bool pend = false;
         float pend_l = 1.f;
-        long long pend_row = -1;   // element offset of this thread's output row, or -1
+        long long pend_q0 = 0;
+        int pend_rows = 0, pend_hq = 0;
+        const uint32_t stg = sbase + kOffStage + s * kStageBytes;   // this head's staging buffer
+        const int wr = warp & 3;                                    // warp within the warpgroup
         int rnd = 0;
         while (ok) {
             AttnUnit w;
@@ -730,37 +737,54 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 ++units;
                 tc_fence_after();
                 const float inv_l = 1.0f / pend_l;
+                // O / l in four chunks of 32 columns: each thread stages its row (16-byte
+                // granules swizzled by row, so that 8 consecutive rows hit distinct banks),
+                // then each warp copies 4 whole rows per instruction to global memory.
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     float o[32];
                     tmem_ld32(tO + 32 * c, o);
                     tmem_wait_ld();
-                    if (pend_row >= 0) {
-                        if (p.out_bf16) {
-                            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + pend_row + 32 * c);
 #pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                dst[e] = make_uint4(pack_bf16x2(o[8 * e] * inv_l, o[8 * e + 1] * inv_l),
-                                                    pack_bf16x2(o[8 * e + 2] * inv_l, o[8 * e + 3] * inv_l),
-                                                    pack_bf16x2(o[8 * e + 4] * inv_l, o[8 * e + 5] * inv_l),
-                                                    pack_bf16x2(o[8 * e + 6] * inv_l, o[8 * e + 7] * inv_l));
-                        } else {
-                            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + pend_row + 32 * c);
+                    for (int g = 0; g < 8; ++g)
+                        st_shared_v4(stg + r * 128 + ((g ^ (r & 7)) << 4),
+                                     make_uint4(__float_as_uint(o[4 * g] * inv_l), __float_as_uint(o[4 * g + 1] * inv_l),
+                                                __float_as_uint(o[4 * g + 2] * inv_l),
+                                                __float_as_uint(o[4 * g + 3] * inv_l)));
+                    // every row of the chunk is staged (the barrier completes twice a chunk, so
+                    // this wait is on even phases and the one below on odd ones)
+                    mbar_arrive(BAR(BAR_STG + s));
+                    ok = __all_sync(0xffffffffu, mbar_wait_hint(BAR(BAR_STG + s), 0, 20u, p.err));
+                    if (!ok) break;
+                    const int g = lane & 7;
 #pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                dst[e] = make_float4(o[4 * e] * inv_l, o[4 * e + 1] * inv_l, o[4 * e + 2] * inv_l,
-                                                     o[4 * e + 3] * inv_l);
+                    for (int it = 0; it < 8; ++it) {
+                        const int row = wr * 32 + it * 4 + (lane >> 3);
+                        const uint4 v = ld_shared_v4(stg + row * 128 + ((g ^ (row & 7)) << 4));
+                        if (row < pend_rows) {
+                            const long long e = ((pend_q0 + row) * p.H + pend_hq) * kHeadDim + 32 * c + 4 * g;
+                            if (p.out_bf16)
+                                *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(p.out) + e) =
+                                    make_uint2(pack_bf16x2(__uint_as_float(v.x), __uint_as_float(v.y)),
+                                               pack_bf16x2(__uint_as_float(v.z), __uint_as_float(v.w)));
+                            else
+                                *reinterpret_cast<uint4 *>(static_cast<float *>(p.out) + e) = v;
                         }
                     }
+                    mbar_arrive(BAR(BAR_STG + s));   // the staging buffer is free again
+                    ok = __all_sync(0xffffffffu, mbar_wait_hint(BAR(BAR_STG + s), 1, 20u, p.err));
+                    if (!ok) break;
                 }
+                if (!ok) break;
                 tc_fence_before();
                 mbar_arrive(BAR(BAR_O_EMPTY + s));
                 pend = false;
             }
             if (!have) break;
 
-            // what the epilogue needs, computed now so that only n_kv and rowkey stay live
-            const long long orow = r < w.rows ? ((w.q0 + r) * p.H + w.hq0 + s) * kHeadDim : -1;
+            // what the epilogue needs, copied now so that only n_kv and rowkey stay live
+            const long long uq0 = w.q0;
+            const int urows = w.rows, uhq = w.hq0 + s;
             const int n_kv = w.n_kv;
             const int rowkey = w.key0 + r;   // token index of this row: sees keys 0 .. rowkey
             float m_run = -INFINITY;   // running max of scaled scores (base 2), possibly stale by < 8
@@ -823,7 +847,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             pend = true;
             pend_l = l_run;
-            pend_row = orow;
+            pend_q0 = uq0;
+            pend_rows = urows;
+            pend_hq = uhq;
             ++rnd;
         }
         tc_fence_before();
