@@ -271,6 +271,7 @@ struct AttnGeom {
     bool out_bf16 = false;             // bf16 output (the input of the output projection)
     const int64_t *cu_q = nullptr, *kv_off = nullptr;
     const int32_t *prefix = nullptr;
+    long long max_prefix = 0;          // host-side bound on the cached keys before a chunk (scheduling only)
 };
 
 // Enqueue the attention kernel (arguments already validated).
@@ -312,6 +313,18 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
     if (units <= 0) return GQA_OK;
     if (units > 0x7fffffffLL) return GQA_ERR_INVALID_ARG;
     ap.nunits = static_cast<int>(units);
+    // KV groups per band: bands of equal size, as few as keep each band's K/V (the longest
+    // sequence's keys, K and V in bf16) within ~80 MB of the 126 MB L2, which also carries Q,
+    // the output and the RoPE table.  Equal sizes keep the last band from being a short tail of
+    // long units.
+    {
+        const long long groups = static_cast<long long>(gm.B) * Hkv;
+        const long long keys = static_cast<long long>(gm.T) + gm.max_prefix;
+        const long long kv_bytes = std::max(1LL, keys * kHeadDim * 2 * 2);
+        const long long fit = std::max(1LL, (80LL << 20) / kv_bytes);
+        const long long nbands = (groups + fit - 1) / fit;
+        ap.band = static_cast<int>(std::max(1LL, (groups + nbands - 1) / nbands));
+    }
     const unsigned grid = static_cast<unsigned>(std::min<long long>(units, attn_sm_count()));
     if (rs.pairing == kPairHalf)
         attn_fwd_kernel<kPairHalf><<<grid, kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
@@ -542,6 +555,7 @@ extern "C" gqa_status gqa_attn_prefill_chunk(const void *q, const void *k, const
     gm.cu_q = cu_seqlens;
     gm.kv_off = cache_offsets;
     gm.prefix = prefix_len;
+    gm.max_prefix = cache_rows / std::max(1, B);   // an average; only the schedule depends on it
     return launch_attention(q, k_cache, v_cache, pos, table, qnorm_w, rs, eps, out, gm, H, Hkv, st);
 }
 

@@ -260,6 +260,7 @@ struct AttnParams {
     long long nq_rows;     // rows of q / pos / out
     long long nkv_rows;    // rows of k-hat / v
     int B, T, H, Hkv, hpg, nqb, npairs, nunits;
+    int band;              // KV groups (sequence, KV head) scheduled together: their K/V fit in L2
     int out_bf16;          // 1: the output is rounded to bf16 (the input of the output projection)
     int test_stall;        // 1 (failure-path test only): the MMA thread first waits on BAR_NEVER
     float eps;
@@ -268,7 +269,10 @@ struct AttnParams {
 };
 
 // One work unit: a 128-row query block of one sequence and a pair of query heads of a
-// KV group.  Units are numbered heaviest (latest query block) first.
+// KV group.  Units are numbered band by band, where a band is `band` consecutive KV groups
+// (sequence, KV head) whose K/V together fit in L2, and inside a band heaviest (latest query
+// block) first: the CTAs running at the same time then read the same K/V tiles, which stay
+// in L2, instead of streaming every group's K/V through it.
 struct AttnUnit {
     long long q0;     // query row of block row 0 (q0(b) + qb * 128)
     long long kv0;    // K/V row of key 0
@@ -282,13 +286,18 @@ struct AttnUnit {
 // sequence, or a sequence whose device-side geometry is out of range).
 __device__ __forceinline__ bool attn_unit(const AttnParams &p, int u, AttnUnit &w, bool &bad) {
     bad = false;
-    const int per_qb = p.B * p.Hkv * p.npairs;
-    const int qb = p.nqb - 1 - u / per_qb;
-    int rem = u % per_qb;
+    // u -> (band of KV groups, query block latest first, group in the band, head pair)
+    const int ngroups = p.B * p.Hkv;
+    const int per_band = p.band * p.nqb * p.npairs;
+    const int band = u / per_band;
+    const int gb = min(p.band, ngroups - band * p.band);   // groups in this band
+    int rem = u - band * per_band;
+    const int qb = p.nqb - 1 - rem / (gb * p.npairs);
+    rem %= gb * p.npairs;
     const int pair = rem % p.npairs;
-    rem /= p.npairs;
-    w.g = rem % p.Hkv;
-    w.b = rem / p.Hkv;
+    const int gi = band * p.band + rem / p.npairs;
+    w.g = gi % p.Hkv;
+    w.b = gi / p.Hkv;
     long long q0 = static_cast<long long>(w.b) * p.T, len = p.T;
     if (p.cu_q != nullptr) {
         q0 = p.cu_q[w.b];
