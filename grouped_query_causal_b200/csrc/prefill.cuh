@@ -227,8 +227,7 @@ enum {
     BAR_DRAIN = 15 + kStages,        // MMA drains its own work before TMEM is released
     BAR_STEP_FULL = 16 + kStages,    // [3] TMA -> MMA: V_j and K_{j+1} landed (one wait per tile)
     BAR_NEVER = 19 + kStages,        // never signalled: the failure-path test waits on it
-    BAR_STG = 20 + kStages,          // [2] softmax WG internal: epilogue chunk staged / copied out (128 arrivals)
-    NUM_BARS = 22 + kStages
+    NUM_BARS = 20 + kStages
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + NUM_BARS * 8;
 constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align the base to 1024
@@ -360,7 +359,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
 template <int PAIRING>
 __device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, const float *table, long long n,
                                                 const float *wq, float eps, const RopeFreqs &rf) {
-    float ss = 0.f;
+    float sq8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // eight short chains, not one of 128
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
         const uint4 v = ld_shared_v4(tile_chunk_addr(sq, r, c));
@@ -368,10 +367,11 @@ __device__ __forceinline__ void transform_q_row(uint32_t sq, int r, int ps, cons
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const float a = bf16lo(u[i]), b = bf16hi(u[i]);
-            ss = fmaf(a, a, ss);
-            ss = fmaf(b, b, ss);
+            sq8[2 * i] = fmaf(a, a, sq8[2 * i]);
+            sq8[2 * i + 1] = fmaf(b, b, sq8[2 * i + 1]);
         }
     }
+    const float ss = ((sq8[0] + sq8[1]) + (sq8[2] + sq8[3])) + ((sq8[4] + sq8[5]) + (sq8[6] + sq8[7]));
     const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + eps);
     if constexpr (PAIRING == kPairHalf) {
         // rotate-half: chunk c (elements 8c .. 8c+7, c < 8) meets chunk c + 8, at the
@@ -529,7 +529,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int i = 0; i < 3; ++i) mbar_init(BAR(BAR_STEP_FULL + i), 1);
         mbar_init(BAR(BAR_DRAIN), 1);
         mbar_init(BAR(BAR_NEVER), 1);
-        for (int i = 0; i < 2; ++i) mbar_init(BAR(BAR_STG + i), kBM);
         fence_mbarrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -748,7 +747,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const float inv_l = 1.0f / pend_l;
                 // O / l in four chunks of 32 columns: each thread stages its row (16-byte
                 // granules swizzled by row, so that 8 consecutive rows hit distinct banks),
-                // then each warp copies 4 whole rows per instruction to global memory.
+                // then its warp copies the warp's 32 rows out, 4 whole rows per instruction.
+                // A warp reads back only rows it wrote, so a warp-level sync orders the two.
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     float o[32];
@@ -760,11 +760,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                      make_uint4(__float_as_uint(o[4 * g] * inv_l), __float_as_uint(o[4 * g + 1] * inv_l),
                                                 __float_as_uint(o[4 * g + 2] * inv_l),
                                                 __float_as_uint(o[4 * g + 3] * inv_l)));
-                    // every row of the chunk is staged (the barrier completes twice a chunk, so
-                    // this wait is on even phases and the one below on odd ones)
-                    mbar_arrive(BAR(BAR_STG + s));
-                    ok = __all_sync(0xffffffffu, mbar_wait_hint(BAR(BAR_STG + s), 0, 20u, p.err));
-                    if (!ok) break;
+                    __syncwarp();
                     const int g = lane & 7;
 #pragma unroll
                     for (int it = 0; it < 8; ++it) {
@@ -780,9 +776,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                 *reinterpret_cast<uint4 *>(static_cast<float *>(p.out) + e) = v;
                         }
                     }
-                    mbar_arrive(BAR(BAR_STG + s));   // the staging buffer is free again
-                    ok = __all_sync(0xffffffffu, mbar_wait_hint(BAR(BAR_STG + s), 1, 20u, p.err));
-                    if (!ok) break;
+                    __syncwarp();   // the warp's rows of the staging buffer are free again
                 }
                 if (!ok) break;
                 tc_fence_before();
