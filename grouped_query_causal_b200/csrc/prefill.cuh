@@ -483,6 +483,10 @@ __device__ __forceinline__ void exp_tile(const float *x, float scale, float negm
     }
 }
 
+__device__ __forceinline__ float max8(const float (&m)[8]) {
+    return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
 // The work unit of round r for this CTA.  Units are numbered heaviest first; the rounds
 // alternate their direction over the CTAs (snake order), so that each pair of rounds
 // gives every CTA about the same causal length.
@@ -810,37 +814,59 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     for (int c = 0; c < 128; ++c)
                         if (c > lim) x[c] = -INFINITY;
                 }
-                // row max with eight independent partial maxima (short dependency chains)
-                float mp[8];
+                // The first tile sets the reference max from its own maximum (key 0 is visible
+                // to every row, so it is finite).  Later tiles compute P against the current
+                // reference straight away: a score more than 2^8 above it would make its own
+                // term, and so the tile's sum, at least 2^8, so only a tile sum >= 250 calls
+                // for the exact maximum and, if it grew by more than 2^8, a second pass.  The
+                // reference, P and l are exactly those of finding the maximum first.
+                if (j == 0) {
+                    float m0[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) mp[e] = x[e];
+                    for (int e = 0; e < 8; ++e) m0[e] = x[e];
 #pragma unroll
-                for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
-                const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-                const float m_new = fmaxf(m_run, mx * p.scale_log2);
-                // Only move the reference max when it grows by more than 2^8; the final
-                // O / l is exact either way because O and l always share the reference.
-                // A row with no visible key yet (only past the end of its sequence) keeps
-                // -inf and adds nothing.
-                const bool need = m_new > m_run + 8.0f;
-                const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
-                if (need) m_run = m_new;
-                l_run *= alpha;
-                const float negm = m_run == -INFINITY ? 0.f : -m_run;
+                    for (int c = 8; c < 128; ++c) m0[c & 7] = fmaxf(m0[c & 7], x[c]);
+                    m_run = max8(m0) * p.scale_log2;
+                }
                 float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                exp_tile(x, p.scale_log2, negm, tS, sp);
-                // Rescale this row of O if the reference moved (rare after the first tiles).
-                // O is stable: P_{j-1} V_{j-1} finished before S_j was signalled.
-                if (__any_sync(0xffffffffu, need) && j > 0) {
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        float o[32];
-                        tmem_ld32(tO + 32 * c, o);
-                        tmem_wait_ld();
+                exp_tile(x, p.scale_log2, m_run == -INFINITY ? 0.f : -m_run, tS, sp);
+                if (__any_sync(0xffffffffu, ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])) >=
+                                                250.0f || m_run == -INFINITY)) {
+                    float mp[8];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                        tmem_st32(tO + 32 * c, o);
+                    for (int e = 0; e < 8; ++e) mp[e] = x[e];
+#pragma unroll
+                    for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+                    const float m_new = fmaxf(m_run, max8(mp) * p.scale_log2);
+                    // A row with no visible key yet (only past the end of its sequence) keeps
+                    // -inf and adds nothing.
+                    const bool need = m_new > m_run + 8.0f;
+                    if (__any_sync(0xffffffffu, need)) {
+                        // Move the reference, rescale l and this row of O (O is stable:
+                        // P_{j-1} V_{j-1} finished before S_j was signalled), and write P again.
+                        const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
+                        if (need) m_run = m_new;
+                        l_run *= alpha;
+                        if (need) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) sp[e] = 0.f;
+                        }
+                        // lanes that keep their reference recompute the same P and sums
+                        float sq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        exp_tile(x, p.scale_log2, m_run == -INFINITY ? 0.f : -m_run, tS, sq);
+                        if (need) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) sp[e] = sq[e];
+                        }
+#pragma unroll 1
+                        for (int c = 0; c < 4; ++c) {
+                            float o[32];
+                            tmem_ld32(tO + 32 * c, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                            tmem_st32(tO + 32 * c, o);
+                        }
                     }
                 }
                 tmem_wait_st();
