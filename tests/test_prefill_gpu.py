@@ -103,6 +103,22 @@ def test_long_context_prefill_strided_rows(gqa):
     assert_close(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, f"long_context, {len(rows)} rows")
 
 
+def test_unequal_bands_odd_groups_strided_rows(gqa):
+    """B=1, T=24539 (a ragged last tile), H=21, Hkv=7: each KV group's K/V (12.6 MB) lets six
+    groups share L2, so the seven groups run as two bands of 4 and 3, and with 3 query heads
+    per group the second head pair of every group has a single head.  Every 128th row of
+    every head (phase shifted per head), tile edges, and the last 128 rows of the heads of
+    the last group (the short second band's longest sweeps)."""
+    B, T, H, Hkv = 1, 24539, 21, 7
+    inp = synthetic.prefill_inputs(B, T, H, Hkv, seed=5)
+    got = _run(gqa, inp)
+    assert np.isfinite(got).all()
+    rows = strided_rows(B, T, H, 128, edges=(0, 1, 127, 128, 129, 12287, 12288, T - 129, T - 128, T - 1),
+                        tail_heads=range(18, 21), tail=128)
+    ref = oracle.prefill_rows(*oracle_prefill_args(inp), rows)
+    assert_close(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, f"unequal bands, {len(rows)} rows")
+
+
 def test_empty_problem_is_noop(gqa):
     dev = "cuda"
     q = torch.empty((0, 5, 4, 128), dtype=torch.bfloat16, device=dev)
