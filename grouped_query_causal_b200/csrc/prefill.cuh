@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t k0_uses = 0;            // units so far (first K tiles)
             uint32_t it = 0;                 // K/V ring items so far (K0 V0 K1 V1 ... per unit)
             uint32_t gs = 0;                 // steps so far (one per K/V tile pair)
-            uint32_t step_arms[3] = {0u, 0u, 0u};   // phases armed on each step barrier
+            uint32_t armed = 0;                     // steps armed so far (step k on barrier k % 3)
             for (int r = 0; ok; ++r) {
                 const int u = attn_unit_of_round(r);
                 if (u >= p.nunits) break;
@@ -572,7 +572,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     for (long long blk = w.q0 >> 7; blk <= ((w.q0 + w.rows - 1) >> 7); ++blk)
                         prefetch_l2_bulk(p.rope_cs + rope_table_index(blk << 7, 0) * 4, 32 * 128 * 16);
                 }
-                for (int s = 0; s < w.nslots && ok; ++s) {
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {   // unrolled: the per-slot counters stay in registers
+                    if (s >= w.nslots || !ok) break;
                     // the slot is free once the previous unit's last Q K^T on it has finished
                     if (q_uses[s] > 0 && !mbar_wait(BAR(BAR_Q_EMPTY + s), (q_uses[s] - 1) & 1, p.err)) {
                         ok = false;
@@ -602,7 +604,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         ++k0_uses;
                     } else if (k & 1) {
                         mbar_arrive_expect_tx(bar, j + 1 < w.n_kv ? 2 * kTileBytes : kTileBytes);
-                        ++step_arms[(gs + j) % 3];
+                        ++armed;
                     }
                     tma_load_3d(dst, m, 0, w.g, row, bar);
                     tma_load_3d(dst + kBoxBytes, m, 64, w.g, row, bar);
@@ -617,8 +619,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int s = 0; s < 2; ++s)
                     if (q_uses[s] > 0) mbar_wait(BAR(BAR_Q_FULL + s), (q_uses[s] - 1) & 1, p.err);
                 if (k0_uses > 0) mbar_wait(BAR(BAR_K0_FULL), (k0_uses - 1) & 1, p.err);
-                for (int i = 0; i < 3; ++i)
-                    if (step_arms[i] > 0) mbar_wait(BAR(BAR_STEP_FULL + i), (step_arms[i] - 1) & 1, p.err);
+                for (int i = 0; i < 3; ++i) {
+                    // steps 0 .. armed-1 were armed in order, so barrier i holds every third
+                    const uint32_t arms = armed / 3 + (static_cast<uint32_t>(i) < armed % 3 ? 1u : 0u);
+                    if (arms > 0) mbar_wait(BAR(BAR_STEP_FULL + i), (arms - 1) & 1, p.err);
+                }
             }
         }
         __syncwarp();
@@ -653,7 +658,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const uint32_t k0_item = it;
                 if (!MMA_WAIT(BAR(BAR_K0_FULL), k0_uses & 1)) { ok = false; break; }
                 ++k0_uses;
-                for (int s = 0; s < w.nslots; ++s) {
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {   // unrolled: the per-head counters stay in registers
+                    if (s >= w.nslots) break;
                     if (!MMA_WAIT(BAR(BAR_Q_READY + s), q_uses[s] & 1)) { ok = false; break; }
                     ++q_uses[s];
                     tc_fence_after();
@@ -667,7 +674,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     const uint32_t iv = k0_item + 2 * j + 1, ik = k0_item + 2 * j + 2;   // ring items of V_j, K_{j+1}
                     const bool more = j + 1 < w.n_kv;
                     if (!MMA_WAIT(BAR(BAR_STEP_FULL + (gs + j) % 3), ((gs + j) / 3) & 1)) { ok = false; break; }
-                    for (int s = 0; s < w.nslots; ++s) {
+#pragma unroll
+                    for (int s = 0; s < 2; ++s) {
+                        if (s >= w.nslots) break;
                         if (!MMA_WAIT(BAR(BAR_P_FULL + s), tiles[s] & 1)) { ok = false; break; }
                         ++tiles[s];
                         if (j == 0 && units[s] > 0 && !MMA_WAIT(BAR(BAR_O_EMPTY + s), (units[s] - 1) & 1)) {
