@@ -4,15 +4,15 @@
 //      bf16 k-hat.  Every K tile is read by all later query blocks of its sequence and
 //      by every query head of its group, so transforming it once is cheaper than
 //      redoing it in each reader (that would multiply the work by h * (T/128) / 2).
-//  (2) attn_fwd_kernel: flash-style causal GQA attention.  One CTA owns one
-//      (batch, KV head, 128-token query block, pair of query heads of the group).
-//      The raw Q tiles are loaded by TMA and normed + rotated in registers in place
-//      (the fused q prologue); K-hat/V tiles stream through a TMA ring and serve both
-//      query heads of the pair; S = Q K^T and O += P V run on the 5th-generation
-//      tensor cores (tcgen05.mma, fp32 accumulators in TMEM); the online softmax
-//      runs in two warpgroups (one per head of the pair, ping-ponging with the tensor
-//      core) with one query row per thread; causal tiles above the diagonal are never
-//      loaded.
+//  (2) attn_fwd_kernel: flash-style causal GQA attention, persistent: one CTA per SM
+//      walks work units, a unit being (sequence, KV head, 128-token query block, pair
+//      of query heads of the group).  The raw Q tiles are loaded by TMA and normed +
+//      rotated in registers in place (the fused q prologue); K-hat/V tiles stream
+//      through a TMA ring and serve both query heads of the pair; S = Q K^T and
+//      O += P V run on the 5th-generation tensor cores (tcgen05.mma, fp32 accumulators
+//      in TMEM); the online softmax runs in two warpgroups (one per head of the pair,
+//      ping-ponging with the tensor core) with one query row per thread; causal tiles
+//      above the diagonal are never loaded.
 //  Both kernels take the RoPE pairing (adjacent or rotate-half) as a template
 //  parameter; the frequencies (plain or scaled) arrive precomputed from the host.
 //
