@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "gqa_attn.h"
 #include "decode.cuh"
@@ -275,6 +276,74 @@ struct AttnGeom {
 };
 
 // Enqueue the attention kernel (arguments already validated).
+// Makespan, in 128-key tiles plus a fixed cost per unit (the next unit's Q transform and
+// this unit's epilogue, about three tiles), of the dense units ordered band by band
+// (`band` KV groups, latest query block first: attn_unit) and dealt to G persistent CTAs in
+// snake order (attn_unit_of_round).  A dense unit of query block qb sweeps qb + 1 tiles.
+long long dense_schedule_makespan(long long groups, int nqb, int npairs, long long band, int G) {
+    constexpr long long kUnitOverheadTiles = 3;
+    const long long per_band = band * nqb * npairs;
+    const long long total = groups * nqb * npairs;
+    std::vector<long long> cost(static_cast<size_t>(G), 0);
+    for (long long r = 0; r * G < total; ++r)
+        for (int c = 0; c < G; ++c) {
+            const long long u = r * G + ((r & 1) ? G - 1 - c : c);
+            if (u >= total) continue;
+            const long long bi = u / per_band;
+            const long long gb = std::min(band, groups - bi * band);
+            const long long qb = nqb - 1 - (u - bi * per_band) / (gb * npairs);
+            cost[static_cast<size_t>(c)] += qb + 1 + kUnitOverheadTiles;
+        }
+    return *std::max_element(cost.begin(), cost.end());
+}
+
+// KV groups (sequence, KV head) per band.  A band's K/V (the longest sequence's keys, K and
+// V in bf16) should stay within ~80 MB of the 126 MB L2, which also carries Q, the output and
+// the RoPE table, so that the CTAs working on a band re-read K/V from L2.  Bands are of equal
+// size (the last one is not a short tail of long units).  Among the band sizes that fit, the
+// band size also decides how evenly the snake order spreads the work over the CTAs, so for
+// dense inputs, whose unit costs the host knows, the fewest bands are traded for up to four
+// more when a simulation of the static schedule finishes earlier with them (decisions are
+// kept per shape).  Packed inputs, whose lengths are on the device, take the fewest bands.
+int attn_band(const AttnGeom &gm, int Hkv, int nqb, int npairs, int G) {
+    const long long groups = static_cast<long long>(gm.B) * Hkv;
+    const long long keys = static_cast<long long>(gm.T) + gm.max_prefix;
+    const long long kv_bytes = std::max(1LL, keys * kHeadDim * 2 * 2);
+    const long long fit = std::max(1LL, (80LL << 20) / kv_bytes);
+    const long long nb_min = (groups + fit - 1) / fit;
+    const long long band0 = std::max(1LL, (groups + nb_min - 1) / nb_min);
+    if (gm.cu_q != nullptr || nb_min == 1 || G <= 0 || groups * nqb * npairs > (1LL << 22))
+        return static_cast<int>(band0);
+    struct Entry {
+        long long groups;
+        int nqb, npairs, G;
+        long long band0;
+        int band;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> cache;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const Entry &e : cache)
+            if (e.groups == groups && e.nqb == nqb && e.npairs == npairs && e.G == G && e.band0 == band0)
+                return e.band;
+    }
+    long long best = band0, best_span = dense_schedule_makespan(groups, nqb, npairs, band0, G);
+    for (long long nb = nb_min + 1; nb <= std::min(groups, nb_min + 4); ++nb) {
+        const long long b = (groups + nb - 1) / nb;
+        if (b == best) continue;
+        const long long span = dense_schedule_makespan(groups, nqb, npairs, b, G);
+        if (span < best_span) {
+            best = b;
+            best_span = span;
+        }
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() >= 64) cache.erase(cache.begin());
+    cache.push_back(Entry{groups, nqb, npairs, G, band0, static_cast<int>(best)});
+    return static_cast<int>(best);
+}
+
 gqa_status launch_attention(const void *q, const void *k_hat, const void *v, const int32_t *pos,
                             const float *rope_cs, const float *qnorm_w, const RopeSpec &rs, float eps, void *out,
                             const AttnGeom &gm, int H, int Hkv, cudaStream_t st) {
@@ -313,19 +382,8 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
     if (units <= 0) return GQA_OK;
     if (units > 0x7fffffffLL) return GQA_ERR_INVALID_ARG;
     ap.nunits = static_cast<int>(units);
-    // KV groups per band: bands of equal size, as few as keep each band's K/V (the longest
-    // sequence's keys, K and V in bf16) within ~80 MB of the 126 MB L2, which also carries Q,
-    // the output and the RoPE table.  Equal sizes keep the last band from being a short tail of
-    // long units.
-    {
-        const long long groups = static_cast<long long>(gm.B) * Hkv;
-        const long long keys = static_cast<long long>(gm.T) + gm.max_prefix;
-        const long long kv_bytes = std::max(1LL, keys * kHeadDim * 2 * 2);
-        const long long fit = std::max(1LL, (80LL << 20) / kv_bytes);
-        const long long nbands = (groups + fit - 1) / fit;
-        ap.band = static_cast<int>(std::max(1LL, (groups + nbands - 1) / nbands));
-    }
     const unsigned grid = static_cast<unsigned>(std::min<long long>(units, attn_sm_count()));
+    ap.band = attn_band(gm, Hkv, ap.nqb, ap.npairs, static_cast<int>(grid));
     if (rs.pairing == kPairHalf)
         attn_fwd_kernel<kPairHalf><<<grid, kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
     else
