@@ -154,10 +154,12 @@ bool attn_smem_attr_set() {
     const int dev = current_device();
     if (dev < 0) return false;
     if (done[dev].load()) return true;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<kPairAdjacent>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_kernel<kPairHalf>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+    const int bytes = static_cast<int>(kSmemBytes);
+    const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    if (cudaFuncSetAttribute(attn_fwd_kernel<kPairAdjacent, false>, attr, bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<kPairHalf, false>, attr, bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<kPairAdjacent, true>, attr, bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<kPairHalf, true>, attr, bytes) != cudaSuccess)
         return false;
     done[dev].store(1);
     return true;
@@ -200,6 +202,10 @@ namespace {
 // (round_up(B*T, 128) tokens x D fp32, blocked layout of rope_table_index).
 size_t khat_bytes(int B, int T, int Hkv) { return round_up(static_cast<size_t>(B) * T * Hkv * kHeadDim * 2, 256); }
 size_t rope_table_bytes(int B, int T) { return round_up(static_cast<size_t>(B) * T, 128) * kHeadDim * sizeof(float); }
+// The unit list of a packed launch: at most one entry per 128 tokens of each sequence plus
+// one per non-empty sequence (so at most N + N/128 + 1), then its count.
+long long unit_list_entries(long long N) { return N + N / 128 + 1; }
+size_t unit_list_bytes(long long N) { return round_up(static_cast<size_t>(unit_list_entries(N)) * 8, 256) + 256; }
 }  // namespace
 
 extern "C" size_t gqa_attn_prefill_workspace_size(int B, int T, int H, int Hkv, int D) {
@@ -273,9 +279,9 @@ struct AttnGeom {
     const int64_t *cu_q = nullptr, *kv_off = nullptr;
     const int32_t *prefix = nullptr;
     long long max_prefix = 0;          // host-side bound on the cached keys before a chunk (scheduling only)
+    void *ulist_ws = nullptr;          // packed inputs: room for the unit list (unit_list_bytes of nq_rows)
 };
 
-// Enqueue the attention kernel (arguments already validated).
 // Makespan, in 128-key tiles plus a fixed cost per unit (the next unit's Q transform and
 // this unit's epilogue, about three tiles), of the dense units ordered band by band
 // (`band` KV groups, latest query block first: attn_unit) and dealt to G persistent CTAs in
@@ -344,6 +350,8 @@ int attn_band(const AttnGeom &gm, int Hkv, int nqb, int npairs, int G) {
     return static_cast<int>(best);
 }
 
+// Enqueue the attention kernel (arguments already validated); for packed inputs with room
+// for a unit list, first the kernel that lists the units with work.
 gqa_status launch_attention(const void *q, const void *k_hat, const void *v, const int32_t *pos,
                             const float *rope_cs, const float *qnorm_w, const RopeSpec &rs, float eps, void *out,
                             const AttnGeom &gm, int H, int Hkv, cudaStream_t st) {
@@ -383,11 +391,40 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
     if (units > 0x7fffffffLL) return GQA_ERR_INVALID_ARG;
     ap.nunits = static_cast<int>(units);
     const unsigned grid = static_cast<unsigned>(std::min<long long>(units, attn_sm_count()));
-    ap.band = attn_band(gm, Hkv, ap.nqb, ap.npairs, static_cast<int>(grid));
-    if (rs.pairing == kPairHalf)
-        attn_fwd_kernel<kPairHalf><<<grid, kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
-    else
-        attn_fwd_kernel<kPairAdjacent><<<grid, kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
+    ap.ulist = nullptr;
+    ap.ulist_n = nullptr;
+    ap.uexp = Hkv * ap.npairs;
+    const long long list_cap = unit_list_entries(gm.nq_rows);
+    if (gm.cu_q != nullptr && gm.ulist_ws != nullptr && list_cap * ap.uexp <= 0x7fff0000LL) {
+        // bands of sequences whose K/V (the longest sequence's keys) fit in ~80 MB of L2
+        const long long seq_kv = std::max(1LL, (static_cast<long long>(gm.T) + gm.max_prefix) * Hkv * kHeadDim * 2 * 2);
+        const long long fit = std::max(1LL, (80LL << 20) / seq_kv);
+        const long long nb = (gm.B + fit - 1) / fit;
+        const int band = static_cast<int>(std::max(1LL, (gm.B + nb - 1) / nb));
+        int2 *list = static_cast<int2 *>(gm.ulist_ws);
+        int *count = reinterpret_cast<int *>(static_cast<char *>(gm.ulist_ws) +
+                                             round_up(static_cast<size_t>(list_cap) * 8, 256));
+        unit_list_kernel<<<1, 1024, 0, st>>>(gm.cu_q, gm.kv_off, gm.prefix, gm.nq_rows, gm.nkv_rows, gm.B, ap.nqb,
+                                             band, list, static_cast<int>(list_cap), count, err);
+        if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+        ap.ulist = list;
+        ap.ulist_n = count;
+        ap.band = 1;
+    } else {
+        ap.band = attn_band(gm, Hkv, ap.nqb, ap.npairs, static_cast<int>(grid));
+    }
+    const bool listed = ap.ulist != nullptr;
+    if (rs.pairing == kPairHalf) {
+        if (listed)
+            attn_fwd_kernel<kPairHalf, true><<<grid, kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
+        else
+            attn_fwd_kernel<kPairHalf, false><<<grid, kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
+    } else {
+        if (listed)
+            attn_fwd_kernel<kPairAdjacent, true><<<grid, kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
+        else
+            attn_fwd_kernel<kPairAdjacent, false><<<grid, kAttnThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, ap);
+    }
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
@@ -528,7 +565,7 @@ bool ragged_shape_ok(int B, int64_t N, int H, int Hkv, int max_len) {
 
 extern "C" size_t gqa_attn_prefill_varlen_workspace_size(int64_t N, int Hkv, int D) {
     if (D != kHeadDim || N <= 0 || Hkv <= 0 || N > (1LL << 31) - 256) return 0;
-    return khat_bytes(1, static_cast<int>(N), Hkv) + rope_table_bytes(1, static_cast<int>(N));
+    return khat_bytes(1, static_cast<int>(N), Hkv) + rope_table_bytes(1, static_cast<int>(N)) + unit_list_bytes(N);
 }
 
 extern "C" gqa_status gqa_attn_prefill_varlen(const void *q, const void *k, const void *v, const int32_t *pos,
@@ -560,12 +597,13 @@ extern "C" gqa_status gqa_attn_prefill_varlen(const void *q, const void *k, cons
     gm.q_row_elems = static_cast<long long>(H) * kHeadDim;
     gm.kv_row_elems = static_cast<long long>(Hkv) * kHeadDim;
     gm.cu_q = cu_seqlens;
+    gm.ulist_ws = reinterpret_cast<char *>(table) + rope_table_bytes(1, static_cast<int>(N));
     return launch_attention(q, khat, v, pos, table, qnorm_w, rs, eps, out, gm, H, Hkv, st);
 }
 
 extern "C" size_t gqa_attn_prefill_chunk_workspace_size(int64_t N, int D) {
     if (D != kHeadDim || N <= 0 || N > (1LL << 31) - 256) return 0;
-    return rope_table_bytes(1, static_cast<int>(N));
+    return rope_table_bytes(1, static_cast<int>(N)) + unit_list_bytes(N);
 }
 
 extern "C" gqa_status gqa_attn_prefill_chunk(const void *q, const void *k, const void *v, const int32_t *pos,
@@ -614,6 +652,7 @@ extern "C" gqa_status gqa_attn_prefill_chunk(const void *q, const void *k, const
     gm.kv_off = cache_offsets;
     gm.prefix = prefix_len;
     gm.max_prefix = cache_rows / std::max(1, B);   // an average; only the schedule depends on it
+    gm.ulist_ws = reinterpret_cast<char *>(table) + rope_table_bytes(1, static_cast<int>(N));
     return launch_attention(q, k_cache, v_cache, pos, table, qnorm_w, rs, eps, out, gm, H, Hkv, st);
 }
 

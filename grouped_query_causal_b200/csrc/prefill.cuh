@@ -260,6 +260,11 @@ struct AttnParams {
     long long nkv_rows;    // rows of k-hat / v
     int B, T, H, Hkv, hpg, nqb, npairs, nunits;
     int band;              // KV groups (sequence, KV head) scheduled together: their K/V fit in L2
+    // Packed inputs: the (sequence, query block) pairs that have work, in schedule order
+    // (unit_list_kernel), each standing for uexp = Hkv * npairs units, and their count.
+    const int2 *ulist;     // or nullptr: every unit of the band order has work
+    const int *ulist_n;
+    int uexp;
     int out_bf16;          // 1: the output is rounded to bf16 (the input of the output projection)
     int test_stall;        // 1 (failure-path test only): the MMA thread first waits on BAR_NEVER
     float eps;
@@ -283,20 +288,40 @@ struct AttnUnit {
 
 // Decode unit u; false when it has no work (a query block past the end of a shorter
 // sequence, or a sequence whose device-side geometry is out of range).
+// Unit u of a listed launch: (sequence, query block, KV head, head pair).  Kept out of line:
+// its divisions would otherwise hold registers in every role that decodes units.
+__device__ __noinline__ int4 listed_unit(const int2 *list, int uexp, int npairs, int u) {
+    const int e = u / uexp, r = u - e * uexp;
+    const int2 ent = list[e];
+    const int g = r / npairs;
+    return make_int4(ent.x, ent.y, g, r - g * npairs);
+}
+
+template <bool LISTED>
 __device__ __forceinline__ bool attn_unit(const AttnParams &p, int u, AttnUnit &w, bool &bad) {
     bad = false;
-    // u -> (band of KV groups, query block latest first, group in the band, head pair)
-    const int ngroups = p.B * p.Hkv;
-    const int per_band = p.band * p.nqb * p.npairs;
-    const int band = u / per_band;
-    const int gb = min(p.band, ngroups - band * p.band);   // groups in this band
-    int rem = u - band * per_band;
-    const int qb = p.nqb - 1 - rem / (gb * p.npairs);
-    rem %= gb * p.npairs;
-    const int pair = rem % p.npairs;
-    const int gi = band * p.band + rem / p.npairs;
-    w.g = gi % p.Hkv;
-    w.b = gi / p.Hkv;
+    int qb, pair;
+    if constexpr (LISTED) {
+        // u -> (listed sequence and query block, KV head, head pair)
+        const int4 d = listed_unit(p.ulist, p.uexp, p.npairs, u);
+        w.b = d.x;
+        qb = d.y;
+        w.g = d.z;
+        pair = d.w;
+    } else {
+        // u -> (band of KV groups, query block latest first, group in the band, head pair)
+        const int ngroups = p.B * p.Hkv;
+        const int per_band = p.band * p.nqb * p.npairs;
+        const int band = u / per_band;
+        const int gb = min(p.band, ngroups - band * p.band);   // groups in this band
+        int rem = u - band * per_band;
+        qb = p.nqb - 1 - rem / (gb * p.npairs);
+        rem %= gb * p.npairs;
+        pair = rem % p.npairs;
+        const int gi = band * p.band + rem / p.npairs;
+        w.g = gi % p.Hkv;
+        w.b = gi / p.Hkv;
+    }
     long long q0 = static_cast<long long>(w.b) * p.T, len = p.T;
     if (p.cu_q != nullptr) {
         q0 = p.cu_q[w.b];
@@ -487,6 +512,83 @@ __device__ __forceinline__ float max8(const float (&m)[8]) {
     return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
 }
 
+// Units of the launch: those listed for packed inputs (the count comes from the list kernel
+// that ran before on the stream), else every unit of the band order.
+template <bool LISTED>
+__device__ __forceinline__ int attn_unit_count(const AttnParams &p) {
+    if constexpr (LISTED) return *p.ulist_n * p.uexp;
+    return p.nunits;
+}
+
+// The (sequence, query block) pairs of a packed launch that have work, in the order the
+// attention kernel deals them out: bands of `band` sequences (whose K/V fit in L2 together),
+// inside a band query blocks latest first, then the sequences of the band.  Units past the end
+// of a shorter sequence would otherwise leave holes in the rounds of the static schedule.
+// One CTA of 1024 threads: each counts the slots of a contiguous range, a block-wide scan
+// gives each range its place, and each writes its entries.  A sequence whose bounds are out
+// of range gets no entries and sets kErrInput.
+__global__ void __launch_bounds__(1024) unit_list_kernel(const int64_t *cu, const int64_t *kv_off, const int32_t *prefix,
+                                                       long long nq_rows, long long nkv_rows, int B, int nqb, int band,
+                                                       int2 *list, int cap, int *count, unsigned *err) {
+    __shared__ int warp_sum[32];
+    const long long per_band = static_cast<long long>(band) * nqb;
+    const long long slots = (static_cast<long long>(B) + band - 1) / band * per_band;
+    const long long per = (slots + blockDim.x - 1) / blockDim.x;
+    const long long s0 = min(slots, per * threadIdx.x), s1 = min(slots, s0 + per);
+    // slot s -> (b, qb), or -1 when the slot has no work
+    auto slot_block = [&](long long s, int &b) -> int {
+        const long long bi = s / per_band, rem = s - bi * per_band;
+        const int qb = nqb - 1 - static_cast<int>(rem / band);
+        b = static_cast<int>(bi * band + rem % band);
+        if (b >= B) return -1;
+        const long long q0 = cu[b], len = cu[b + 1] - q0;
+        const long long kv0 = kv_off != nullptr ? kv_off[b] : q0;
+        const long long pre = prefix != nullptr ? prefix[b] : 0;
+        if (q0 < 0 || len < 0 || q0 + len > nq_rows || len > static_cast<long long>(nqb) * 128 || pre < 0 ||
+            kv0 < 0 || kv0 + pre + len > nkv_rows || pre + len > 0x7fff0000LL) {
+            if (qb == 0) atomicOr(err, kErrInput);
+            return -1;
+        }
+        return static_cast<long long>(qb) * 128 < len ? qb : -1;
+    };
+    int n = 0;
+    for (long long s = s0; s < s1; ++s) {
+        int b;
+        if (slot_block(s, b) >= 0) ++n;
+    }
+    // exclusive scan of n over the block: within each warp, then over the warp totals
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int incl = n;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_sum[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int t = lane < static_cast<int>(blockDim.x >> 5) ? warp_sum[lane] : 0;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += u;
+        }
+        warp_sum[lane] = t;   // inclusive over warps
+    }
+    __syncthreads();
+    int pos = (wid > 0 ? warp_sum[wid - 1] : 0) + incl - n;
+    for (long long s = s0; s < s1; ++s) {
+        int b;
+        const int qb = slot_block(s, b);
+        if (qb < 0) continue;
+        // sequences that overlap (cu not ascending) can list more than the buffer holds
+        if (pos < cap)
+            list[pos] = make_int2(b, qb);
+        else
+            atomicOr(err, kErrInput);
+        ++pos;
+    }
+    if (threadIdx.x == blockDim.x - 1) *count = min(pos, cap);
+}
+
 // The work unit of round r for this CTA.  Units are numbered heaviest first; the rounds
 // alternate their direction over the CTAs (snake order), so that each pair of rounds
 // gives every CTA about the same causal length.
@@ -499,8 +601,9 @@ __device__ __forceinline__ int attn_unit_of_round(int r) {
 // round (attn_unit_of_round).  The K/V ring, the barrier
 // phases and the TMEM buffers carry over from unit to unit, so that the next unit's Q
 // and first K/V tiles load, and its Q tile is normed and rotated, while the current
-// unit's last P V and epilogue run.
-template <int PAIRING>
+// unit's last P V and epilogue run.  LISTED: the units are those of the unit list
+// (packed inputs), else every unit of the band order.
+template <int PAIRING, bool LISTED>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
@@ -548,6 +651,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
+    const int nun = attn_unit_count<LISTED>(p);
     if (warp < 4) {
     regs_dec<kRegsCtl>();
     if (warp == 0) {
@@ -561,10 +665,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t armed = 0;                     // steps armed so far (step k on barrier k % 3)
             for (int r = 0; ok; ++r) {
                 const int u = attn_unit_of_round(r);
-                if (u >= p.nunits) break;
+                if (u >= nun) break;
                 AttnUnit w;
                 bool bad;
-                if (!attn_unit(p, u, w, bad)) {
+                if (!attn_unit<LISTED>(p, u, w, bad)) {
                     if (bad) atomicOr(p.err, kErrInput);
                     continue;
                 }
@@ -651,10 +755,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (p.test_stall) ok = mbar_wait(BAR(BAR_NEVER), 0, p.err, 100000ull);
             for (int r = 0; ok; ++r) {
                 const int u = attn_unit_of_round(r);
-                if (u >= p.nunits) break;
+                if (u >= nun) break;
                 AttnUnit w;
                 bool bad;
-                if (!attn_unit(p, u, w, bad)) continue;
+                if (!attn_unit<LISTED>(p, u, w, bad)) continue;
                 const uint32_t k0_item = it;
                 if (!MMA_WAIT(BAR(BAR_K0_FULL), k0_uses & 1)) { ok = false; break; }
                 ++k0_uses;
@@ -734,8 +838,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             bool have = false, bad;
             for (;; ++rnd) {
                 const int u = attn_unit_of_round(rnd);
-                if (u >= p.nunits) break;
-                if (attn_unit(p, u, w, bad) && s < w.nslots) {
+                if (u >= nun) break;
+                if (attn_unit<LISTED>(p, u, w, bad) && s < w.nslots) {
                     have = true;
                     break;
                 }

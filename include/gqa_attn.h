@@ -324,7 +324,9 @@ gqa_status gqa_attn_decode_append_ex(const void *q, const void *k_new, const voi
  *   out       fp32 [N, H, D]      row t of sequence b attends to keys 0 .. t of b only
  *   max_seqlen host-side bound on every sequence's length (sizes the launch)
  *   workspace >= gqa_attn_prefill_varlen_workspace_size(N, Hkv, D) bytes, 256-byte
- *             aligned (k-hat of the N tokens and their RoPE cos/sin).
+ *             aligned (k-hat of the N tokens, their RoPE cos/sin, and the list of the
+ *             (sequence, 128-token query block) pairs that have work, which a small kernel
+ *             writes before the attention kernel so that no CTA is dealt empty work).
  * Sequence bounds are read on the device: a sequence that breaks them (or is longer than
  * max_seqlen, whose tail then goes unwritten) is skipped and sets GQA_ERR_DEVICE_INPUT;
  * its output rows are undefined.  B = 0, N = 0 or max_seqlen = 0 is a no-op.
@@ -354,7 +356,8 @@ gqa_status gqa_attn_prefill_varlen(const void *q, const void *k, const void *v, 
  *   prefix_len        int32 [B], device, rows already cached (0 = plain prefill of the chunk)
  *   max_chunk_len     host-side bound on every chunk's length
  *   workspace >= gqa_attn_prefill_chunk_workspace_size(N, D) bytes, 256-byte aligned
- *             (the chunk tokens' RoPE cos/sin).
+ *             (the chunk tokens' RoPE cos/sin and the list of the (sequence, query block)
+ *             pairs that have work, as for gqa_attn_prefill_varlen).
  * A chunk token whose cache row falls outside its sequence's rows is not written and
  * sets GQA_ERR_DEVICE_INPUT (that sequence's output is then undefined); the same for
  * sequence bounds out of range.  prefix_len is not advanced (the caller does that).
