@@ -516,9 +516,10 @@ def run_packed_leg(gqa, name, dev, stream, world, K, W):
     what = (f"{B} sequences, {prefix[0]} cached rows + a {w.lens[0]}-token chunk each, H{H} Hkv{Hkv} D{D}"
             if chunk else f"{B} packed sequences, lengths U[256,8192] (N={N}), H{H} Hkv{Hkv} D{D}")
     return {"value": round(whole_job_rate(flops * K, world, sec) / 1e12, 2), "unit": "TFLOP/s",
-            "ms": round(1e3 * sec / K, 4), "workload": what, "flops_per_call": flops, "gpu_launches": 2 * K,
+            "ms": round(1e3 * sec / K, 4), "workload": what, "flops_per_call": flops, "gpu_launches": 3 * K,
             "roofline": {"bound": "tensor", "achieved": round(flops * K / sec / 1e12, 2), "unit": "TFLOP/s",
-                         "traffic": None, "kernel": "k_prologue_kernel + attn_fwd_kernel (one call)"}}
+                         "traffic": None,
+                         "kernel": "k_prologue_kernel + unit_list_kernel + attn_fwd_kernel (one call)"}}
 
 
 def run_projection_leg(gqa, dev, stream, world, K, W):
