@@ -188,3 +188,32 @@ def test_chunk_overflowing_its_rows_is_a_device_input_error(gqa):
     kcpu = kc.cpu()
     assert (kcpu[:5] == 0).all() and (kcpu[45:70] == 0).all()   # nothing before the rows it may write
     assert gqa.device_status() == 0
+
+
+def test_varlen_sequence_longer_than_max_is_a_device_input_error(gqa):
+    """A sequence longer than max_seqlen gets no work (the unit list leaves it out) and
+    raises the device input status; the other sequences are still right."""
+    lens = [300, 200, 50]
+    q, k, v, pos, cu, wq, wk, theta, eps = _packed(lens, 8, 2, seed=170)
+    out = gqa.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), cu.cuda(), wq.cuda(), wk.cuda(),
+                             max_seqlen=256, eps=eps, rope=gqa.RopeConfig.make(theta=theta))
+    torch.cuda.synchronize()
+    assert gqa.device_status() == -6
+    assert gqa.device_status() == 0
+    ref = oracle.prefill_varlen_ex(bits(q), bits(k), bits(v), cu.numpy(), pos.numpy(), wq.numpy(), wk.numpy(),
+                                   oracle.Rope(theta=theta), eps)
+    assert_close(out.cpu().numpy()[300:], ref[300:], "the sequences within max_seqlen")
+
+
+def test_varlen_overlapping_sequences_cannot_overrun_the_unit_list(gqa):
+    """cu_seqlens that is not ascending describes overlapping sequences whose units can
+    outnumber the list's room (one entry per 128 tokens plus one per sequence of N tokens):
+    the list keeps to its room and the call raises the device input status."""
+    N, B = 10, 40
+    q, k, v, pos, _, wq, wk, theta, eps = _packed([N], 4, 2, seed=171)
+    cu = torch.tensor([0 if i % 2 == 0 else N for i in range(B + 1)], dtype=torch.int64)   # 0, N, 0, N, ...
+    gqa.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), cu.cuda(), wq.cuda(), wk.cuda(), max_seqlen=N,
+                       eps=eps, rope=gqa.RopeConfig.make(theta=theta))
+    torch.cuda.synchronize()
+    assert gqa.device_status() == -6
+    assert gqa.device_status() == 0
