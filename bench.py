@@ -767,7 +767,11 @@ def run_decode_paged(gqa, dec, dq, kc, vc, sl, dwq, dev, stream, world, K, W, pa
 
 def run_e2e(gqa, pin, dec, dev, stream, rank, world, steps):
     """Same metrics through the public API with host (pinned) buffers: every step copies
-    that step's inputs host->device, runs the call, and reads the result back."""
+    that step's inputs host->device, runs the call, and reads the result back.  The steps
+    are pipelined as a serving loop would run them: copies in on one stream, the calls on
+    the compute stream, copies out on a third, with two device buffer sets, so that step
+    i+1's inputs and step i-1's result cross PCIe while step i computes (events order
+    each buffer set's reuse)."""
     lib = gqa.load()
     sh = stream.cuda_stream
     B, T, H, D = pin.q.shape
@@ -778,56 +782,81 @@ def run_e2e(gqa, pin, dec, dev, stream, rank, world, steps):
     hp = {n: getattr(pin, n).pin_memory() for n in ("q", "k", "v", "pos", "wq", "wk")}
     hd = {"q": dec.q.pin_memory(), "k_cache": dec.k_cache.pin_memory(), "v_cache": dec.v_cache.pin_memory(),
           "offsets": dec.offsets.pin_memory(), "seqlens": dec.seqlens.pin_memory(), "wq": dec.wq.pin_memory()}
-    dp = {n: torch.empty_like(t, device=dev) for n, t in hp.items()}
-    dd = {n: torch.empty_like(t, device=dev) for n, t in hd.items()}
-    out = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
     hout = torch.empty((B, T, H, D), dtype=torch.float32).pin_memory()
-    dout = torch.empty((dB, dH, D), dtype=torch.float32, device=dev)
     hdout = torch.empty((dB, dH, D), dtype=torch.float32).pin_memory()
     pws = torch.empty(gqa.prefill_workspace_size(B, T, H, Hkv, D), dtype=torch.uint8, device=dev)
     dws = torch.empty(gqa.decode_workspace_size(dB, dH, dHkv, max_len, D), dtype=torch.uint8, device=dev)
     ptr = lambda t: t.data_ptr()  # noqa: E731
     p_in = sum(t.numel() * t.element_size() for t in hp.values())
     d_in = sum(t.numel() * t.element_size() for t in hd.values())
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def prefill_step():
-        for n in hp:
-            dp[n].copy_(hp[n], non_blocking=True)
-        st = lib.gqa_attn_prefill(ptr(dp["q"]), ptr(dp["k"]), ptr(dp["v"]), ptr(dp["pos"]), ptr(dp["wq"]),
-                                  ptr(dp["wk"]), pin.theta, pin.eps, ptr(out), B, T, H, Hkv, D, ptr(pws),
-                                  pws.numel(), sh)
-        hout.copy_(out, non_blocking=True)
-        return st
+    def prefill_set():
+        d = {n: torch.empty_like(t, device=dev) for n, t in hp.items()}
+        d["out"] = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
+        return d
 
-    def decode_step():
-        for n in hd:
-            dd[n].copy_(hd[n], non_blocking=True)
-        st = lib.gqa_attn_decode(ptr(dd["q"]), ptr(dd["k_cache"]), ptr(dd["v_cache"]), ptr(dd["offsets"]),
-                                 ptr(dd["seqlens"]), None, ptr(dd["wq"]), dec.theta, dec.eps, ptr(dout), dB, dH,
-                                 dHkv, D, max_len, ptr(dws), dws.numel(), sh)
-        hdout.copy_(dout, non_blocking=True)
-        return st
+    def prefill_call(d):
+        return lib.gqa_attn_prefill(ptr(d["q"]), ptr(d["k"]), ptr(d["v"]), ptr(d["pos"]), ptr(d["wq"]),
+                                    ptr(d["wk"]), pin.theta, pin.eps, ptr(d["out"]), B, T, H, Hkv, D, ptr(pws),
+                                    pws.numel(), sh)
+
+    def decode_set():
+        d = {n: torch.empty_like(t, device=dev) for n, t in hd.items()}
+        d["out"] = torch.empty((dB, dH, D), dtype=torch.float32, device=dev)
+        return d
+
+    def decode_call(d):
+        return lib.gqa_attn_decode(ptr(d["q"]), ptr(d["k_cache"]), ptr(d["v_cache"]), ptr(d["offsets"]),
+                                   ptr(d["seqlens"]), None, ptr(d["wq"]), dec.theta, dec.eps, ptr(d["out"]), dB, dH,
+                                   dHkv, D, max_len, ptr(dws), dws.numel(), sh)
+
+    def run(host_in, host_out, sets, call, n):
+        """n pipelined steps; returns the device time from the first copy in to the last copy out."""
+        ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        computed, copied = [None, None], [None, None]
+        start, end = ev(), ev()
+        start.record(s_in)
+        for i in range(n):
+            d = sets[i % 2]
+            with torch.cuda.stream(s_in):
+                if computed[i % 2] is not None:
+                    s_in.wait_event(computed[i % 2])       # the call two steps back has read this set
+                for k in host_in:
+                    d[k].copy_(host_in[k], non_blocking=True)
+                loaded = ev()
+                loaded.record(s_in)
+            stream.wait_event(loaded)
+            if copied[i % 2] is not None:
+                stream.wait_event(copied[i % 2])           # this set's previous result has been read out
+            if call(d) != 0:
+                raise RuntimeError("e2e call failed")
+            computed[i % 2] = ev()
+            computed[i % 2].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(computed[i % 2])
+                host_out.copy_(d["out"], non_blocking=True)
+                copied[i % 2] = ev()
+                copied[i % 2].record(s_out)
+        end.record(s_out)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / 1e3
 
     res = {}
-    for name, fn, units, unit, scale, b_in, b_out in (
-            ("prefill", prefill_step, prefill_flops(B, T, H, D), "TFLOP/s", 1e12, p_in, hout.numel() * 4),
-            ("decode", decode_step, decode_bytes(dec.seqlens.tolist(), dH, dHkv, D), "GB/s", 1e9, d_in,
-             hdout.numel() * 4)):
-        if fn() != 0:
-            raise RuntimeError(f"e2e {name} failed")
-        torch.cuda.synchronize()
+    for name, make_set, call, host_in, host_out, units, unit, scale, b_in in (
+            ("prefill", prefill_set, prefill_call, hp, hout, prefill_flops(B, T, H, D), "TFLOP/s", 1e12, p_in),
+            ("decode", decode_set, decode_call, hd, hdout, decode_bytes(dec.seqlens.tolist(), dH, dHkv, D), "GB/s",
+             1e9, d_in)):
+        sets = [make_set(), make_set()]
+        run(host_in, host_out, sets, call, 2)   # warm-up
         if world > 1:
             torch.distributed.barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(steps):
-            if fn() != 0:
-                raise RuntimeError(f"e2e {name} failed")
-        b.record(stream)
-        torch.cuda.synchronize()
-        sec = max_over_ranks([a.elapsed_time(b)], dev, world)[0] / 1e3
+        sec = max_over_ranks([run(host_in, host_out, sets, call, steps) * 1e3], dev, world)[0] / 1e3
         res[name] = {"value": round(whole_job_rate(units * steps, world, sec) / scale, 3), "unit": unit,
-                     "h2d_bytes_per_step": int(b_in), "d2h_bytes_per_step": int(b_out), "steps": steps}
+                     "h2d_bytes_per_step": int(b_in), "d2h_bytes_per_step": int(host_out.numel() * 4),
+                     "steps": steps, "pipelined": "copies in, calls and copies out on three streams, "
+                                                  "two device buffer sets"}
+        del sets
     return res
 
 
