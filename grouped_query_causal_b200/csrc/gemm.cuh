@@ -29,7 +29,8 @@ constexpr int kGemmGroupM = 8;
 constexpr uint32_t kGemmABytes = kGemmBM * kGemmBK * 2;   // 16 KB
 constexpr uint32_t kGemmBBytes = kGemmBN * kGemmBK * 2;   // 32 KB
 constexpr uint32_t kGemmStageBytes = kGemmABytes + kGemmBBytes;
-constexpr uint32_t kGemmOffBar = kGemmStages * kGemmStageBytes;
+constexpr uint32_t kGemmOffStage = kGemmStages * kGemmStageBytes;   // epilogue staging: 4 warps x 32 rows x 128 B
+constexpr uint32_t kGemmOffBar = kGemmOffStage + 4 * 32 * 128;
 enum {
     GB_FULL = 0,                          // [stages] TMA -> MMA
     GB_EMPTY = kGemmStages,               // [stages] MMA (commit) -> TMA
@@ -179,30 +180,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!__all_sync(0xffffffffu, mbar_wait(GBAR(GB_ACC_FULL + a), acc_uses[a] & 1, p.err))) break;
             ++acc_uses[a];
             tc_fence_after();
-            const int row = mb * kGemmBM + q * 32 + lane;
+            const int row0 = mb * kGemmBM + q * 32;   // this warp's 32 output rows
             const int col0 = nb * kGemmBN;
             const uint32_t tacc = tmem + lane_base + static_cast<uint32_t>(a) * kGemmBN;
+            // Each 32-column chunk: every thread stages its row (16-byte granules swizzled by
+            // row, so that no two lanes of a quarter-warp hit the same banks), then the warp
+            // copies its 32 rows out whole-row: 4 fp32 rows (128 B each) or 8 bf16 rows (64 B
+            // each) per instruction instead of 32 scattered 16-byte pieces.
+            const uint32_t stg = sbase + kGemmOffStage + static_cast<uint32_t>(q) * 32 * 128;
 #pragma unroll 1
             for (int c = 0; c < kGemmBN / 32; ++c) {
                 float v[32];
                 tmem_ld32(tacc + 32 * c, v);
                 tmem_wait_ld();
                 const int col = col0 + 32 * c;
-                if (row < p.M && col < p.N) {   // N is a multiple of 32
-                    if (p.y_fp32) {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.y) + row * p.ldy + col);
+                if (p.y_fp32) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-                    } else {
-                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.y) + row * p.ldy + col);
+                    for (int g = 0; g < 8; ++g)
+                        st_shared_v4(stg + lane * 128 + ((g ^ (lane & 7)) << 4),
+                                     make_uint4(__float_as_uint(v[4 * g]), __float_as_uint(v[4 * g + 1]),
+                                                __float_as_uint(v[4 * g + 2]), __float_as_uint(v[4 * g + 3])));
+                    __syncwarp();
+                    const int g = lane & 7;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(pack_bf16x2(v[8 * e], v[8 * e + 1]), pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
-                                                pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
-                                                pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
+                    for (int it = 0; it < 8; ++it) {
+                        const int r = it * 4 + (lane >> 3);
+                        const uint4 u = ld_shared_v4(stg + r * 128 + ((g ^ (r & 7)) << 4));
+                        if (row0 + r < p.M && col < p.N)   // N is a multiple of 32
+                            *reinterpret_cast<uint4 *>(static_cast<float *>(p.y) + (row0 + r) * p.ldy + col + 4 * g) = u;
+                    }
+                } else {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        st_shared_v4(stg + lane * 128 + ((g ^ (lane & 7)) << 4),
+                                     make_uint4(pack_bf16x2(v[8 * g], v[8 * g + 1]), pack_bf16x2(v[8 * g + 2], v[8 * g + 3]),
+                                                pack_bf16x2(v[8 * g + 4], v[8 * g + 5]),
+                                                pack_bf16x2(v[8 * g + 6], v[8 * g + 7])));
+                    __syncwarp();
+                    const int g = lane & 3;
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        const int r = it * 8 + (lane >> 2);
+                        const uint4 u = ld_shared_v4(stg + r * 128 + ((g ^ (r & 7)) << 4));
+                        if (row0 + r < p.M && col < p.N)
+                            *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.y) + (row0 + r) * p.ldy + col + 8 * g) = u;
                     }
                 }
+                __syncwarp();   // the warp's staging rows are free again
             }
             tc_fence_before();
             mbar_arrive(GBAR(GB_ACC_EMPTY + a));
