@@ -310,7 +310,9 @@ long long dense_schedule_makespan(long long groups, int nqb, int npairs, long lo
 // band size also decides how evenly the snake order spreads the work over the CTAs, so for
 // dense inputs, whose unit costs the host knows, the fewest bands are traded for up to four
 // more when a simulation of the static schedule finishes earlier with them (decisions are
-// kept per shape).  Packed inputs, whose lengths are on the device, take the fewest bands.
+// kept per shape).  Packed inputs, whose lengths are on the device, are scheduled through the
+// unit list instead (bands of whole sequences, launch_attention); without one they take the
+// fewest bands.
 int attn_band(const AttnGeom &gm, int Hkv, int nqb, int npairs, int G) {
     const long long groups = static_cast<long long>(gm.B) * Hkv;
     const long long keys = static_cast<long long>(gm.T) + gm.max_prefix;
