@@ -381,6 +381,23 @@ def prefill_chunk_ex(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, offsets
     return out, khat
 
 
+def prefill_chunk_paged_ex(q_bits, k_bits, v_bits, k_pages_bits, v_pages_bits, page_table, page_size, prefix_len,
+                           pos, wq, wk, rope: Rope, eps: float):
+    """Chunked prefill against a paged cache prefix: cached row r of sequence b is row
+    r % page_size of page page_table[b, r // page_size]; the attention is prefill_chunk_ex
+    on the gathered prefix rows.  Returns (out [B,C,H,D], chunk k-hat [B,C,Hkv,D]), fp64."""
+    k_pages_bits = _c(k_pages_bits, np.uint16)
+    v_pages_bits = _c(v_pages_bits, np.uint16)
+    table = np.asarray(page_table)
+    pl = np.asarray(prefix_len, np.int64)
+    Hkv, D = k_pages_bits.shape[2], k_pages_bits.shape[3]
+    none = np.zeros((0, Hkv, D), np.uint16)
+    kc = np.concatenate([none] + [_gather_pages(k_pages_bits, table[b], page_size, pl[b]) for b in range(len(pl))])
+    vc = np.concatenate([none] + [_gather_pages(v_pages_bits, table[b], page_size, pl[b]) for b in range(len(pl))])
+    offsets = np.concatenate([[0], np.cumsum(pl)]).astype(np.int64)
+    return prefill_chunk_ex(q_bits, k_bits, v_bits, kc, vc, offsets, pl.astype(np.int32), pos, wq, wk, rope, eps)
+
+
 def prefill_varlen_ex(q_bits, k_bits, v_bits, cu_seqlens, pos, wq, wk, rope: Rope, eps: float) -> np.ndarray:
     """Packed variable-length prefill: q [N,H,D], k/v [N,Hkv,D] bf16 bits, sequence b on
     tokens cu_seqlens[b] .. cu_seqlens[b+1]-1, positions pos [N]; causal within each

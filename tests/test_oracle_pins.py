@@ -697,6 +697,23 @@ def test_chunk_after_a_prefix_equals_the_tail_of_prefill():
     np.testing.assert_array_equal(khat, kh[:, P:])
 
 
+def test_paged_chunk_equals_contiguous_chunk():
+    """The chunk against a prefix kept in pages handed out in a shuffled order is, bit for
+    bit, the chunk against the same prefix kept contiguously."""
+    B, P, C, H, Hkv, D = 2, 37, 9, 4, 2, 16
+    inp, kh, kc, vc, offsets = _chunk_setup(B, P, C, H, Hkv, D, seed=84)
+    args = (_bits(inp.q)[:, P:], _bits(inp.k)[:, P:], _bits(inp.v)[:, P:])
+    rest = (inp.pos.numpy()[:, P:], inp.wq.numpy(), inp.wk.numpy(), oracle.Rope(theta=inp.theta), inp.eps)
+    ref, kref = oracle.prefill_chunk_ex(*args, _bits(kc), _bits(vc), offsets, np.full(B, P, np.int32), *rest)
+    for ps in (16, 32):
+        pc = synthetic.page_cache(kc, vc, torch.from_numpy(offsets), [P] * B, ps, seed=85)
+        assert not np.array_equal(pc.page_table.numpy()[0, :2], [0, 1])   # not the identity
+        got, kgot = oracle.prefill_chunk_paged_ex(*args, _bits(pc.k_pages), _bits(pc.v_pages), pc.page_table.numpy(),
+                                                  ps, np.full(B, P, np.int32), *rest)
+        np.testing.assert_array_equal(got, ref)
+        np.testing.assert_array_equal(kgot, kref)
+
+
 def test_chunk_without_prefix_is_plain_prefill():
     B, C, H, Hkv, D = 2, 9, 4, 2, 16
     inp = synthetic.prefill_inputs(B, C, H, Hkv, D=D, seed=81)
