@@ -285,6 +285,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- packed variable-length and chunked prefill, the projections (own timed regions)
     varlen = run_packed_leg(gqa, "varlen_prefill", dev, stream, world, K, args.warmup)
     chunked = run_packed_leg(gqa, "chunked_prefill", dev, stream, world, K, args.warmup)
+    chunked_paged = run_packed_leg(gqa, "chunked_prefill", dev, stream, world, K, args.warmup, page_size=16)
     proj = run_projection_leg(gqa, dev, stream, world, K, args.warmup)
     block = run_block_leg(gqa, dev, stream, world, K, args.warmup)
     # ---- the decode step that appends the new token first, and the plain decode, each in
@@ -311,8 +312,8 @@ def run_ours(args, rank, world, local_rank):
     traffic_attn = traffic_from_profiles("attn_fwd_kernel", PREFILL)
     traffic_dec = traffic_from_profiles("decode_split_kernel", DECODE)
     for key, legd in (("large_prefill", extra), ("varlen_prefill", varlen), ("chunked_prefill", chunked),
-                      ("projections", proj), ("attn_block", block), ("decode_append", app),
-                      ("decode_paged", paged), ("decode_alone", dalone)):
+                      ("chunked_prefill_paged", chunked_paged), ("projections", proj), ("attn_block", block),
+                      ("decode_append", app), ("decode_paged", paged), ("decode_alone", dalone)):
         legd["clocks"] = LEG_CLOCKS.get(key)
     hbm_line = lambda leg: dict(leg, roofline=dict(leg["roofline"], peak=hbm,  # noqa: E731
                                                    frac=round(leg["roofline"]["achieved"] / hbm, 4),
@@ -369,6 +370,7 @@ def run_ours(args, rank, world, local_rank):
         "large_prefill": tc_line(extra),
         "varlen_prefill": tc_line(varlen),
         "chunked_prefill": tc_line(chunked),
+        "chunked_prefill_paged": tc_line(chunked_paged),
         "projections": tc_line(proj),
         "attn_block": tc_line(block),
         "decode_append": hbm_line(app),
@@ -463,10 +465,11 @@ def packed_flops(lens, prefix, H, D=128):
     return sum(4 * D * H * (n * p + n * (n + 1) // 2) for n, p in zip(lens, prefix))
 
 
-def run_packed_leg(gqa, name, dev, stream, world, K, W):
+def run_packed_leg(gqa, name, dev, stream, world, K, W, page_size=None):
     """gqa_attn_prefill_varlen (no prefix) or gqa_attn_prefill_chunk (each sequence has
     cached rows; the chunk is appended to the cache first) on a packed workload, inputs
-    resident, CUDA events around each call, L2 flushed between calls."""
+    resident, CUDA events around each call, L2 flushed between calls.  With page_size, the
+    chunk workload's cache in shuffled pages of that many rows (gqa_attn_prefill_chunk_paged)."""
     lib = gqa.load()
     sh = stream.cuda_stream
     w = synthetic.make(name)
@@ -475,7 +478,16 @@ def run_packed_leg(gqa, name, dev, stream, world, K, W):
     B = len(w.lens)
     chunk = w.prefix is not None
     t = {n: getattr(w, n).to(dev) for n in ("q", "k", "v", "pos", "cu", "wq", "wk")}
-    if chunk:
+    paged = chunk and page_size is not None
+    leg = name + ("_paged" if paged else "")
+    if paged:
+        caps = [p + n for p, n in zip(w.prefix.tolist(), w.lens)]
+        pc = synthetic.page_cache(w.k_cache, w.v_cache, w.cache_offsets, caps, page_size, seed=31)
+        t.update(k_pages=pc.k_pages.to(dev), v_pages=pc.v_pages.to(dev), table=pc.page_table.to(dev),
+                 prefix=w.prefix.to(dev))
+        ws_n = lib.gqa_attn_prefill_chunk_paged_workspace_size(N, D)
+        del pc
+    elif chunk:
         t.update({n: getattr(w, n).to(dev) for n in ("k_cache", "v_cache", "cache_offsets", "prefix")})
         ws_n = lib.gqa_attn_prefill_chunk_workspace_size(N, D)
     else:
@@ -491,7 +503,13 @@ def run_packed_leg(gqa, name, dev, stream, world, K, W):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)] if st_ is not None else None
         if ev:
             ev[0].record(st_)
-        if chunk:
+        if paged:
+            st = lib.gqa_attn_prefill_chunk_paged(
+                ptr(t["q"]), ptr(t["k"]), ptr(t["v"]), ptr(t["pos"]), ptr(t["cu"]), ptr(t["k_pages"]),
+                ptr(t["v_pages"]), ptr(t["table"]), t["k_pages"].shape[0], page_size, t["table"].shape[1],
+                ptr(t["prefix"]), ptr(t["wq"]), ptr(t["wk"]), ctypes.byref(rope), w.eps, ptr(out), B, N, H, Hkv, D,
+                maxlen, ptr(ws), ws.numel(), sh)
+        elif chunk:
             st = lib.gqa_attn_prefill_chunk(ptr(t["q"]), ptr(t["k"]), ptr(t["v"]), ptr(t["pos"]), ptr(t["cu"]),
                                             ptr(t["k_cache"]), ptr(t["v_cache"]), ptr(t["cache_offsets"]),
                                             ptr(t["prefix"]), t["k_cache"].shape[0], ptr(t["wq"]), ptr(t["wk"]),
@@ -504,16 +522,17 @@ def run_packed_leg(gqa, name, dev, stream, world, K, W):
         if ev:
             ev[1].record(st_)
         if st != 0:
-            raise RuntimeError(f"{name}: library call failed with status {st}")
+            raise RuntimeError(f"{leg}: library call failed with status {st}")
         return ev
 
-    sec = timed_calls(call, stream, world, dev, K, W, flush, leg=name)[0]
+    sec = timed_calls(call, stream, world, dev, K, W, flush, leg=leg)[0]
     if gqa.device_status() != 0:
-        raise RuntimeError(f"device status error in the {name} timing")
+        raise RuntimeError(f"device status error in the {leg} timing")
     prefix = w.prefix.tolist() if chunk else [0] * B
     flops = packed_flops(w.lens, prefix, H, D)
     del t, ws, out, flush
     what = (f"{B} sequences, {prefix[0]} cached rows + a {w.lens[0]}-token chunk each, H{H} Hkv{Hkv} D{D}"
+            + (f", cache in shuffled {page_size}-row pages" if paged else "")
             if chunk else f"{B} packed sequences, lengths U[256,8192] (N={N}), H{H} Hkv{Hkv} D{D}")
     return {"value": round(whole_job_rate(flops * K, world, sec) / 1e12, 2), "unit": "TFLOP/s",
             "ms": round(1e3 * sec / K, 4), "workload": what, "flops_per_call": flops, "gpu_launches": 3 * K,

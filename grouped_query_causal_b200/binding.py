@@ -28,6 +28,7 @@ EXPORTS = ("gqa_status_string", "gqa_attn_prefill_workspace_size", "gqa_attn_pre
            "gqa_attn_prefill_khat_ex", "gqa_attn_decode_ex", "gqa_attn_decode_append_ex",
            "gqa_attn_decode_paged", "gqa_attn_decode_append_paged", "gqa_attn_prefill_varlen_workspace_size",
            "gqa_attn_prefill_varlen", "gqa_attn_prefill_chunk_workspace_size", "gqa_attn_prefill_chunk",
+           "gqa_attn_prefill_chunk_paged_workspace_size", "gqa_attn_prefill_chunk_paged",
            "gqa_linear", "gqa_attn_block_prefill_workspace_size", "gqa_attn_block_prefill",
            "gqa_attn_test_stall")
 
@@ -128,6 +129,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_attn_prefill_chunk_workspace_size.argtypes = [L, I]
     lib.gqa_attn_prefill_chunk_workspace_size.restype = Z
     lib.gqa_attn_prefill_chunk.argtypes = [P, P, P, P, P, P, P, P, P, L, P, P, R, F, P, I, L, I, I, I, I, P, Z, P]
+    lib.gqa_attn_prefill_chunk_paged_workspace_size.argtypes = [L, I]
+    lib.gqa_attn_prefill_chunk_paged_workspace_size.restype = Z
+    lib.gqa_attn_prefill_chunk_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, P, P, P, R, F, P, I, L, I, I, I, I, P,
+                                                 Z, P]
     lib.gqa_attn_test_stall.argtypes = [I]
     lib.gqa_attn_test_stall.restype = None
     lib.gqa_linear.argtypes = [P, P, P, I, L, I, I, P]
@@ -347,6 +352,42 @@ def prefill_chunk(q, k, v, pos, cu_seqlens, k_cache, v_cache, cache_offsets, pre
                                     Hkv, D, int(max_chunk_len), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _raise(st, "gqa_attn_prefill_chunk")
+    return out
+
+
+def prefill_chunk_paged(q, k, v, pos, cu_seqlens, k_pages, v_pages, page_table, prefix_len, qnorm_w, knorm_w,
+                        max_chunk_len: int, eps: float = 1e-6, rope: Optional[RopeConfig] = None,
+                        out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Chunked prefill on a paged cache: as prefill_chunk, with the cache in pages
+    (k_pages/v_pages [num_pages, page_size, Hkv, D], page_table [B, max_pages] int32)."""
+    lib = load()
+    for t, n, dt, d in ((q, "q", torch.bfloat16, 3), (k, "k", torch.bfloat16, 3), (v, "v", torch.bfloat16, 3),
+                        (pos, "pos", torch.int32, 1), (cu_seqlens, "cu_seqlens", torch.int64, 1),
+                        (k_pages, "k_pages", torch.bfloat16, 4), (v_pages, "v_pages", torch.bfloat16, 4),
+                        (page_table, "page_table", torch.int32, 2), (prefix_len, "prefix_len", torch.int32, 1),
+                        (qnorm_w, "qnorm_w", torch.float32, 1), (knorm_w, "knorm_w", torch.float32, 1)):
+        _check(t, n, dt, d)
+    N, H, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    num_pages, page_size = k_pages.shape[0], k_pages.shape[1]
+    if (k.shape != (N, Hkv, D) or v.shape != k.shape or pos.shape != (N,) or k_pages.shape[2:] != (Hkv, D)
+            or v_pages.shape != k_pages.shape or page_table.shape[0] != B or prefix_len.shape != (B,)):
+        raise ValueError("shape mismatch")
+    rope = rope if rope is not None else RopeConfig.make()
+    if out is None:
+        out = torch.empty((N, H, D), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 3)
+    need = int(lib.gqa_attn_prefill_chunk_paged_workspace_size(N, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib.gqa_attn_prefill_chunk_paged(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(cu_seqlens), _ptr(k_pages),
+                                          _ptr(v_pages), _ptr(page_table), num_pages, page_size, page_table.shape[1],
+                                          _ptr(prefix_len), _ptr(qnorm_w), _ptr(knorm_w), ctypes.byref(rope),
+                                          float(eps), _ptr(out), B, N, H, Hkv, D, int(max_chunk_len), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _raise(st, "gqa_attn_prefill_chunk_paged")
     return out
 
 

@@ -67,12 +67,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // 3-D bf16 tensor [rows][heads][128] (head vectors contiguous, `row_bytes` between rows),
 // box (64, 1, 128): half a head vector of 128 consecutive rows, 128-byte swizzle, zero
 // fill outside the tensor.
-bool make_rows_map(CUtensorMap *m, const void *base, uint64_t heads, uint64_t rows, uint64_t row_bytes) {
+bool make_rows_map(CUtensorMap *m, const void *base, uint64_t heads, uint64_t rows, uint64_t row_bytes,
+                   uint32_t box_rows = 128) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), heads, rows};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2, row_bytes};
-    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t box[3] = {64, 1, box_rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -228,6 +229,8 @@ struct KRows {
     const int32_t *prefix = nullptr;
     int B = 0;
     long long rows = 0;   // rows of the destination buffers
+    const int32_t *pages = nullptr;   // paged destination (with cu): page table [B, max_pages]
+    int page_size = 0, max_pages = 0, num_pages = 0;
 };
 
 // Enqueue the k-hat prologue (arguments already validated).  k rows are k_stride
@@ -248,6 +251,10 @@ gqa_status launch_k_norm_rope(const void *k, long long k_stride, const void *v, 
     kp.cu = dst.cu;
     kp.cache_off = dst.cache_off;
     kp.prefix = dst.prefix;
+    kp.pages = dst.pages;
+    kp.page_size = dst.page_size;
+    kp.max_pages = dst.max_pages;
+    kp.num_pages = dst.num_pages;
     kp.err = err;
     kp.ntok = ntok;
     kp.k_stride = k_stride;
@@ -280,6 +287,8 @@ struct AttnGeom {
     const int32_t *prefix = nullptr;
     long long max_prefix = 0;          // host-side bound on the cached keys before a chunk (scheduling only)
     void *ulist_ws = nullptr;          // packed inputs: room for the unit list (unit_list_bytes of nq_rows)
+    const int32_t *kv_pages = nullptr; // paged K/V: page table [B, kv_max_pages] (nkv_rows = kv_max_pages * kv_page_size)
+    int kv_page_size = 0, kv_max_pages = 0, kv_num_pages = 0;
 };
 
 // Makespan, in 128-key tiles plus a fixed cost per unit (the next unit's Q transform and
@@ -360,9 +369,13 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
     unsigned *err = device_error_word();
     if (!err) return GQA_ERR_CUDA;
     CUtensorMap tm_q, tm_k, tm_v;
+    // paged K/V: the maps cover the pages' rows, one box per page segment of a tile
+    const long long kv_map_rows =
+        gm.kv_pages != nullptr ? static_cast<long long>(gm.kv_num_pages) * gm.kv_page_size : gm.nkv_rows;
+    const uint32_t kv_box = gm.kv_pages != nullptr ? static_cast<uint32_t>(std::min(gm.kv_page_size, kBN)) : 128u;
     if (!make_rows_map(&tm_q, q, H, gm.nq_rows, gm.q_row_elems * 2) ||
-        !make_rows_map(&tm_k, k_hat, Hkv, gm.nkv_rows, gm.kv_row_elems * 2) ||
-        !make_rows_map(&tm_v, v, Hkv, gm.nkv_rows, (gm.v_row_elems ? gm.v_row_elems : gm.kv_row_elems) * 2))
+        !make_rows_map(&tm_k, k_hat, Hkv, kv_map_rows, gm.kv_row_elems * 2, kv_box) ||
+        !make_rows_map(&tm_v, v, Hkv, kv_map_rows, (gm.v_row_elems ? gm.v_row_elems : gm.kv_row_elems) * 2, kv_box))
         return GQA_ERR_CUDA;
     if (!attn_smem_attr_set()) return GQA_ERR_CUDA;
     AttnParams ap;
@@ -374,6 +387,12 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
     ap.cu_q = gm.cu_q;
     ap.kv_off = gm.kv_off;
     ap.prefix = gm.prefix;
+    ap.kv_pages = gm.kv_pages;
+    ap.kv_page_size = gm.kv_page_size;
+    ap.kv_max_pages = gm.kv_max_pages;
+    ap.kv_num_pages = gm.kv_num_pages;
+    ap.kv_segs = gm.kv_page_size > 0 && gm.kv_page_size < kBN ? kBN / gm.kv_page_size : 1;
+    ap.kv_seg_rows = kBN / ap.kv_segs;
     ap.nq_rows = gm.nq_rows;
     ap.nkv_rows = gm.nkv_rows;
     ap.B = gm.B;
@@ -406,8 +425,9 @@ gqa_status launch_attention(const void *q, const void *k_hat, const void *v, con
         int2 *list = static_cast<int2 *>(gm.ulist_ws);
         int *count = reinterpret_cast<int *>(static_cast<char *>(gm.ulist_ws) +
                                              round_up(static_cast<size_t>(list_cap) * 8, 256));
-        unit_list_kernel<<<1, 1024, 0, st>>>(gm.cu_q, gm.kv_off, gm.prefix, gm.nq_rows, gm.nkv_rows, gm.B, ap.nqb,
-                                             band, list, static_cast<int>(list_cap), count, err);
+        unit_list_kernel<<<1, 1024, 0, st>>>(gm.cu_q, gm.kv_off, gm.prefix, gm.kv_pages != nullptr, gm.nq_rows,
+                                             gm.nkv_rows, gm.B, ap.nqb, band, list, static_cast<int>(list_cap), count,
+                                             err);
         if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
         ap.ulist = list;
         ap.ulist_n = count;
@@ -656,6 +676,72 @@ extern "C" gqa_status gqa_attn_prefill_chunk(const void *q, const void *k, const
     gm.max_prefix = cache_rows / std::max(1, B);   // an average; only the schedule depends on it
     gm.ulist_ws = reinterpret_cast<char *>(table) + rope_table_bytes(1, static_cast<int>(N));
     return launch_attention(q, k_cache, v_cache, pos, table, qnorm_w, rs, eps, out, gm, H, Hkv, st);
+}
+
+extern "C" size_t gqa_attn_prefill_chunk_paged_workspace_size(int64_t N, int D) {
+    return gqa_attn_prefill_chunk_workspace_size(N, D);
+}
+
+extern "C" gqa_status gqa_attn_prefill_chunk_paged(const void *q, const void *k, const void *v, const int32_t *pos,
+                                                   const int64_t *cu_seqlens, void *k_pages, void *v_pages,
+                                                   const int32_t *page_table, int num_pages, int page_size,
+                                                   int max_pages, const int32_t *prefix_len, const float *qnorm_w,
+                                                   const float *knorm_w, const gqa_rope_config *rope, float eps,
+                                                   float *out, int B, int64_t N, int H, int Hkv, int D,
+                                                   int max_chunk_len, void *workspace, size_t workspace_bytes,
+                                                   void *stream) {
+    RopeSpec rs;
+    if (!rope_spec(rope, rs) || !eps_ok(eps)) return GQA_ERR_INVALID_ARG;
+    if (D != kHeadDim) return D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
+    if (!ragged_shape_ok(B, N, H, Hkv, max_chunk_len)) return GQA_ERR_INVALID_ARG;
+    if (num_pages <= 0 || max_pages <= 0 || page_size <= 0 || page_size % 16 != 0) return GQA_ERR_INVALID_ARG;
+    // a 128-key tile must be whole pages or lie inside one page
+    if (kBN % page_size != 0 && page_size % kBN != 0) return GQA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(num_pages) * page_size > (1LL << 31) - 256 ||
+        static_cast<long long>(max_pages) * page_size > (1LL << 31) - 256)
+        return GQA_ERR_INVALID_ARG;
+    if (B == 0 || N == 0 || max_chunk_len == 0) return GQA_OK;
+    if (!q || !k || !v || !pos || !cu_seqlens || !k_pages || !v_pages || !page_table || !prefix_len || !qnorm_w ||
+        !knorm_w || !out)
+        return GQA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(qnorm_w, 16) ||
+        !aligned(knorm_w, 16) || !aligned(pos, 4) || !aligned(cu_seqlens, 8) || !aligned(k_pages, 16) ||
+        !aligned(v_pages, 16) || !aligned(page_table, 4) || !aligned(prefix_len, 4))
+        return GQA_ERR_INVALID_ARG;
+    const size_t need = gqa_attn_prefill_chunk_paged_workspace_size(N, D);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *table = static_cast<float *>(workspace);
+    // the chunk's k-hat and v go into the pages after each sequence's cached rows ...
+    KRows dst;
+    dst.cu = cu_seqlens;
+    dst.prefix = prefix_len;
+    dst.B = B;
+    dst.rows = static_cast<long long>(num_pages) * page_size;
+    dst.pages = page_table;
+    dst.page_size = page_size;
+    dst.max_pages = max_pages;
+    dst.num_pages = num_pages;
+    const long long kv = static_cast<long long>(Hkv) * kHeadDim;
+    gqa_status s = launch_k_norm_rope(k, kv, v, kv, pos, knorm_w, rs, eps, k_pages, v_pages, table, N, Hkv, dst, st);
+    if (s != GQA_OK) return s;
+    // ... and the chunk's queries attend to all of them through the page table
+    AttnGeom gm;
+    gm.B = B;
+    gm.T = max_chunk_len;
+    gm.nq_rows = N;
+    gm.nkv_rows = static_cast<long long>(max_pages) * page_size;
+    gm.q_row_elems = static_cast<long long>(H) * kHeadDim;
+    gm.kv_row_elems = kv;
+    gm.cu_q = cu_seqlens;
+    gm.prefix = prefix_len;
+    gm.max_prefix = static_cast<long long>(num_pages) * page_size / std::max(1, B);   // scheduling only
+    gm.ulist_ws = reinterpret_cast<char *>(table) + rope_table_bytes(1, static_cast<int>(N));
+    gm.kv_pages = page_table;
+    gm.kv_page_size = page_size;
+    gm.kv_max_pages = max_pages;
+    gm.kv_num_pages = num_pages;
+    return launch_attention(q, k_pages, v_pages, pos, table, qnorm_w, rs, eps, out, gm, H, Hkv, st);
 }
 
 // ---------------------------------------------------------------- projections

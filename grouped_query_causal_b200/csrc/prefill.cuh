@@ -54,6 +54,10 @@ struct KPrologueParams {
     const int64_t *cu;        // [B + 1]
     const int64_t *cache_off; // [B + 1]
     const int32_t *prefix;    // [B]
+    // Paged destination (pages != nullptr, with cu): the token's row in its sequence,
+    // prefix[b] + n - cu[b], is row r % page_size of page pages[b * max_pages + r / page_size].
+    const int32_t *pages;
+    int page_size, max_pages, num_pages;
     unsigned *err;
     long long ntok, k_stride, v_stride, rows;
     int Hkv, B;
@@ -71,8 +75,15 @@ __device__ __forceinline__ long long k_prologue_row(const KPrologueParams &p, lo
         else hi = mid;
     }
     const long long c0 = p.cu[lo], c1 = p.cu[lo + 1];
-    const long long r0 = p.cache_off[lo], r1 = p.cache_off[lo + 1];
     const long long pre = p.prefix[lo];
+    if (p.pages != nullptr) {
+        const long long r = pre + (n - c0), pg = r / p.page_size;
+        if (!(c0 <= n && n < c1 && pre >= 0 && pg < p.max_pages)) return -1;
+        const int id = p.pages[static_cast<long long>(lo) * p.max_pages + pg];
+        if (id < 0 || id >= p.num_pages) return -1;
+        return static_cast<long long>(id) * p.page_size + (r - pg * p.page_size);
+    }
+    const long long r0 = p.cache_off[lo], r1 = p.cache_off[lo + 1];
     const long long row = r0 + pre + (n - c0);
     if (!(c0 <= n && n < c1 && pre >= 0 && r0 >= 0 && row < r1 && r1 <= p.rows)) return -1;
     return row;
@@ -256,8 +267,15 @@ struct AttnParams {
     const int64_t *cu_q;   // [B + 1] query-row offsets, or nullptr: b T
     const int64_t *kv_off; // [B] first K/V row, or nullptr: the query-row offset
     const int32_t *prefix; // [B] cached keys before the first query token, or nullptr: 0
+    // Paged K/V (kv_pages != nullptr): key row r of sequence b is row r % kv_page_size of page
+    // kv_pages[b * kv_max_pages + r / kv_page_size]; the tensor maps cover the pages' rows,
+    // in boxes of min(kv_page_size, 128) rows.
+    const int32_t *kv_pages;
+    int kv_page_size, kv_max_pages, kv_num_pages;
+    int kv_segs;           // page segments of a tile: 128 / kv_page_size, or 1 when a page holds whole tiles
+    int kv_seg_rows;       // rows of a segment: 128 / kv_segs
     long long nq_rows;     // rows of q / pos / out
-    long long nkv_rows;    // rows of k-hat / v
+    long long nkv_rows;    // rows of k-hat / v (paged: rows a sequence can address, kv_max_pages * kv_page_size)
     int B, T, H, Hkv, hpg, nqb, npairs, nunits;
     int band;              // KV groups (sequence, KV head) scheduled together: their K/V fit in L2
     // Packed inputs: the (sequence, query block) pairs that have work, in schedule order
@@ -327,7 +345,7 @@ __device__ __forceinline__ bool attn_unit(const AttnParams &p, int u, AttnUnit &
         q0 = p.cu_q[w.b];
         len = p.cu_q[w.b + 1] - q0;
     }
-    const long long kv0 = p.kv_off != nullptr ? p.kv_off[w.b] : q0;
+    const long long kv0 = p.kv_pages != nullptr ? 0 : p.kv_off != nullptr ? p.kv_off[w.b] : q0;
     const long long pre = p.prefix != nullptr ? p.prefix[w.b] : 0;
     if (q0 < 0 || len < 0 || q0 + len > p.nq_rows || len > static_cast<long long>(p.nqb) * kBM || pre < 0 ||
         kv0 < 0 || kv0 + pre + len > p.nkv_rows || pre + len > 0x7fff0000LL) {
@@ -520,6 +538,31 @@ __device__ __forceinline__ int attn_unit_count(const AttnParams &p) {
     return p.nunits;
 }
 
+// Paged K/V: the page ids of the segments of 128-key tile j of sequence b: kv_segs whole
+// pages (up to kMaxSegs, for 16-row pages), or the one page that holds the tile.  Segments
+// past the last visible key, lim, or past the table's row are not looked up (-1).  The
+// loads are independent, so they are in flight together.  Returns the tile's first row
+// inside its page (0 for whole pages).
+constexpr int kMaxSegs = 128 / 16;
+static_assert(kMaxSegs * 16 == kBN, "a 16-row page is the smallest segment");
+__device__ __forceinline__ int kv_page_ids(const AttnParams &p, int b, int j, int lim, int (&ids)[kMaxSegs]) {
+    const int32_t *row = p.kv_pages + static_cast<long long>(b) * p.kv_max_pages;
+    const int key = j * kBN;
+    if (p.kv_segs == 1) {
+        const int pg = key / p.kv_page_size;
+        ids[0] = (key < lim && pg < p.kv_max_pages) ? __ldg(row + pg) : -1;
+#pragma unroll
+        for (int i = 1; i < kMaxSegs; ++i) ids[i] = -1;
+        return key - pg * p.kv_page_size;
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxSegs; ++i) {
+        const int pg = j * p.kv_segs + i;
+        ids[i] = (i < p.kv_segs && pg * p.kv_page_size < lim && pg < p.kv_max_pages) ? __ldg(row + pg) : -1;
+    }
+    return 0;
+}
+
 // The (sequence, query block) pairs of a packed launch that have work, in the order the
 // attention kernel deals them out: bands of `band` sequences (whose K/V fit in L2 together),
 // inside a band query blocks latest first, then the sequences of the band.  Units past the end
@@ -528,8 +571,9 @@ __device__ __forceinline__ int attn_unit_count(const AttnParams &p) {
 // gives each range its place, and each writes its entries.  A sequence whose bounds are out
 // of range gets no entries and sets kErrInput.
 __global__ void __launch_bounds__(1024) unit_list_kernel(const int64_t *cu, const int64_t *kv_off, const int32_t *prefix,
-                                                       long long nq_rows, long long nkv_rows, int B, int nqb, int band,
-                                                       int2 *list, int cap, int *count, unsigned *err) {
+                                                       bool kv_paged, long long nq_rows, long long nkv_rows, int B,
+                                                       int nqb, int band, int2 *list, int cap, int *count,
+                                                       unsigned *err) {
     __shared__ int warp_sum[32];
     const long long per_band = static_cast<long long>(band) * nqb;
     const long long slots = (static_cast<long long>(B) + band - 1) / band * per_band;
@@ -542,7 +586,7 @@ __global__ void __launch_bounds__(1024) unit_list_kernel(const int64_t *cu, cons
         b = static_cast<int>(bi * band + rem % band);
         if (b >= B) return -1;
         const long long q0 = cu[b], len = cu[b + 1] - q0;
-        const long long kv0 = kv_off != nullptr ? kv_off[b] : q0;
+        const long long kv0 = kv_paged ? 0 : kv_off != nullptr ? kv_off[b] : q0;
         const long long pre = prefix != nullptr ? prefix[b] : 0;
         if (q0 < 0 || len < 0 || q0 + len > nq_rows || len > static_cast<long long>(nqb) * 128 || pre < 0 ||
             kv0 < 0 || kv0 + pre + len > nkv_rows || pre + len > 0x7fff0000LL) {
@@ -672,6 +716,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     if (bad) atomicOr(p.err, kErrInput);
                     continue;
                 }
+                // paged K/V: the page ids of a tile's segments (whole pages, or one slice of a
+                // page), loaded together one tile ahead and used for both K and V; a segment
+                // with no visible key is not looked up
+                const int kv_lim = w.key0 + w.rows;
+                int pid_cur[kMaxSegs], pid_nxt[kMaxSegs], poff_cur = 0, poff_nxt = 0;
+                if (p.kv_pages != nullptr) poff_cur = kv_page_ids(p, w.b, 0, kv_lim, pid_cur);
                 if (p.rope_cs != nullptr) {   // the table blocks holding this query block's tokens
                     for (long long blk = w.q0 >> 7; blk <= ((w.q0 + w.rows - 1) >> 7); ++blk)
                         prefetch_l2_bulk(p.rope_cs + rope_table_index(blk << 7, 0) * 4, 32 * 128 * 16);
@@ -710,8 +760,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         mbar_arrive_expect_tx(bar, j + 1 < w.n_kv ? 2 * kTileBytes : kTileBytes);
                         ++armed;
                     }
-                    tma_load_3d(dst, m, 0, w.g, row, bar);
-                    tma_load_3d(dst + kBoxBytes, m, 64, w.g, row, bar);
+                    if (p.kv_pages == nullptr) {
+                        tma_load_3d(dst, m, 0, w.g, row, bar);
+                        tma_load_3d(dst + kBoxBytes, m, 64, w.g, row, bar);
+                    } else {
+                        // one box per segment; a segment with no visible key, or behind a bad
+                        // page id (reported once, with K), is read as zeros: a row past the
+                        // pages' rows
+                        const int ps = p.kv_page_size, seg = p.kv_seg_rows;
+#pragma unroll
+                        for (int i = 0; i < kMaxSegs; ++i) {
+                            if (i >= p.kv_segs) break;
+                            const int id = pid_cur[i];
+                            int prow = p.kv_num_pages * ps;
+                            if (row + i * seg < kv_lim) {
+                                if (id >= 0 && id < p.kv_num_pages) prow = id * ps + poff_cur;
+                                else if (!(k & 1)) atomicOr(p.err, kErrInput);
+                            }
+                            const uint32_t off = static_cast<uint32_t>(i * seg) * 128u;
+                            tma_load_3d(dst + off, m, 0, w.g, prow, bar);
+                            tma_load_3d(dst + kBoxBytes + off, m, 64, w.g, prow, bar);
+                        }
+                        if (!(k & 1)) {   // K_j issued: fetch tile j+1's ids while the ring turns
+                            if ((k >> 1) + 1 < w.n_kv) poff_nxt = kv_page_ids(p, w.b, (k >> 1) + 1, kv_lim, pid_nxt);
+                        } else if ((k >> 1) + 1 < w.n_kv) {
+#pragma unroll
+                            for (int i = 0; i < kMaxSegs; ++i) pid_cur[i] = pid_nxt[i];
+                            poff_cur = poff_nxt;
+                        }
+                    }
                 }
                 if (ok) gs += w.n_kv;
             }

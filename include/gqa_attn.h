@@ -361,6 +361,8 @@ gqa_status gqa_attn_prefill_varlen(const void *q, const void *k, const void *v, 
  * A chunk token whose cache row falls outside its sequence's rows is not written and
  * sets GQA_ERR_DEVICE_INPUT (that sequence's output is then undefined); the same for
  * sequence bounds out of range.  prefix_len is not advanced (the caller does that).
+ * Keys are read in 128-row tiles from cache_offsets[b]: up to 127 cache rows after a
+ * sequence's last key are read and weighted by zero, so they must hold finite values.
  */
 size_t gqa_attn_prefill_chunk_workspace_size(int64_t N, int D);
 gqa_status gqa_attn_prefill_chunk(const void *q, const void *k, const void *v, const int32_t *pos,
@@ -370,6 +372,37 @@ gqa_status gqa_attn_prefill_chunk(const void *q, const void *k, const void *v, c
                                   const gqa_rope_config *rope, float eps, float *out, int B,
                                   int64_t N, int H, int Hkv, int D, int max_chunk_len,
                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Chunked prefill on a paged KV cache: as gqa_attn_prefill_chunk, with cached row r of
+ * sequence b kept as row r % page_size of page page_table[b * max_pages + r / page_size]
+ * (the decode-side paged layout).  The chunk's k-hat and v are written into the pages at
+ * rows prefix_len[b] .. prefix_len[b] + chunk length - 1 of the sequence, then the chunk
+ * attends to rows 0 .. prefix_len[b] + t through the page table.
+ *
+ *   k_pages, v_pages  bf16 [num_pages, page_size, Hkv, D]; the pages the table names for the
+ *                     chunk's rows must exist (allocated by the caller)
+ *   page_table        int32 [B, max_pages], device; entries past a sequence's rows are unused
+ *   page_size         a multiple of 16 that divides 128 or is a multiple of 128 (so that a
+ *                     128-key tile is whole pages or lies inside one page), else
+ *                     GQA_ERR_UNSUPPORTED; num_pages * page_size < 2^31 - 256
+ *   workspace >= gqa_attn_prefill_chunk_paged_workspace_size(N, D) bytes (as for
+ *             gqa_attn_prefill_chunk).
+ * A chunk row behind a page id outside [0, num_pages) (or past max_pages) is not written,
+ * and a visible key behind one is read as zero; both set GQA_ERR_DEVICE_INPUT and leave that
+ * sequence's output undefined.  Page segments of a 128-key tile past a sequence's last key
+ * are not read; the rows after the last key inside its last page are read and weighted by
+ * zero, so they must hold finite values (zeros, or any earlier contents of the cache).
+ */
+size_t gqa_attn_prefill_chunk_paged_workspace_size(int64_t N, int D);
+gqa_status gqa_attn_prefill_chunk_paged(const void *q, const void *k, const void *v, const int32_t *pos,
+                                        const int64_t *cu_seqlens, void *k_pages, void *v_pages,
+                                        const int32_t *page_table, int num_pages, int page_size,
+                                        int max_pages, const int32_t *prefix_len, const float *qnorm_w,
+                                        const float *knorm_w, const gqa_rope_config *rope, float eps,
+                                        float *out, int B, int64_t N, int H, int Hkv, int D,
+                                        int max_chunk_len, void *workspace, size_t workspace_bytes,
+                                        void *stream);
 
 /* ----------------------------------------------------------------- paged KV cache
  *

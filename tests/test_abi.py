@@ -182,6 +182,37 @@ def test_paged_decode_argument_errors_are_caught_on_the_host(lib):
                                             2, 128, 64, 256, 1 << 20, None) == -1
 
 
+def test_paged_chunk_argument_errors_are_caught_on_the_host(lib):
+    r = ctypes.byref(_rope())
+
+    def chunk(**kw):
+        a = dict(q=16, k=16, v=16, pos=16, cu=16, kp=16, vp=16, tab=16, npages=10, ps=16, maxp=4, pl=16, wq=16,
+                 wk=16, rope=r, eps=1e-6, out=16, B=2, N=40, H=8, Hkv=2, D=128, mcl=32, ws=256, wsb=1 << 20)
+        a.update(kw)
+        return lib.gqa_attn_prefill_chunk_paged(a["q"], a["k"], a["v"], a["pos"], a["cu"], a["kp"], a["vp"], a["tab"],
+                                                a["npages"], a["ps"], a["maxp"], a["pl"], a["wq"], a["wk"], a["rope"],
+                                                a["eps"], a["out"], a["B"], a["N"], a["H"], a["Hkv"], a["D"],
+                                                a["mcl"], a["ws"], a["wsb"], None)
+    assert chunk(ps=8) == -1        # page size must be a multiple of 16
+    assert chunk(ps=48) == -2       # ... that divides 128 or is a multiple of it
+    assert chunk(ps=160) == -2
+    assert chunk(npages=0) == -1
+    assert chunk(maxp=0) == -1
+    assert chunk(npages=1 << 27, ps=16) == -1   # page rows must stay below 2^31 - 256
+    assert chunk(tab=None) == -1
+    assert chunk(tab=18) == -1      # int32 table must be 4-byte aligned
+    assert chunk(kp=24) == -1
+    assert chunk(cu=20) == -1
+    assert chunk(rope=None) == -1
+    assert chunk(D=64) == -2
+    assert chunk(H=8, Hkv=3) == -1
+    assert chunk(wsb=10) == -3
+    assert chunk(ws=128) == -3
+    assert chunk(B=0) == 0
+    assert chunk(N=0, q=None) == 0
+    assert lib.gqa_attn_prefill_chunk_paged_workspace_size(40, 128) == lib.gqa_attn_prefill_chunk_workspace_size(40, 128)
+
+
 def test_binding_fails_loudly_without_the_library(tmp_path):
     saved = binding._lib
     binding._lib = None
