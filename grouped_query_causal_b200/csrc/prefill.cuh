@@ -538,29 +538,23 @@ __device__ __forceinline__ int attn_unit_count(const AttnParams &p) {
     return p.nunits;
 }
 
-// Paged K/V: the page ids of the segments of 128-key tile j of sequence b: kv_segs whole
-// pages (up to kMaxSegs, for 16-row pages), or the one page that holds the tile.  Segments
-// past the last visible key, lim, or past the table's row are not looked up (-1).  The
-// loads are independent, so they are in flight together.  Returns the tile's first row
-// inside its page (0 for whole pages).
+// Paged K/V: the page id of segment i of 128-key tile j of sequence b.  A tile is kv_segs
+// whole pages (up to kMaxSegs, for 16-row pages) or lies inside one page.  A segment past
+// the tile, past the last visible key, lim, or past the table's row is not looked up (-1).
+// off is the tile's first row inside the page (0 for whole pages).
 constexpr int kMaxSegs = 128 / 16;
-static_assert(kMaxSegs * 16 == kBN, "a 16-row page is the smallest segment");
-__device__ __forceinline__ int kv_page_ids(const AttnParams &p, int b, int j, int lim, int (&ids)[kMaxSegs]) {
+static_assert(kMaxSegs * 16 == kBN && 2 * kMaxSegs <= 32, "one lane per box of a 16-row-page tile");
+__device__ __forceinline__ int kv_page_id(const AttnParams &p, int b, int j, int lim, int i, int &off) {
     const int32_t *row = p.kv_pages + static_cast<long long>(b) * p.kv_max_pages;
     const int key = j * kBN;
     if (p.kv_segs == 1) {
         const int pg = key / p.kv_page_size;
-        ids[0] = (key < lim && pg < p.kv_max_pages) ? __ldg(row + pg) : -1;
-#pragma unroll
-        for (int i = 1; i < kMaxSegs; ++i) ids[i] = -1;
-        return key - pg * p.kv_page_size;
+        off = key - pg * p.kv_page_size;
+        return (i == 0 && key < lim && pg < p.kv_max_pages) ? __ldg(row + pg) : -1;
     }
-#pragma unroll
-    for (int i = 0; i < kMaxSegs; ++i) {
-        const int pg = j * p.kv_segs + i;
-        ids[i] = (i < p.kv_segs && pg * p.kv_page_size < lim && pg < p.kv_max_pages) ? __ldg(row + pg) : -1;
-    }
-    return 0;
+    const int pg = j * p.kv_segs + i;
+    off = 0;
+    return (i < p.kv_segs && pg * p.kv_page_size < lim && pg < p.kv_max_pages) ? __ldg(row + pg) : -1;
 }
 
 // The (sequence, query block) pairs of a packed launch that have work, in the order the
@@ -700,49 +694,61 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     regs_dec<kRegsCtl>();
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+        // Lane 0 walks the schedule, waits for free buffers and arms the barriers.  With
+        // paged K/V the whole warp walks it: each lane issues one box of a tile (a half of
+        // one page segment), so a tile of 16-row pages is one warp instruction, not 16
+        // issued one after the other; every lane waits for the buffer it writes itself.
+        const bool paged = p.kv_pages != nullptr;
+        const unsigned wmask = paged ? 0xffffffffu : 1u;
+        if (lane == 0 || paged) {
             bool ok = true;
             uint32_t q_uses[2] = {0u, 0u};   // Q loads per slot so far
             uint32_t k0_uses = 0;            // units so far (first K tiles)
             uint32_t it = 0;                 // K/V ring items so far (K0 V0 K1 V1 ... per unit)
             uint32_t gs = 0;                 // steps so far (one per K/V tile pair)
             uint32_t armed = 0;                     // steps armed so far (step k on barrier k % 3)
+            // paged: this lane's box is half (lane & 1) of segment lane >> 1 of the tile
+            const int seg_i = lane >> 1, half = lane & 1;
             for (int r = 0; ok; ++r) {
                 const int u = attn_unit_of_round(r);
                 if (u >= nun) break;
                 AttnUnit w;
                 bool bad;
                 if (!attn_unit<LISTED>(p, u, w, bad)) {
-                    if (bad) atomicOr(p.err, kErrInput);
+                    if (bad && lane == 0) atomicOr(p.err, kErrInput);
                     continue;
                 }
-                // paged K/V: the page ids of a tile's segments (whole pages, or one slice of a
-                // page), loaded together one tile ahead and used for both K and V; a segment
-                // with no visible key is not looked up
+                // paged K/V: the page id of this lane's segment, loaded one tile ahead and
+                // used for both K and V; a segment with no visible key is not looked up
                 const int kv_lim = w.key0 + w.rows;
-                int pid_cur[kMaxSegs], pid_nxt[kMaxSegs], poff_cur = 0, poff_nxt = 0;
-                if (p.kv_pages != nullptr) poff_cur = kv_page_ids(p, w.b, 0, kv_lim, pid_cur);
-                if (p.rope_cs != nullptr) {   // the table blocks holding this query block's tokens
-                    for (long long blk = w.q0 >> 7; blk <= ((w.q0 + w.rows - 1) >> 7); ++blk)
-                        prefetch_l2_bulk(p.rope_cs + rope_table_index(blk << 7, 0) * 4, 32 * 128 * 16);
-                }
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {   // unrolled: the per-slot counters stay in registers
-                    if (s >= w.nslots || !ok) break;
-                    // the slot is free once the previous unit's last Q K^T on it has finished
-                    if (q_uses[s] > 0 && !mbar_wait(BAR(BAR_Q_EMPTY + s), (q_uses[s] - 1) & 1, p.err)) {
-                        ok = false;
-                        break;
+                int pid_cur = -1, pid_nxt = -1, poff_cur = 0, poff_nxt = 0;
+                if (paged) pid_cur = kv_page_id(p, w.b, 0, kv_lim, seg_i, poff_cur);
+                if (lane == 0) {
+                    if (p.rope_cs != nullptr) {   // the table blocks holding this query block's tokens
+                        for (long long blk = w.q0 >> 7; blk <= ((w.q0 + w.rows - 1) >> 7); ++blk)
+                            prefetch_l2_bulk(p.rope_cs + rope_table_index(blk << 7, 0) * 4, 32 * 128 * 16);
                     }
-                    const uint32_t dst = sQ0 + s * kTileBytes;
-                    mbar_arrive_expect_tx(BAR(BAR_Q_FULL + s), kTileBytes);
-                    tma_load_3d(dst, &tm_q, 0, w.hq0 + s, static_cast<int>(w.q0), BAR(BAR_Q_FULL + s));
-                    tma_load_3d(dst + kBoxBytes, &tm_q, 64, w.hq0 + s, static_cast<int>(w.q0), BAR(BAR_Q_FULL + s));
-                    ++q_uses[s];
+#pragma unroll
+                    for (int s = 0; s < 2; ++s) {   // unrolled: the per-slot counters stay in registers
+                        if (s >= w.nslots || !ok) break;
+                        // the slot is free once the previous unit's last Q K^T on it has finished
+                        if (q_uses[s] > 0 && !mbar_wait(BAR(BAR_Q_EMPTY + s), (q_uses[s] - 1) & 1, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t dst = sQ0 + s * kTileBytes;
+                        mbar_arrive_expect_tx(BAR(BAR_Q_FULL + s), kTileBytes);
+                        tma_load_3d(dst, &tm_q, 0, w.hq0 + s, static_cast<int>(w.q0), BAR(BAR_Q_FULL + s));
+                        tma_load_3d(dst + kBoxBytes, &tm_q, 64, w.hq0 + s, static_cast<int>(w.q0),
+                                    BAR(BAR_Q_FULL + s));
+                        ++q_uses[s];
+                    }
                 }
+                ok = __shfl_sync(wmask, ok, 0);
                 for (int k = 0; k < 2 * w.n_kv && ok; ++k, ++it) {   // K0, V0, K1, V1, ...
                     const uint32_t buf = it % kStages, use = it / kStages;
-                    if (use > 0 && !mbar_wait(BAR(BAR_KV_EMPTY + buf), (use - 1) & 1, p.err)) {
+                    if (use > 0 && !mbar_wait(BAR(BAR_KV_EMPTY + buf), (use - 1) & 1, p.err)) ok = false;
+                    if (!__all_sync(wmask, ok)) {
                         ok = false;
                         break;
                     }
@@ -754,45 +760,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     const int j = (k - 1) >> 1;
                     const uint32_t bar = k == 0 ? BAR(BAR_K0_FULL) : BAR(BAR_STEP_FULL + (gs + j) % 3);
                     if (k == 0) {
-                        mbar_arrive_expect_tx(bar, kTileBytes);
+                        if (lane == 0) mbar_arrive_expect_tx(bar, kTileBytes);
                         ++k0_uses;
                     } else if (k & 1) {
-                        mbar_arrive_expect_tx(bar, j + 1 < w.n_kv ? 2 * kTileBytes : kTileBytes);
+                        if (lane == 0) mbar_arrive_expect_tx(bar, j + 1 < w.n_kv ? 2 * kTileBytes : kTileBytes);
                         ++armed;
                     }
-                    if (p.kv_pages == nullptr) {
+                    if (!paged) {
                         tma_load_3d(dst, m, 0, w.g, row, bar);
                         tma_load_3d(dst + kBoxBytes, m, 64, w.g, row, bar);
                     } else {
-                        // one box per segment; a segment with no visible key, or behind a bad
-                        // page id (reported once, with K), is read as zeros: a row past the
-                        // pages' rows
-                        const int ps = p.kv_page_size, seg = p.kv_seg_rows;
-#pragma unroll
-                        for (int i = 0; i < kMaxSegs; ++i) {
-                            if (i >= p.kv_segs) break;
-                            const int id = pid_cur[i];
+                        // a segment with no visible key, or behind a bad page id (reported
+                        // once, with K), is read as zeros: a row past the pages' rows.  The
+                        // boxes go out after lane 0 has armed the barrier.
+                        __syncwarp();
+                        if (seg_i < p.kv_segs) {
+                            const int ps = p.kv_page_size;
                             int prow = p.kv_num_pages * ps;
-                            if (row + i * seg < kv_lim) {
-                                if (id >= 0 && id < p.kv_num_pages) prow = id * ps + poff_cur;
-                                else if (!(k & 1)) atomicOr(p.err, kErrInput);
+                            if (row + seg_i * p.kv_seg_rows < kv_lim) {
+                                if (pid_cur >= 0 && pid_cur < p.kv_num_pages) prow = pid_cur * ps + poff_cur;
+                                else if (!(k & 1) && half == 0) atomicOr(p.err, kErrInput);
                             }
-                            const uint32_t off = static_cast<uint32_t>(i * seg) * 128u;
-                            tma_load_3d(dst + off, m, 0, w.g, prow, bar);
-                            tma_load_3d(dst + kBoxBytes + off, m, 64, w.g, prow, bar);
+                            const uint32_t off = static_cast<uint32_t>(half) * kBoxBytes +
+                                                 static_cast<uint32_t>(seg_i * p.kv_seg_rows) * 128u;
+                            tma_load_3d(dst + off, m, 64 * half, w.g, prow, bar);
                         }
-                        if (!(k & 1)) {   // K_j issued: fetch tile j+1's ids while the ring turns
-                            if ((k >> 1) + 1 < w.n_kv) poff_nxt = kv_page_ids(p, w.b, (k >> 1) + 1, kv_lim, pid_nxt);
-                        } else if ((k >> 1) + 1 < w.n_kv) {
-#pragma unroll
-                            for (int i = 0; i < kMaxSegs; ++i) pid_cur[i] = pid_nxt[i];
+                        if (!(k & 1)) {   // K_j issued: fetch tile j+1's id while the ring turns
+                            if ((k >> 1) + 1 < w.n_kv)
+                                pid_nxt = kv_page_id(p, w.b, (k >> 1) + 1, kv_lim, seg_i, poff_nxt);
+                        } else {
+                            pid_cur = pid_nxt;
                             poff_cur = poff_nxt;
                         }
                     }
                 }
                 if (ok) gs += w.n_kv;
             }
-            if (!ok) {
+            if (!ok && lane == 0) {
                 // Failure path: let every copy still in flight land before the CTA exits.  No
                 // barrier is re-armed before its previous phase completed, so waiting for the
                 // last armed phase of each covers every copy (a step barrier armed for two
