@@ -1,5 +1,6 @@
 """Seeded sweep of small random problems through the C ABI against the fp64 oracle, every
-output row: dense prefill, packed variable-length prefill, contiguous and paged decode, over
+output row: dense prefill, packed variable-length prefill, chunked prefill on a paged cache,
+contiguous and paged decode, over
 random batch sizes, lengths (ragged tails, single tokens), head groupings (MHA to MQA, odd
 heads per group), positions and RoPE variants.  The draws are fixed by the seed, so a failure
 names a reproducible case.  Tolerance: max-abs 2e-2, mean-abs 2e-3 per element."""
@@ -100,3 +101,45 @@ def test_decode_sweep(gqa, case):
     what = f"decode case {case}: seqlens {seqlens} H{H} Hkv{Hkv} {kw}"
     assert_close(out.cpu().numpy(), ref, what)
     assert_close(paged.cpu().numpy(), ref, f"paged ({page}-row pages) " + what)
+
+
+@pytest.mark.parametrize("case", range(8))
+def test_paged_chunk_sweep(gqa, case):
+    rng, H, Hkv, kw = _draw(300 + case)
+    B = int(rng.integers(1, 5))
+    prefix = [int(x) for x in rng.choice([0, 1, 15, 16, 127, 128, 300, 1000], size=B)]
+    chunk = [int(x) for x in rng.choice([1, 2, 64, 129, 200, 384], size=B)]
+    page = int(rng.choice([16, 32, 64, 128, 256]))
+    N = int(sum(chunk))
+    inp = synthetic.prefill_inputs(1, N, H, Hkv, seed=9500 + case)
+    q, k, v = inp.q[0].contiguous(), inp.k[0].contiguous(), inp.v[0].contiguous()
+    pos = torch.cat([torch.arange(p, p + c, dtype=torch.int32) for p, c in zip(prefix, chunk)])
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(chunk)]), dtype=torch.int64)
+    ro, rc = oracle.Rope(theta=inp.theta, **kw), gqa.RopeConfig.make(theta=inp.theta, **kw)
+    # the cached prefix: the oracle's k-hat of random raw keys at positions 0 .. P-1, random values
+    g = torch.Generator().manual_seed(9600 + case)
+    caps = [p + c for p, c in zip(prefix, chunk)]
+    offs = np.concatenate([[0], np.cumsum(caps)]).astype(np.int64)
+    kc = torch.zeros(int(offs[-1]), Hkv, 128, dtype=torch.bfloat16)
+    vc = torch.randn(int(offs[-1]), Hkv, 128, generator=g).to(torch.bfloat16)
+    for b, p in enumerate(prefix):
+        if p:
+            raw = torch.randn(p, Hkv, 128, generator=g).to(torch.bfloat16)
+            kh = oracle.qk_transform_ex(bits(raw), np.arange(p, dtype=np.int32), inp.wk.numpy(), ro, inp.eps)
+            kc[offs[b]:offs[b] + p] = torch.from_numpy(kh).to(torch.bfloat16)
+    pc = synthetic.page_cache(kc, vc, offs, caps, page, seed=9700 + case)
+    out = gqa.prefill_chunk_paged(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), cu.cuda(), pc.k_pages.cuda(),
+                                  pc.v_pages.cuda(), pc.page_table.cuda(), torch.tensor(prefix, dtype=torch.int32).cuda(),
+                                  inp.wq.cuda(), inp.wk.cuda(), max_chunk_len=max(chunk), eps=inp.eps, rope=rc)
+    torch.cuda.synchronize()
+    gqa.check_device_status()
+    got = out.cpu().numpy()
+    table = pc.page_table.numpy()
+    for b, (p, c) in enumerate(zip(prefix, chunk)):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        ref, _ = oracle.prefill_chunk_paged_ex(
+            bits(q[lo:hi]).reshape(1, c, H, 128), bits(k[lo:hi]).reshape(1, c, Hkv, 128),
+            bits(v[lo:hi]).reshape(1, c, Hkv, 128), bits(pc.k_pages), bits(pc.v_pages), table[b:b + 1], page,
+            np.array([p], np.int32), pos[lo:hi].numpy().reshape(1, c), inp.wq.numpy(), inp.wk.numpy(), ro, inp.eps)
+        assert_close(got[lo:hi], ref[0], f"paged chunk case {case}, sequence {b}: P={prefix} C={chunk} "
+                                         f"page {page} H{H} Hkv{Hkv} {kw}")
