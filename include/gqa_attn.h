@@ -383,16 +383,16 @@ gqa_status gqa_attn_prefill_chunk(const void *q, const void *k, const void *v, c
  *   k_pages, v_pages  bf16 [num_pages, page_size, Hkv, D]; the pages the table names for the
  *                     chunk's rows must exist (allocated by the caller)
  *   page_table        int32 [B, max_pages], device; entries past a sequence's rows are unused
- *   page_size         a multiple of 16 that divides 128 or is a multiple of 128 (so that a
- *                     128-key tile is whole pages or lies inside one page), else
- *                     GQA_ERR_UNSUPPORTED; num_pages * page_size < 2^31 - 256
+ *   page_size         a multiple of 16 (else GQA_ERR_INVALID_ARG) that divides 128 or is a
+ *                     multiple of 128 (so that a 128-key tile is whole pages or lies inside
+ *                     one page; else GQA_ERR_UNSUPPORTED); num_pages * page_size < 2^31 - 256
  *   workspace >= gqa_attn_prefill_chunk_paged_workspace_size(N, D) bytes (as for
  *             gqa_attn_prefill_chunk).
  * A chunk row behind a page id outside [0, num_pages) (or past max_pages) is not written,
  * and a visible key behind one is read as zero; both set GQA_ERR_DEVICE_INPUT and leave that
  * sequence's output undefined.  Page segments of a 128-key tile past a sequence's last key
  * are not read; the rows after the last key inside its last page are read and weighted by
- * zero, so they must hold finite values (zeros, or any earlier contents of the cache).
+ * zero, so they must hold finite values (zeros, or finite rows written earlier).
  */
 size_t gqa_attn_prefill_chunk_paged_workspace_size(int64_t N, int D);
 gqa_status gqa_attn_prefill_chunk_paged(const void *q, const void *k, const void *v, const int32_t *pos,

@@ -2,8 +2,8 @@
 the C ABI: outputs against the fp64 oracle (max-abs 2e-2, mean-abs 2e-3 per element) and
 bit for bit against the contiguous-cache chunk on the same rows; the chunk's k-hat and v
 land in the pages the table names, bit for bit as the contiguous chunk writes them, and
-every other page row is untouched.  Page sizes 16 .. 256, pages handed out in a shuffled
-order, prefixes that end inside a page."""
+every other page row is untouched.  Page sizes 16 to 512 (384 included), pages handed out
+in a shuffled order, prefixes that end inside a page."""
 import numpy as np
 import pytest
 import torch
