@@ -119,6 +119,42 @@ def test_unequal_bands_odd_groups_strided_rows(gqa):
     assert_close(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, f"unequal bands, {len(rows)} rows")
 
 
+def _aligned_keys_inputs(T, H, Hkv, seed):
+    """Queries all near one direction u; keys random for the first 256 tokens, then turning
+    towards u tile by tile, so a row's scores keep rising past its first tile's maximum."""
+    inp = synthetic.prefill_inputs(1, T, H, Hkv, seed=seed)
+    g = torch.Generator().manual_seed(seed + 7)
+    u = torch.randn(128, generator=g)
+    inp.q = (u + 0.1 * torch.randn(1, T, H, 128, generator=g)).to(torch.bfloat16)
+    k = torch.randn(1, T, Hkv, 128, generator=g)
+    t = torch.arange(T, dtype=torch.float32)
+    ang = ((t - 256).clamp(min=0) / max(1, T - 256) * (np.pi / 2)).view(1, T, 1, 1)
+    inp.k = (torch.cos(ang) * k + torch.sin(ang) * 3.0 * u).to(torch.bfloat16)
+    return inp
+
+
+def test_running_max_growth_rescales(gqa):
+    """Scores that grow along the keys by more than 2^8 (base 2) over a row's first tile drive
+    the softmax's exact-maximum pass and the rescale of l and O; every row against the
+    oracle.  The inputs are checked to reach that case for many rows."""
+    T, H, Hkv = 640, 4, 2
+    inp = _aligned_keys_inputs(T, H, Hkv, seed=190)
+    ro = oracle.Rope(theta=inp.theta)
+    qh = oracle.qk_transform_ex(bits_of(inp.q[0]), inp.pos[0].numpy(), inp.wq.numpy(), ro, inp.eps)
+    kh = oracle.qk_transform_ex(bits_of(inp.k[0]), inp.pos[0].numpy(), inp.wk.numpy(), ro, inp.eps)
+    grows = 0
+    for h in range(H):
+        sc = qh[:, h, :] @ kh[:, h // (H // Hkv), :].T / np.sqrt(128.0) * np.log2(np.e)
+        for i in range(128, T):
+            first = sc[i, :128].max()
+            later = sc[i, 128:i + 1].max()
+            grows += later > first + 8.0
+    assert grows > 500, grows
+    got = _run(gqa, inp)
+    ref = oracle.prefill(*oracle_prefill_args(inp))
+    assert_close(got, ref, "scores growing along the keys")
+
+
 def test_empty_problem_is_noop(gqa):
     dev = "cuda"
     q = torch.empty((0, 5, 4, 128), dtype=torch.bfloat16, device=dev)
