@@ -531,22 +531,63 @@ void oracle_decode_append(const uint16_t *q, const uint16_t *k_new, const uint16
     free(f);
 }
 
+/* One output row of the chunk: chunk row i of query head hq of sequence b against the
+ * sequence's P_b cached rows (k-hat and v, from row offsets[b] on) and the chunk's k-hat
+ * rows 0 .. i (khat [B, C, Hkv, D], already computed).  Scratch: tmp, qi [D]; s, p
+ * [P_b + C]; vbuf [(P_b + C) * D]; vr [P_b + C]. */
+static void chunk_one_row(const uint16_t *q, const uint16_t *v, const uint16_t *k_cache,
+                          const uint16_t *v_cache, const int64_t *offsets, const int32_t *prefix_len,
+                          const int32_t *pos, const double *wqd, const double *inv_freq, int pairing,
+                          double inv_sqrt_d, double eps, int C, int H, int Hkv, int D, const double *khat,
+                          int b, int hq, int i, double *tmp, double *qi, double *s, double *p, double *vbuf,
+                          const double **vr, double *out_row)
+{
+    int g = hq / (H / Hkv);
+    int32_t P = prefix_len[b];
+    int64_t n = (int64_t)b * C + i;
+    norm_then_rope(q + (n * H + hq) * D, wqd, pos[n], inv_freq, pairing, eps, D, tmp, qi);
+    int nkeys = P + i + 1;
+    for (int j = 0; j < nkeys; ++j) {
+        double dot = 0.0;
+        if (j < P) {
+            int64_t row = offsets[b] + j;
+            const uint16_t *kj = k_cache + (row * Hkv + g) * D;
+            const uint16_t *vj = v_cache + (row * Hkv + g) * D;
+            for (int d = 0; d < D; ++d) {
+                dot += qi[d] * bf16_bits_to_double(kj[d]);
+                vbuf[(int64_t)j * D + d] = bf16_bits_to_double(vj[d]);
+            }
+        } else {
+            int64_t m = (int64_t)b * C + (j - P);
+            const double *kj = khat + (m * Hkv + g) * D;
+            const uint16_t *vj = v + (m * Hkv + g) * D;
+            for (int d = 0; d < D; ++d) {
+                dot += qi[d] * kj[d];
+                vbuf[(int64_t)j * D + d] = bf16_bits_to_double(vj[d]);
+            }
+        }
+        s[j] = dot * inv_sqrt_d;
+        vr[j] = vbuf + (int64_t)j * D;
+    }
+    softmax_weighted_sum(s, nkeys, vr, D, p, out_row);
+}
+
 /* Chunked prefill against a cache prefix ([A] D2-3: a sequence's earlier tokens already
- * sit in the KV cache; [A] D1-5: the causal mask on the token index).  Sequence b holds
+ * sit in the KV cache; [A] D1-5: the causal mask on the token index).  Sequence b has
  * P_b = prefix_len[b] cached rows (k-hat and v) from row offsets[b] on, and brings a
  * chunk of C new tokens: raw q [B, C, H, D], k and v [B, C, Hkv, D] (bf16 bits), at
  * positions pos [B, C].  Chunk row i of query head hq attends to the P_b cached rows of
  * KV head hq / (H/Hkv) and to the chunk's rows 0 .. i (token indices up to P_b + i).
  * The chunk's k-hat goes to khat_out [B, C, Hkv, D] (what a caller appends to the
- * cache); out is [B, C, H, D]. */
-void oracle_prefill_chunk_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                             const uint16_t *k_cache, const uint16_t *v_cache,
-                             const int64_t *offsets, const int32_t *prefix_len, const int32_t *pos,
-                             const float *wq, const float *wk, const double *inv_freq, int pairing,
-                             double logit_mult, double eps, int B, int C, int H, int Hkv, int D,
-                             double *out, double *khat_out)
+ * cache).  With rows == NULL, out is [B, C, H, D], every row; else out is [nrows, D], the
+ * rows (b, hq, i) listed in rows [nrows, 3]. */
+static void prefill_chunk_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                               const uint16_t *k_cache, const uint16_t *v_cache,
+                               const int64_t *offsets, const int32_t *prefix_len, const int32_t *pos,
+                               const float *wq, const float *wk, const double *inv_freq, int pairing,
+                               double logit_mult, double eps, int B, int C, int H, int Hkv, int D,
+                               int64_t nrows, const int64_t *rows, double *out, double *khat_out)
 {
-    int h_per_kv = H / Hkv;
     double inv_sqrt_d = logit_mult / sqrt((double)D);
     int32_t maxkeys = 1;
     for (int b = 0; b < B; ++b)
@@ -567,6 +608,7 @@ void oracle_prefill_chunk_ex(const uint16_t *q, const uint16_t *k, const uint16_
                                khat_out + (n * Hkv + g) * D);
         free(tmp);
     }
+    int64_t count = rows ? nrows : (int64_t)B * H * C;
 #pragma omp parallel
     {
         double *tmp = (double *)malloc(sizeof(double) * D);
@@ -575,39 +617,24 @@ void oracle_prefill_chunk_ex(const uint16_t *q, const uint16_t *k, const uint16_
         double *p = (double *)malloc(sizeof(double) * maxkeys);
         double *vbuf = (double *)malloc(sizeof(double) * (size_t)maxkeys * D);
         const double **vr = (const double **)malloc(sizeof(double *) * maxkeys);
-#pragma omp for collapse(3) schedule(dynamic, 1)
-        for (int b = 0; b < B; ++b)
-            for (int hq = 0; hq < H; ++hq)
-                for (int i = 0; i < C; ++i) {
-                    int g = hq / h_per_kv;
-                    int32_t P = prefix_len[b];
-                    int64_t n = (int64_t)b * C + i;
-                    norm_then_rope(q + (n * H + hq) * D, wqd, pos[n], inv_freq, pairing, eps, D, tmp, qi);
-                    int nkeys = P + i + 1;
-                    for (int j = 0; j < nkeys; ++j) {
-                        double dot = 0.0;
-                        if (j < P) {
-                            int64_t row = offsets[b] + j;
-                            const uint16_t *kj = k_cache + (row * Hkv + g) * D;
-                            const uint16_t *vj = v_cache + (row * Hkv + g) * D;
-                            for (int d = 0; d < D; ++d) {
-                                dot += qi[d] * bf16_bits_to_double(kj[d]);
-                                vbuf[(int64_t)j * D + d] = bf16_bits_to_double(vj[d]);
-                            }
-                        } else {
-                            int64_t m = (int64_t)b * C + (j - P);
-                            const double *kj = khat_out + (m * Hkv + g) * D;
-                            const uint16_t *vj = v + (m * Hkv + g) * D;
-                            for (int d = 0; d < D; ++d) {
-                                dot += qi[d] * kj[d];
-                                vbuf[(int64_t)j * D + d] = bf16_bits_to_double(vj[d]);
-                            }
-                        }
-                        s[j] = dot * inv_sqrt_d;
-                        vr[j] = vbuf + (int64_t)j * D;
-                    }
-                    softmax_weighted_sum(s, nkeys, vr, D, p, out + (n * H + hq) * D);
-                }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < count; ++r) {
+            int b, hq, i;
+            double *dst;
+            if (rows) {
+                b = (int)rows[3 * r];
+                hq = (int)rows[3 * r + 1];
+                i = (int)rows[3 * r + 2];
+                dst = out + r * D;
+            } else {
+                b = (int)(r / ((int64_t)H * C));
+                hq = (int)(r / C % H);
+                i = (int)(r % C);
+                dst = out + (((int64_t)b * C + i) * H + hq) * D;
+            }
+            chunk_one_row(q, v, k_cache, v_cache, offsets, prefix_len, pos, wqd, inv_freq, pairing,
+                          inv_sqrt_d, eps, C, H, Hkv, D, khat_out, b, hq, i, tmp, qi, s, p, vbuf, vr, dst);
+        }
         free(tmp);
         free(qi);
         free(s);
@@ -617,6 +644,30 @@ void oracle_prefill_chunk_ex(const uint16_t *q, const uint16_t *k, const uint16_
     }
     free(wqd);
     free(wkd);
+}
+
+void oracle_prefill_chunk_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                             const uint16_t *k_cache, const uint16_t *v_cache,
+                             const int64_t *offsets, const int32_t *prefix_len, const int32_t *pos,
+                             const float *wq, const float *wk, const double *inv_freq, int pairing,
+                             double logit_mult, double eps, int B, int C, int H, int Hkv, int D,
+                             double *out, double *khat_out)
+{
+    prefill_chunk_impl(q, k, v, k_cache, v_cache, offsets, prefix_len, pos, wq, wk, inv_freq, pairing,
+                       logit_mult, eps, B, C, H, Hkv, D, 0, NULL, out, khat_out);
+}
+
+/* The rows (b, hq, i) of oracle_prefill_chunk_ex listed in rows [nrows, 3] (for checks of
+ * launches too large to compute whole); out [nrows, D], khat_out as there. */
+void oracle_prefill_chunk_rows_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                  const uint16_t *k_cache, const uint16_t *v_cache,
+                                  const int64_t *offsets, const int32_t *prefix_len, const int32_t *pos,
+                                  const float *wq, const float *wk, const double *inv_freq, int pairing,
+                                  double logit_mult, double eps, int B, int C, int H, int Hkv, int D,
+                                  int64_t nrows, const int64_t *rows, double *out, double *khat_out)
+{
+    prefill_chunk_impl(q, k, v, k_cache, v_cache, offsets, prefix_len, pos, wq, wk, inv_freq, pairing,
+                       logit_mult, eps, B, C, H, Hkv, D, nrows, rows, out, khat_out);
 }
 
 /* Variable-length packed prefill: B sequences laid end to end, sequence b owning tokens

@@ -67,6 +67,8 @@ def _load():
                                                     I, I, P, P]
             lib.oracle_prefill_chunk_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, Dd, Dd, I, I, I,
                                                     I, I, P, P]
+            lib.oracle_prefill_chunk_rows_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, Dd, Dd, I, I, I,
+                                                         I, I, L, P, P, P]
             lib.oracle_prefill_varlen_ex.argtypes = [P, P, P, P, P, P, P, P, I, Dd, Dd, I, I, I, I, P]
             lib.oracle_linear.argtypes = [P, P, L, L, L, P]
             lib.oracle_num_threads.restype = I
@@ -379,6 +381,31 @@ def prefill_chunk_ex(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, offsets
                                     _p(_c(wk, np.float32)), _p(f), rope.pair_code(), rope.logit_mult(), eps, B, C,
                                     H, Hkv, D, _p(out), _p(khat))
     return out, khat
+
+
+def prefill_chunk_rows_ex(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, offsets, prefix_len, pos, wq, wk,
+                          rope: Rope, eps: float, rows) -> np.ndarray:
+    """The rows (b, hq, i) of prefill_chunk_ex listed in rows [n, 3] (chunk row i of query
+    head hq of sequence b), for launches too large to compute whole: out [n, D], fp64."""
+    q_bits = _c(q_bits, np.uint16)
+    k_bits = _c(k_bits, np.uint16)
+    v_bits = _c(v_bits, np.uint16)
+    B, C, H, D = q_bits.shape
+    Hkv = k_bits.shape[2]
+    assert k_bits.shape == (B, C, Hkv, D) and v_bits.shape == k_bits.shape
+    pl = _c(prefix_len, np.int32)
+    assert (pl >= 0).all()
+    rows = _c(rows, np.int64).reshape(-1, 3)
+    assert (rows[:, 0] < B).all() and (rows[:, 1] < H).all() and (rows[:, 2] < C).all() and (rows >= 0).all()
+    f = rope.inv_freq(D)
+    out = np.empty((rows.shape[0], D), np.float64)
+    khat = np.empty((B, C, Hkv, D), np.float64)
+    _load().oracle_prefill_chunk_rows_ex(_p(q_bits), _p(k_bits), _p(v_bits), _p(_c(k_cache_bits, np.uint16)),
+                                         _p(_c(v_cache_bits, np.uint16)), _p(_c(offsets, np.int64)), _p(pl),
+                                         _p(_c(pos, np.int32).reshape(B, C)), _p(_c(wq, np.float32)),
+                                         _p(_c(wk, np.float32)), _p(f), rope.pair_code(), rope.logit_mult(), eps, B,
+                                         C, H, Hkv, D, rows.shape[0], _p(rows), _p(out), _p(khat))
+    return out
 
 
 def prefill_chunk_paged_ex(q_bits, k_bits, v_bits, k_pages_bits, v_pages_bits, page_table, page_size, prefix_len,

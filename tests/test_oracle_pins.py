@@ -714,6 +714,24 @@ def test_paged_chunk_equals_contiguous_chunk():
         np.testing.assert_array_equal(kgot, kref)
 
 
+def test_chunk_rows_equal_the_whole_chunk():
+    """The sampled-rows chunk oracle returns, bit for bit, the listed rows (b, hq, i) of the
+    whole-chunk oracle: every row in order, and a shuffled subset with repeats."""
+    B, P, C, H, Hkv, D = 2, 37, 9, 4, 2, 16
+    inp, kh, kc, vc, offsets = _chunk_setup(B, P, C, H, Hkv, D, seed=86)
+    args = (_bits(inp.q)[:, P:], _bits(inp.k)[:, P:], _bits(inp.v)[:, P:], _bits(kc), _bits(vc), offsets,
+            np.array([P, 5], np.int32), inp.pos.numpy()[:, P:], inp.wq.numpy(), inp.wk.numpy(),
+            oracle.Rope(theta=inp.theta, pairing="half"), inp.eps)
+    ref, _ = oracle.prefill_chunk_ex(*args)
+    every = np.array([(b, h, i) for b in range(B) for h in range(H) for i in range(C)], np.int64)
+    got = oracle.prefill_chunk_rows_ex(*args, every)
+    np.testing.assert_array_equal(got, ref[every[:, 0], every[:, 2], every[:, 1]])
+    rng = np.random.default_rng(87)
+    some = every[rng.integers(0, len(every), 25)]
+    got = oracle.prefill_chunk_rows_ex(*args, some)
+    np.testing.assert_array_equal(got, ref[some[:, 0], some[:, 2], some[:, 1]])
+
+
 def test_chunk_without_prefix_is_plain_prefill():
     B, C, H, Hkv, D = 2, 9, 4, 2, 16
     inp = synthetic.prefill_inputs(B, C, H, Hkv, D=D, seed=81)
