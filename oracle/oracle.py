@@ -386,7 +386,8 @@ def prefill_chunk_ex(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, offsets
 def prefill_chunk_rows_ex(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, offsets, prefix_len, pos, wq, wk,
                           rope: Rope, eps: float, rows) -> np.ndarray:
     """The rows (b, hq, i) of prefill_chunk_ex listed in rows [n, 3] (chunk row i of query
-    head hq of sequence b), for launches too large to compute whole: out [n, D], fp64."""
+    head hq of sequence b), for launches too large to compute whole.  Returns (out [n, D],
+    chunk k-hat [B,C,Hkv,D]), both fp64."""
     q_bits = _c(q_bits, np.uint16)
     k_bits = _c(k_bits, np.uint16)
     v_bits = _c(v_bits, np.uint16)
@@ -405,7 +406,7 @@ def prefill_chunk_rows_ex(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, of
                                          _p(_c(pos, np.int32).reshape(B, C)), _p(_c(wq, np.float32)),
                                          _p(_c(wk, np.float32)), _p(f), rope.pair_code(), rope.logit_mult(), eps, B,
                                          C, H, Hkv, D, rows.shape[0], _p(rows), _p(out), _p(khat))
-    return out
+    return out, khat
 
 
 def prefill_chunk_paged_ex(q_bits, k_bits, v_bits, k_pages_bits, v_pages_bits, page_table, page_size, prefix_len,

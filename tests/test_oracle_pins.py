@@ -724,11 +724,12 @@ def test_chunk_rows_equal_the_whole_chunk():
             oracle.Rope(theta=inp.theta, pairing="half"), inp.eps)
     ref, _ = oracle.prefill_chunk_ex(*args)
     every = np.array([(b, h, i) for b in range(B) for h in range(H) for i in range(C)], np.int64)
-    got = oracle.prefill_chunk_rows_ex(*args, every)
+    got, khat = oracle.prefill_chunk_rows_ex(*args, every)
     np.testing.assert_array_equal(got, ref[every[:, 0], every[:, 2], every[:, 1]])
+    np.testing.assert_array_equal(khat, oracle.prefill_chunk_ex(*args)[1])
     rng = np.random.default_rng(87)
     some = every[rng.integers(0, len(every), 25)]
-    got = oracle.prefill_chunk_rows_ex(*args, some)
+    got, _ = oracle.prefill_chunk_rows_ex(*args, some)
     np.testing.assert_array_equal(got, ref[some[:, 0], some[:, 2], some[:, 1]])
 
 

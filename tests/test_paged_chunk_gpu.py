@@ -83,6 +83,78 @@ def test_paged_chunk_against_oracle(gqa, prefix, chunk, H, Hkv, page_size):
     _paged_chunk_case(gqa, prefix, chunk, H, Hkv, page_size, seed=400 + page_size)
 
 
+def _pages_in_order(kc, vc, offs, caps, ps, order):
+    """Cache rows cut into pages of ps rows, handed out in the given order of page ids (a
+    permutation of the pool), sequence after sequence; two spare pages at the end."""
+    need = [(c + ps - 1) // ps for c in caps]
+    npg = sum(need) + 2
+    ids = list(order) + [i for i in range(npg) if i not in set(order)]
+    Hkv, D = kc.shape[1], kc.shape[2]
+    kp = torch.zeros(npg, ps, Hkv, D, dtype=kc.dtype)
+    vp = torch.zeros_like(kp)
+    table = torch.full((len(caps), max(need)), -1, dtype=torch.int32)
+    nxt = 0
+    for b, c in enumerate(caps):
+        o = int(offs[b])
+        for j in range(need[b]):
+            pid = ids[nxt]
+            nxt += 1
+            table[b, j] = pid
+            n = min(ps, c - j * ps)
+            kp[pid, :n] = kc[o + j * ps:o + j * ps + n]
+            vp[pid, :n] = vc[o + j * ps:o + j * ps + n]
+    return kp, vp, table
+
+
+@pytest.mark.parametrize("ps,layout", [(16, "in_order"), (32, "in_order"), (64, "in_order"), (16, "runs"),
+                                       (32, "runs"), (16, "descending")])
+def test_paged_chunk_page_layouts(gqa, ps, layout):
+    """Page layouts other than a random shuffle: pages in order, runs of 8 consecutive pages
+    in shuffled order (tiles straddle runs at some prefixes and not at others), and pages in
+    descending order.  Outputs bit for bit equal to the contiguous chunk's and within
+    tolerance of the oracle; the chunk's rows land in the right pages."""
+    prefix, chunk, H, Hkv = [500, 0, 1000], [300, 129, 77], 16, 4
+    q, k, v, _, cu, wq, wk, theta, eps = _packed(chunk, H, Hkv, seed=520 + ps)
+    pos = torch.cat([torch.arange(p, p + c, dtype=torch.int32) for p, c in zip(prefix, chunk)])
+    kc, vc, offs = _cache_with_prefix(prefix, chunk, Hkv, wk, theta, eps, {}, seed=521 + ps)
+    caps = [p + c for p, c in zip(prefix, chunk)]
+    npg = sum((c + ps - 1) // ps for c in caps)
+    if layout == "in_order":
+        order = list(range(npg))
+    elif layout == "descending":
+        order = list(range(npg - 1, -1, -1))
+    else:
+        runs = [list(range(r, min(r + 8, npg))) for r in range(0, npg, 8)]
+        rng = np.random.default_rng(522)
+        order = [i for r in rng.permutation(len(runs)) for i in runs[r]]
+    kp, vp, table = _pages_in_order(kc, vc, offs, caps, ps, order)
+    pl = torch.tensor(prefix, dtype=torch.int32)
+    rope = gqa.RopeConfig.make(theta=theta)
+    dev = [t.cuda() for t in (q, k, v, pos, cu)]
+    kpd, vpd = kp.cuda(), vp.cuda()
+    out = gqa.prefill_chunk_paged(*dev, kpd, vpd, table.cuda(), pl.cuda(), wq.cuda(), wk.cuda(),
+                                  max_chunk_len=max(chunk), eps=eps, rope=rope)
+    kcd, vcd = kc.cuda(), vc.cuda()
+    flat = gqa.prefill_chunk(*dev, kcd, vcd, offs.cuda(), pl.cuda(), wq.cuda(), wk.cuda(), max_chunk_len=max(chunk),
+                             eps=eps, rope=rope)
+    torch.cuda.synchronize()
+    gqa.check_device_status()
+    assert torch.equal(out.cpu(), flat.cpu()), f"paged ({layout}, {ps}-row pages) and contiguous chunk differ"
+    kpd, vpd, kcd, vcd = kpd.cpu(), vpd.cpu(), kcd.cpu(), vcd.cpu()
+    t = table.numpy()
+    for b, (p, c) in enumerate(zip(prefix, chunk)):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        r = np.arange(p, p + c)
+        pg = t[b, r // ps].astype(np.int64)
+        o = int(offs[b])
+        assert torch.equal(kpd[pg, r % ps], kcd[o + p:o + p + c]) and torch.equal(vpd[pg, r % ps], vcd[o + p:o + p + c])
+        ref, _ = oracle.prefill_chunk_paged_ex(
+            bits(q[lo:hi]).reshape(1, c, H, 128), bits(k[lo:hi]).reshape(1, c, Hkv, 128),
+            bits(v[lo:hi]).reshape(1, c, Hkv, 128), bits(kp), bits(vp), t[b:b + 1], ps, np.array([p], np.int32),
+            pos[lo:hi].numpy().reshape(1, c), wq.numpy(), wk.numpy(), oracle.Rope(theta=theta), eps)
+        assert_close(out.cpu().numpy()[lo:hi], ref[0], f"{layout} {ps}-row pages, sequence {b}")
+
+
 def test_paged_chunk_with_rope_variant(gqa):
     _paged_chunk_case(gqa, [333, 90], [200, 130], 16, 4, 32, seed=460,
                       rope_kw=dict(pairing="half", scaling="yarn", factor=4.0, original_max_position=256))
